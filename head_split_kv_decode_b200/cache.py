@@ -1,0 +1,148 @@
+"""PyTorch-facing wrapper of the C ABI: allocates the cache and workspace as
+torch tensors, checks tensor arguments and forwards to :mod:`.binding`.
+
+PyTorch is used for device memory and streams only; every byte of K/V/Q/O is
+read and written by the library's kernels.
+"""
+
+import torch
+
+from . import binding as B
+
+_TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "int4": torch.bfloat16}
+_ALIGN = 256
+
+
+def _aligned_buffer(nbytes, device, zero):
+    buf = (torch.zeros if zero else torch.empty)(nbytes + _ALIGN, dtype=torch.uint8, device=device)
+    base = buf.data_ptr()
+    off = (-base) % _ALIGN
+    return buf, off
+
+
+def _stream_handle(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+class DuoCache:
+    """A head-split KV cache for ``layers`` layers bound to torch-allocated memory.
+
+    head_mask: [layers, n_kv_heads] of 0/1 (1 = retrieval head).
+    kv_dtype: "f32", "bf16" or "int4" (K/V given in bf16 and quantised on append).
+    """
+
+    def __init__(self, layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype, capacity,
+                 head_mask, S, R, device="cuda"):
+        mask = torch.as_tensor(head_mask).reshape(-1).to(torch.uint8).tolist()
+        self.handle = B.duo_cache_create(layers, batch, n_q_heads, n_kv_heads, head_dim,
+                                         kv_dtype, capacity, mask, S, R)
+        self.layers, self.batch = layers, batch
+        self.n_q_heads, self.n_kv_heads, self.head_dim = n_q_heads, n_kv_heads, head_dim
+        self.kv_dtype, self.capacity, self.S, self.R = kv_dtype, capacity, S, R
+        self.io_dtype = _TORCH_DTYPE[kv_dtype]
+        self.device = torch.device(device)
+        if self.device.type == "cuda" and self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        self.cache_bytes, self.ws_bytes = B.duo_cache_required_bytes(self.handle)
+        self._storage, off = _aligned_buffer(self.cache_bytes, self.device, zero=False)
+        self.base_ptr = self._storage.data_ptr() + off
+        self.storage = self._storage[off:off + self.cache_bytes]
+        B.duo_cache_bind(self.handle, self.base_ptr, self.cache_bytes)
+        self._ws, woff = _aligned_buffer(self.ws_bytes, self.device, zero=True)
+        self.ws_ptr = self._ws.data_ptr() + woff
+
+    # ------------------------------------------------------------ checks
+    def _check(self, t, shape, name, dtype=None):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError("%s must be a torch tensor" % name)
+        if t.device != self.device:
+            raise ValueError("%s is on %s, cache on %s" % (name, t.device, self.device))
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+        if t.dtype != (dtype or self.io_dtype):
+            raise ValueError("%s has dtype %s, expected %s" % (name, t.dtype, dtype or self.io_dtype))
+        if not t.is_contiguous():
+            raise ValueError("%s must be contiguous" % name)
+
+    # ------------------------------------------------------------ calls
+    def append(self, layer, k, v, stream=None):
+        """k, v: [batch, n_tokens, n_kv_heads, head_dim]."""
+        n = k.shape[1]
+        shape = (self.batch, n, self.n_kv_heads, self.head_dim)
+        self._check(k, shape, "k")
+        self._check(v, shape, "v")
+        B.duo_append_kv(self.handle, layer, k.data_ptr(), v.data_ptr(), n,
+                        _stream_handle(stream, self.device))
+
+    def decode(self, layer, q, out=None, scale=0.0, stream=None):
+        """q: [batch, n_q_heads, head_dim] at position seq_len-1.  Returns out."""
+        shape = (self.batch, self.n_q_heads, self.head_dim)
+        self._check(q, shape, "q")
+        if out is None:
+            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
+        self._check(out, shape, "out")
+        B.duo_decode_attn(self.handle, layer, q.data_ptr(), out.data_ptr(), float(scale),
+                          self.ws_ptr, self.ws_bytes, _stream_handle(stream, self.device))
+        return out
+
+    def prefill(self, layer, q, k, v, out=None, scale=0.0, stream=None):
+        """q: [batch, C, n_q_heads, d]; k, v: [batch, C, n_kv_heads, d].  Attends only."""
+        C = q.shape[1]
+        self._check(q, (self.batch, C, self.n_q_heads, self.head_dim), "q")
+        self._check(k, (self.batch, C, self.n_kv_heads, self.head_dim), "k")
+        self._check(v, (self.batch, C, self.n_kv_heads, self.head_dim), "v")
+        if out is None:
+            out = torch.empty_like(q)
+        self._check(out, tuple(q.shape), "out")
+        B.duo_prefill_attn(self.handle, layer, q.data_ptr(), k.data_ptr(), v.data_ptr(), C,
+                           out.data_ptr(), float(scale), None, 0,
+                           _stream_handle(stream, self.device))
+        return out
+
+    # ------------------------------------------------------------ introspection
+    def seq_len(self, layer):
+        return B.duo_seq_len(self.handle, layer)
+
+    def kv_bytes(self):
+        return B.duo_kv_bytes(self.handle)
+
+    def layout(self, layer):
+        return B.duo_layout_info(self.handle, layer)
+
+    def set_decode_splits(self, splits):
+        B.duo_set_decode_splits(self.handle, splits)
+
+    def decode_splits(self, layer):
+        return B.duo_decode_splits(self.handle, layer)
+
+    def reset(self):
+        B.duo_cache_reset(self.handle)
+
+    def region(self, layer, name):
+        """Raw view of one buffer of one layer (for inspection and tests).
+
+        name in ret_k, ret_v, str_k, str_v (rows of K/V elements or int4 codes) and,
+        for int4, ret_k_sz, ret_v_sz, str_k_sz, str_v_sz (fp16 scale/zero pairs).
+        Returns a uint8 tensor [batch, heads, rows, row_bytes] (or [..., 4]).
+        """
+        lv = self.layout(layer)
+        off = getattr(lv, name)
+        if off < 0:
+            return None
+        heads = lv.n_retrieval if name.startswith("ret") else lv.n_streaming
+        rows = lv.capacity if name.startswith("ret") else lv.window
+        width = 4 if name.endswith("_sz") else lv.row_bytes
+        nbytes = self.batch * heads * rows * width
+        return self.storage[off:off + nbytes].view(self.batch, heads, rows, width)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            B.duo_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,153 @@
+// Cache append/evict: write the K/V of new tokens into the two layouts.
+//
+// Retrieval KV heads keep every token (full KV cache); streaming KV heads keep
+// S sink slots and an R-slot ring of the most recent tokens, so writing a
+// token into its ring slot evicts the token R positions older.  Pages:
+// "What is DuoAttention" (nav.superapi.store), section "Technical principles of
+// DuoAttention"; "DuoAttention: Efficient Long-Context LLM Inference with
+// Retrieval and Streaming Heads" (hotpaper.ai), section "기술적 접근법".
+//
+// For a chunk of n_tok tokens a streaming head writes only the positions that
+// survive the chunk: p < S (sinks) and the last R positions.  Those land in
+// distinct slots, so the result equals appending token by token.
+#include "common.cuh"
+
+namespace duo {
+
+// One thread per 16-byte chunk of one (token, KV head) row of K and of V.
+__global__ void append_kernel(const __grid_constant__ AppendParams a, int row_bytes) {
+  const int ch = row_bytes / 16;
+  const int64_t total = (int64_t)a.B * a.n_tok * a.Hkv * ch;
+  const int64_t end = a.n_cur + a.n_tok;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % ch);
+    int64_t r = i / ch;
+    const int h = (int)(r % a.Hkv);
+    r /= a.Hkv;
+    const int64_t t = r % a.n_tok;
+    const int b = (int)(r / a.n_tok);
+    const int64_t p = a.n_cur + t;
+    const int idx = a.h.index[h];
+    int64_t off;
+    uint8_t *dk, *dv;
+    if (a.h.kind[h]) {
+      off = (((int64_t)b * a.n_ret + idx) * a.cap + p) * row_bytes;
+      dk = a.p.ret_k;
+      dv = a.p.ret_v;
+    } else {
+      if (!(p < a.S || p >= end - a.R)) continue;
+      const int64_t slot = p < a.S ? p : a.S + (p - a.S) % a.R;
+      off = (((int64_t)b * a.n_str + idx) * a.W + slot) * row_bytes;
+      dk = a.p.str_k;
+      dv = a.p.str_v;
+    }
+    // The input is [B][n_tok][Hkv][row], so chunk i of the input is chunk i.
+    const uint4 kk = __ldg(reinterpret_cast<const uint4 *>(a.k) + i);
+    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(a.v) + i);
+    reinterpret_cast<uint4 *>(dk + off)[c] = kk;
+    reinterpret_cast<uint4 *>(dv + off)[c] = vv;
+  }
+}
+
+// INT4: one warp per (token, KV head, K or V) row of D bf16 channels.  Lane l
+// owns channels [l*CPL, l*CPL + CPL).  The encoder performs, in this order,
+// correctly rounded fp32 operations:
+//   span = mx - mn; sc = fp16(span / 15); zp = fp16(mn);
+//   u = clamp(rint((x - zp) / sc), 0, 15), u = 0 when sc == 0.
+template <int D>
+__global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
+  constexpr int CPL = D / 32;
+  static_assert(CPL == 2 || CPL == 4, "head_dim 64 or 128");
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)a.B * a.n_tok * a.Hkv * 2;
+  const int64_t end = a.n_cur + a.n_tok;
+  const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t w = gw; w < warps; w += nw) {
+    const int which = (int)(w & 1);  // 0 = K, 1 = V
+    int64_t r = w >> 1;
+    const int h = (int)(r % a.Hkv);
+    r /= a.Hkv;
+    const int64_t t = r % a.n_tok;
+    const int b = (int)(r / a.n_tok);
+    const int64_t p = a.n_cur + t;
+    const int idx = a.h.index[h];
+    int64_t row;
+    uint8_t *codes, *sz;
+    if (a.h.kind[h]) {
+      row = ((int64_t)b * a.n_ret + idx) * a.cap + p;
+      codes = which ? a.p.ret_v : a.p.ret_k;
+      sz = which ? a.p.ret_v_sz : a.p.ret_k_sz;
+    } else {
+      if (!(p < a.S || p >= end - a.R)) continue;
+      const int64_t slot = p < a.S ? p : a.S + (p - a.S) % a.R;
+      row = ((int64_t)b * a.n_str + idx) * a.W + slot;
+      codes = which ? a.p.str_v : a.p.str_k;
+      sz = which ? a.p.str_v_sz : a.p.str_k_sz;
+    }
+    const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(which ? a.v : a.k) +
+                               (((int64_t)b * a.n_tok + t) * a.Hkv + h) * D + lane * CPL;
+    float x[CPL];
+    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+      x[j] = __bfloat162float(src[j]);
+      mn = fminf(mn, x[j]);
+      mx = fmaxf(mx, x[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const __half sch = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+    const __half zph = __float2half_rn(mn);
+    const float scf = __half2float(sch);
+    const float zpf = __half2float(zph);
+    uint32_t u[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+      float q = 0.0f;
+      if (scf != 0.0f) q = fminf(15.0f, fmaxf(0.0f, rintf(__fdiv_rn(__fsub_rn(x[j], zpf), scf))));
+      u[j] = (uint32_t)q;
+    }
+    uint8_t *dst = codes + row * (D / 2) + lane * (CPL / 2);
+    if (CPL == 4) {
+      const uint16_t packed = (uint16_t)(u[0] | (u[1] << 4) | (u[2] << 8) | (u[3] << 12));
+      *reinterpret_cast<uint16_t *>(dst) = packed;
+    } else {
+      *dst = (uint8_t)(u[0] | (u[1] << 4));
+    }
+    if (lane == 0) {
+      __half2 pair;
+      pair.x = sch;
+      pair.y = zph;
+      reinterpret_cast<__half2 *>(sz)[row] = pair;
+    }
+  }
+}
+
+cudaError_t launch_append(const AppendParams &a, int kv_type, cudaStream_t s) {
+  if (a.n_tok <= 0) return cudaSuccess;
+  if (kv_type == kINT4) {
+    const int64_t warps = (int64_t)a.B * a.n_tok * a.Hkv * 2;
+    const int threads = 256;
+    const int64_t blocks = (warps * 32 + threads - 1) / threads;
+    const int grid = (int)(blocks < 148 * 64 ? blocks : 148 * 64);
+    if (a.D == 128)
+      append_int4_kernel<128><<<grid, threads, 0, s>>>(a);
+    else
+      append_int4_kernel<64><<<grid, threads, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  const int row_bytes = a.D * (kv_type == kF32 ? 4 : 2);
+  const int64_t total = (int64_t)a.B * a.n_tok * a.Hkv * (row_bytes / 16);
+  const int threads = 256;
+  const int64_t blocks = (total + threads - 1) / threads;
+  const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
+  append_kernel<<<grid, threads, 0, s>>>(a, row_bytes);
+  return cudaGetLastError();
+}
+
+}  // namespace duo

@@ -181,3 +181,57 @@ WORKLOADS = {
         "int4", 32, 1, 32, 8, 128, 1048576, 64, 256, 0.25, steps=64,
         outlier_frac=0.01, outlier_mult=10.0),
 }
+
+
+# ---------------------------------------------------------------- materialisers
+#
+# One consistent stream per (workload, layer, K or V): the K/V of position p is
+# the same whether it is part of the pre-filled context or appended by a decode
+# step, and the query of a decode step sits at the position of the token that
+# step appends.
+
+
+def history(w, layer, which, batch_ids, positions, heads=None, device="cpu", mask_row=None):
+    """K (which="k") or V (which="v") values, float32
+    [len(batch_ids), len(positions), len(heads), d], with the workload's planted
+    structure: scale, outlier channels, and (K only) one needle key per
+    retrieval head placed at a seeded position in [S, context - R)."""
+    heads = list(range(w.n_kv_heads)) if heads is None else list(heads)
+    tid = T_K if which == "k" else T_V
+    x = kv_field(layer_seed(w.wid, layer, tid), batch_ids, positions, w.n_kv_heads,
+                 w.head_dim, heads=heads, device=device)
+    if w.kv_scale != 1.0:
+        x = x * w.kv_scale
+    if w.outlier_frac > 0:
+        for j, h in enumerate(heads):
+            ch = outlier_channels(layer_seed(w.wid, layer, T_OUTLIER) * 128 + h, w.head_dim,
+                                  w.outlier_frac).to(device)
+            x[:, :, j, ch] = x[:, :, j, ch] * w.outlier_mult
+    if which == "k" and w.needle_sigma > 0 and mask_row is not None:
+        pos_t = torch.as_tensor(positions)
+        for j, h in enumerate(heads):
+            if not int(mask_row[h]):
+                continue
+            for bi, b in enumerate(batch_ids):
+                p = needle_position(layer_seed(w.wid, layer, T_NEEDLE) * 4096 + int(b) * 64 + h,
+                                    w.S, w.context - w.R)
+                hit = (pos_t == p).nonzero()
+                if len(hit):
+                    q0 = queries(w, layer, [b], [w.context], heads=[h * w.group])[0, 0, 0]
+                    x[bi, int(hit[0]), j] = needle_key(q0, w.needle_sigma, w.kv_scale).to(device)
+    return x
+
+
+def queries(w, layer, batch_ids, positions, heads=None, device="cpu"):
+    """Query values float32 [len(batch_ids), len(positions), len(heads), d]."""
+    return kv_field(layer_seed(w.wid, layer, T_Q), batch_ids, positions, w.n_q_heads,
+                    w.head_dim, heads=heads, device=device)
+
+
+def workload_mask(w):
+    """The workload's retrieval-head mask, uint8 [layers, n_kv_heads]."""
+    return head_mask(layer_seed(w.wid, 0, T_MASK), w.layers, w.n_kv_heads, w.retrieval_frac)
+
+
+def io_dtype(w):
+    return torch.float32 if w.kv_dtype == "f32" else torch.bfloat16

@@ -1,0 +1,200 @@
+/*
+ * duo.h -- C ABI of libduo: attention over a head-split KV cache
+ * (DuoAttention: retrieval heads with a full KV cache, streaming heads with a
+ * constant-length cache of attention sinks plus recent tokens), for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources (pages; the method is stated in prose only):
+ *  - "DuoAttention: Efficient Long-Context LLM Inference with Retrieval and
+ *    Streaming Heads" (hotpaper.ai), abstract: retrieval heads need full
+ *    attention over all tokens; streaming heads attend to recent tokens and
+ *    attention sinks through a light-weight constant-length KV cache; this
+ *    cuts both decoding and pre-filling cost.  Same page, section
+ *    "기술적 접근법" (technical approach): two KV caches per layer; MHA and GQA;
+ *    compatible with a 4-bit KV cache.
+ *  - "What is DuoAttention" (nav.superapi.store), section "Technical
+ *    principles of DuoAttention": full KV cache for retrieval heads,
+ *    fixed-length KV cache for streaming heads.
+ *  - "韩松团队长上下文LLM推理高效框架" (cn.bg3.co), section "研究背景": decoding
+ *    cost grows linearly and pre-filling cost quadratically with the context.
+ *
+ * Definitions used by every call (readings where the pages are silent):
+ *  - Query head h uses KV head h / G, G = n_q_heads / n_kv_heads.  One mask bit
+ *    per KV head: 1 = retrieval, 0 = streaming.
+ *  - A query at absolute position i sees key j iff j <= i and, for a streaming
+ *    head, (j < S or i - j < R).  Softmax scale defaults to 1/sqrt(head_dim).
+ *  - Streaming slot of position p: p if p < S, else S + ((p - S) mod R).
+ *  - Q and K arrive post-RoPE; the library does no position arithmetic.
+ *
+ * Conventions:
+ *  - The caller owns all device memory: the cache storage (bound once with
+ *    duo_cache_bind), Q/K/V/O and workspaces.  The handle owns host metadata.
+ *  - Tensors are dense, row-major, in device memory:
+ *      decode  q, out   [batch, n_q_heads, head_dim]
+ *      append  k, v     [batch, n_tokens, n_kv_heads, head_dim]
+ *      prefill q, out   [batch, C, n_q_heads, head_dim]; k, v [batch, C, n_kv_heads, head_dim]
+ *    Element type: float32 for a DUO_F32 cache; bfloat16 for DUO_BF16 and for
+ *    the K/V/Q/O of a DUO_INT4 cache (K/V are quantised on append).
+ *  - Every call with a stream is asynchronous on that stream.  Argument,
+ *    capacity and layout errors are detected on the host and returned before
+ *    anything is enqueued; a failed launch returns DUO_ERR_CUDA.  Nothing
+ *    throws across this boundary.  Calls on one cache must be ordered by the
+ *    caller (one stream, or events).
+ *  - Ordering: decode is append-then-attend (duo_append_kv with one token, then
+ *    duo_decode_attn; the new token sees itself).  Pre-fill is
+ *    attend-then-append (duo_prefill_attn reads the cache as it stood before
+ *    the chunk plus the chunk's own K/V; the caller then appends the chunk).
+ */
+#ifndef DUO_H
+#define DUO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DUO_MAX_KV_HEADS 64
+#define DUO_MAX_SPLITS 512
+
+typedef struct CUstream_st *duo_stream; /* a cudaStream_t; NULL = legacy stream */
+
+typedef enum duo_status {
+  DUO_OK = 0,
+  DUO_ERR_ARG = 1,         /* null pointer, bad size, bad layer, misaligned pointer */
+  DUO_ERR_CAPACITY = 2,    /* an append would overflow a retrieval page */
+  DUO_ERR_LAYOUT = 3,      /* head mask / head counts inconsistent */
+  DUO_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+  DUO_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  DUO_ERR_TIMEOUT = 6,     /* a bounded in-kernel wait gave up (see duo_poll_device_error) */
+  DUO_ERR_UNSUPPORTED = 7, /* valid request this build does not implement */
+  DUO_ERR_STATE = 8        /* cache not bound, or call out of order */
+} duo_status;
+
+typedef enum duo_kv_dtype { DUO_F32 = 0, DUO_BF16 = 1, DUO_INT4 = 2 } duo_kv_dtype;
+
+typedef enum duo_layout {
+  /* Retrieval KV heads: one contiguous [capacity, d] page each for K and V.
+   * Streaming KV heads: one [S + R, d] slot buffer each for K and V. */
+  DUO_LAYOUT_PACKED = 0
+} duo_layout;
+
+typedef struct duo_cache_desc {
+  int32_t layers;
+  int32_t batch;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;  /* <= DUO_MAX_KV_HEADS, divides n_q_heads */
+  int32_t head_dim;    /* 64 or 128 */
+  int32_t kv_dtype;    /* duo_kv_dtype */
+  int64_t capacity;    /* max tokens a retrieval page holds */
+} duo_cache_desc;
+
+typedef struct duo_cache duo_cache;
+
+/* Where one layer's buffers live inside the bound device memory.  Offsets are
+ * in bytes from the bound base pointer; -1 where a buffer does not exist. */
+typedef struct duo_layout_view {
+  int32_t n_retrieval;   /* retrieval KV heads in this layer */
+  int32_t n_streaming;   /* streaming KV heads in this layer */
+  int32_t window;        /* S + R */
+  int32_t row_bytes;     /* bytes of one token of one head: d*4 (f32), d*2 (bf16), d/2 (int4 codes) */
+  int64_t capacity;
+  int64_t seq_len;       /* tokens appended so far */
+  int64_t ret_k, ret_v;  /* [batch][n_retrieval][capacity][row] */
+  int64_t str_k, str_v;  /* [batch][n_streaming][window][row] */
+  int64_t ret_k_sz, ret_v_sz, str_k_sz, str_v_sz; /* int4 only: fp16 (scale, zero) per token, same indexing */
+  int32_t kind[DUO_MAX_KV_HEADS];         /* 1 retrieval, 0 streaming, per KV head */
+  int32_t packed_index[DUO_MAX_KV_HEADS]; /* index among heads of the same kind */
+} duo_layout_view;
+
+/* Create a cache description.  head_mask: host array [layers][n_kv_heads] of
+ * 0/1 (1 = retrieval).  S >= 0 sinks, R >= 1 recent slots.  layout must be
+ * DUO_LAYOUT_PACKED.  No device memory is touched.
+ * Errors: DUO_ERR_ARG (null/out-of-range), DUO_ERR_LAYOUT (heads inconsistent). */
+duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc,
+                            const uint8_t *head_mask, int32_t S, int32_t R,
+                            int32_t layout);
+
+void duo_cache_destroy(duo_cache *cache);
+
+/* Bytes of device memory the cache needs (cache_bytes), and the decode
+ * workspace size that covers every layer and split count (workspace_bytes). */
+duo_status duo_cache_required_bytes(const duo_cache *cache, size_t *cache_bytes,
+                                    size_t *workspace_bytes);
+
+/* Bind caller-owned device memory (256-byte aligned, >= cache_bytes).  The
+ * memory is zero-filled synchronously and every layer's length reset to 0. */
+duo_status duo_cache_bind(duo_cache *cache, void *device_mem, size_t bytes);
+
+/* Reset every layer's length to 0 without touching device memory. */
+duo_status duo_cache_reset(duo_cache *cache);
+
+/* Append n_tokens tokens (positions seq_len .. seq_len+n_tokens-1) of K and V
+ * to one layer: retrieval heads write page rows, streaming heads write only the
+ * positions that survive the chunk (sinks and the last R positions) into their
+ * slots, evicting what was there.  INT4 caches quantise each (token, head) row
+ * of head_dim channels (asymmetric min/max, fp16 scale and zero, 4-bit codes,
+ * low nibble = even channel).  Advances the layer length by n_tokens.
+ * Errors: DUO_ERR_CAPACITY if seq_len + n_tokens > capacity. */
+duo_status duo_append_kv(duo_cache *cache, int32_t layer, const void *k,
+                         const void *v, int32_t n_tokens, duo_stream stream);
+
+/* Single-token decode attention for one layer: the query at position
+ * seq_len-1 of every query head attends to its KV head's visible set.
+ * Retrieval heads run split-K flash decoding (per-split log-sum-exp partials
+ * in the workspace, merged by the last split of each head); streaming heads
+ * run one pass over their slot buffer.  softmax_scale <= 0 means 1/sqrt(d).
+ * The workspace must be zero-filled before its first use with any cache; each
+ * call leaves its counters at zero again.  Workspace size: from
+ * duo_cache_required_bytes.  Errors: DUO_ERR_STATE if the layer is empty. */
+duo_status duo_decode_attn(duo_cache *cache, int32_t layer, const void *q,
+                           void *out, float softmax_scale, void *workspace,
+                           size_t workspace_bytes, duo_stream stream);
+
+/* Chunked pre-fill attention for one layer: C queries at positions
+ * seq_len .. seq_len+C-1 attend to the cache as it stands (positions below
+ * seq_len) plus the chunk's own k/v: causal for retrieval heads, Lambda mask
+ * (sinks plus the R most recent positions) for streaming heads, with key tiles
+ * outside the Lambda band skipped.  Runs on the sm_100a tensor cores
+ * (tcgen05.mma, accumulators in tensor memory, operands loaded by TMA).  Does
+ * not append; call duo_append_kv with the same k/v afterwards.  Requires a
+ * DUO_BF16 cache with head_dim 128 (other cases: DUO_ERR_UNSUPPORTED).  The
+ * workspace argument is unused (pass NULL, 0). */
+duo_status duo_prefill_attn(duo_cache *cache, int32_t layer, const void *q,
+                            const void *k, const void *v, int32_t C, void *out,
+                            float softmax_scale, void *workspace,
+                            size_t workspace_bytes, duo_stream stream);
+
+duo_status duo_seq_len(const duo_cache *cache, int32_t layer, int64_t *n);
+
+/* KV bytes held now (kept) and what a full cache of every head would hold
+ * (full_equivalent): kept = sum over layers, batch, KV heads of
+ * (retrieval ? n : min(n, S+R)) * bytes_per_token_per_head. */
+duo_status duo_kv_bytes(const duo_cache *cache, int64_t *kept,
+                        int64_t *full_equivalent);
+
+duo_status duo_layout_info(const duo_cache *cache, int32_t layer,
+                           duo_layout_view *out);
+
+/* Force the split count of retrieval decode (1..DUO_MAX_SPLITS), or 0 for the
+ * automatic choice (enough splits to fill every SM once).  The result never
+ * depends on it beyond rounding. */
+duo_status duo_set_decode_splits(duo_cache *cache, int32_t splits);
+
+/* Split count the next decode of this layer will use. */
+duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
+                             int32_t *splits);
+
+/* Read and clear the device-side error word that bounded in-kernel waits set
+ * when they give up.  Synchronises the device.  Returns DUO_ERR_TIMEOUT if it
+ * was set, DUO_OK otherwise; *code (may be NULL) receives the raw word. */
+duo_status duo_poll_device_error(int32_t *code);
+
+const char *duo_status_string(duo_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUO_H */

@@ -1,0 +1,44 @@
+"""Shared test helpers: tolerances and seeded case builders.
+
+The tolerances are the parity bar for this library (fixed before any kernel
+existed): fp32 max |err| <= 1e-5; bf16 max |err| <= 2e-2 and mean |err| <= 2e-3;
+INT4 (against an oracle fed the identically dequantised K/V) max |err| <= 2e-2;
+cache contents and INT4 codes bit-exact.
+"""
+
+import numpy as np
+import torch
+
+TOL = {
+    "f32": dict(max=1e-5, mean=None),
+    "bf16": dict(max=2e-2, mean=2e-3),
+    "int4": dict(max=2e-2, mean=None),
+}
+
+
+def parity_errors(got, ref):
+    g = got.detach().to("cpu", torch.float64).numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    err = np.abs(g - r)
+    return float(err.max()), float(err.mean())
+
+
+def assert_parity(got, ref, kind, what=""):
+    mx, mean = parity_errors(got, ref)
+    tol = TOL[kind]
+    assert np.isfinite(mx), "%s: non-finite output" % what
+    assert mx <= tol["max"], "%s: max |err| %.3g > %.3g" % (what, mx, tol["max"])
+    if tol["mean"] is not None:
+        assert mean <= tol["mean"], "%s: mean |err| %.3g > %.3g" % (what, mean, tol["mean"])
+    return mx, mean
+
+
+def seeded_mask(seed, n_kv, n_ret):
+    g = torch.Generator().manual_seed(seed)
+    m = torch.zeros(n_kv, dtype=torch.uint8)
+    m[torch.randperm(n_kv, generator=g)[:n_ret]] = 1
+    return m
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()

@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and loads,
+it exports every function ``include/duo.h`` declares, and the host logic
+(argument checks, layout planning, byte accounting) behaves."""
+
+import os
+import re
+
+import pytest
+
+from head_split_kv_decode_b200 import binding as B
+from head_split_kv_decode_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.lib()
+
+
+def declared_functions():
+    names = []
+    for hdr in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not hdr.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(duo_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in B.SIGNATURES, "binding lacks %s" % n
+
+
+def _create(**kw):
+    args = dict(layers=2, batch=2, n_q_heads=8, n_kv_heads=4, head_dim=128, kv_dtype="bf16",
+                capacity=1000, head_mask=[1, 0, 0, 1, 0, 0, 0, 0], S=4, R=60)
+    args.update(kw)
+    return B.duo_cache_create(**args)
+
+
+def test_create_and_layout(lib):
+    h = _create()
+    try:
+        cb, wb = B.duo_cache_required_bytes(h)
+        v0 = B.duo_layout_info(h, 0)
+        v1 = B.duo_layout_info(h, 1)
+        assert (v0.n_retrieval, v0.n_streaming) == (2, 2)
+        assert (v1.n_retrieval, v1.n_streaming) == (0, 4)
+        assert v0.window == 64 and v0.row_bytes == 256 and v0.capacity == 1000
+        assert list(v0.kind)[:4] == [1, 0, 0, 1]
+        assert list(v0.packed_index)[:4] == [0, 0, 1, 1]
+        assert v1.ret_k == -1 and v1.ret_v == -1
+        assert v0.ret_k_sz == -1  # bf16 has no scale/zero buffers
+        regions = [(v0.ret_k, 2 * 2 * 1000 * 256), (v0.ret_v, 2 * 2 * 1000 * 256),
+                   (v0.str_k, 2 * 2 * 64 * 256), (v0.str_v, 2 * 2 * 64 * 256),
+                   (v1.str_k, 2 * 4 * 64 * 256), (v1.str_v, 2 * 4 * 64 * 256)]
+        for off, size in regions:
+            assert off % 256 == 0
+        regions.sort()
+        for (a, sa), (b, _) in zip(regions, regions[1:]):
+            assert a + sa <= b, "regions overlap"
+        assert regions[-1][0] + regions[-1][1] <= cb
+        assert wb > 0
+        assert B.duo_kv_bytes(h) == (0, 0)
+        assert B.duo_seq_len(h, 1) == 0
+    finally:
+        B.duo_cache_destroy(h)
+
+
+def test_int4_layout_has_scale_zero(lib):
+    h = _create(kv_dtype="int4")
+    try:
+        v = B.duo_layout_info(h, 0)
+        assert v.row_bytes == 64
+        assert min(v.ret_k_sz, v.ret_v_sz, v.str_k_sz, v.str_v_sz) >= 0
+    finally:
+        B.duo_cache_destroy(h)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(n_kv_heads=3, head_mask=[1, 0, 0, 0, 1, 0]),  # does not divide n_q_heads
+    dict(head_dim=96),
+    dict(capacity=0),
+    dict(R=0),
+    dict(S=-1),
+    dict(kv_dtype=7),
+    dict(head_mask=[2, 0, 0, 0, 0, 0, 0, 0]),
+    dict(n_kv_heads=80, n_q_heads=80, head_mask=[0] * 160),
+])
+def test_create_rejects_bad_arguments(lib, bad):
+    with pytest.raises(B.DuoError) as e:
+        _create(**bad)
+    assert e.value.name in ("DUO_ERR_ARG", "DUO_ERR_LAYOUT")
+
+
+def test_mask_length_checked_in_binding(lib):
+    with pytest.raises(ValueError):
+        _create(head_mask=[1, 0, 0])
+
+
+def test_calls_before_bind_fail_cleanly(lib):
+    h = _create()
+    try:
+        with pytest.raises(B.DuoError) as e:
+            B.duo_append_kv(h, 0, 16, 16, 1)
+        assert e.value.name == "DUO_ERR_STATE"
+        with pytest.raises(B.DuoError) as e:
+            B.duo_decode_attn(h, 0, 16, 16, 0.0, None, 0)
+        assert e.value.name == "DUO_ERR_STATE"
+        with pytest.raises(B.DuoError) as e:
+            B.duo_append_kv(h, 5, 16, 16, 1)
+        assert e.value.name == "DUO_ERR_ARG"
+        with pytest.raises(B.DuoError):
+            B.duo_set_decode_splits(h, B.MAX_SPLITS + 1)
+        B.duo_set_decode_splits(h, 7)
+        B.duo_set_decode_splits(h, 0)
+    finally:
+        B.duo_cache_destroy(h)
+
+
+def test_status_strings(lib):
+    for s in range(9):
+        assert B.duo_status_string(s)
+    assert "unknown" in B.duo_status_string(99)
