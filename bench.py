@@ -1,0 +1,584 @@
+#!/usr/bin/env python
+"""Benchmark of attention over a head-split KV cache on B200.
+
+Default workload: Llama-3-8B-shaped GQA decode at 128K context (32 layers,
+32 query / 8 KV heads, head_dim 128, bf16, 50% retrieval KV heads, S=64 sinks +
+R=256 recent), batch 1.  One step = one decode token through all 32 layers:
+append the token's K/V (append/evict kernel) then attend (split-K retrieval +
+streaming + log-sum-exp merge, one launch per layer).  The chunked pre-fill
+(32K prompt, 4K chunks, tcgen05 tensor cores) is measured in the same run and
+reported under "prefill".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl duo|reference]
+
+Under torchrun every rank runs its own replica on its own GPU with distinct
+sequences (weak scaling, no data-path collective); timing is the max over
+ranks of CUDA-event time.  ``--impl reference`` times the fp64 CPU oracle on a
+bounded sample of the same workload instead.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from head_split_kv_decode_b200 import binding as B  # noqa: E402
+from head_split_kv_decode_b200 import synth  # noqa: E402
+
+METRIC = "decode attn HBM GB/s (% of 8 TB/s) at 128K ctx; prefill attn TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- util
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- decode
+
+
+def decode_bytes_per_layer(w, batch, n, n_ret, n_str):
+    """Algorithmic bytes of one decode-attention launch (visible KV + Q + O)."""
+    per_tok = 4 * w.head_dim if w.kv_dtype != "int4" else 2 * (w.head_dim // 2 + 4)
+    io = 2 if w.kv_dtype != "f32" else 4
+    kv = batch * (n_ret * n + n_str * min(n, w.S + w.R)) * per_tok
+    qo = 2 * batch * w.n_q_heads * w.head_dim * io
+    return kv + qo
+
+
+def append_bytes(w, batch):
+    io = 2 if w.kv_dtype != "f32" else 4
+    return 2 * batch * w.n_kv_heads * w.head_dim * io
+
+
+def fill_cache(cache, w, mask, b_ids, chunk=8192):
+    """Pre-fill every layer with the workload's context through duo_append_kv."""
+    dt = synth.io_dtype(w)
+    for layer in range(w.layers):
+        for p0 in range(0, w.context, chunk):
+            pos = range(p0, min(w.context, p0 + chunk))
+            k = synth.history(w, layer, "k", b_ids, pos, device="cuda", mask_row=mask[layer]).to(dt)
+            v = synth.history(w, layer, "v", b_ids, pos, device="cuda", mask_row=mask[layer]).to(dt)
+            cache.append(layer, k.contiguous(), v.contiguous())
+        torch.cuda.synchronize()
+
+
+def decode_inputs(w, mask, b_ids, first, count):
+    """Per layer: q [count, B, Hq, d], k/v [count, B, 1, Hkv, d] for decode steps."""
+    dt = synth.io_dtype(w)
+    qs, ks, vs = [], [], []
+    pos = range(first, first + count)
+    for layer in range(w.layers):
+        q = synth.queries(w, layer, b_ids, pos, device="cuda").to(dt)        # [B, T, Hq, d]
+        k = synth.history(w, layer, "k", b_ids, pos, device="cuda", mask_row=mask[layer]).to(dt)
+        v = synth.history(w, layer, "v", b_ids, pos, device="cuda", mask_row=mask[layer]).to(dt)
+        qs.append(q.permute(1, 0, 2, 3).contiguous())
+        ks.append(k.permute(1, 0, 2, 3).unsqueeze(2).contiguous())
+        vs.append(v.permute(1, 0, 2, 3).unsqueeze(2).contiguous())
+    return qs, ks, vs
+
+
+def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
+    from head_split_kv_decode_b200.cache import DuoCache
+
+    K, W = args.steps, args.warmup
+    mask = synth.workload_mask(w)
+    b_ids = [rank * batch + b for b in range(batch)]
+    total_steps = W + 2 * K
+    cache = DuoCache(w.layers, batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.kv_dtype,
+                     w.context + total_steps + 1, mask, w.S, w.R)
+    t0 = time.time()
+    fill_cache(cache, w, mask, b_ids)
+    fill_s = time.time() - t0
+    qs, ks, vs = decode_inputs(w, mask, b_ids, w.context, total_steps)
+    outs = [torch.empty(batch, w.n_q_heads, w.head_dim, dtype=synth.io_dtype(w), device="cuda")
+            for _ in range(w.layers)]
+    lib = B.lib()
+    h = cache.handle
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    ws, wsb = cache.ws_ptr, cache.ws_bytes
+    n_ret = [int(mask[layer].sum()) for layer in range(w.layers)]
+    n_str = [w.n_kv_heads - r for r in n_ret]
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K * w.layers)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K * w.layers)]
+
+    def step(s, timed_idx=None):
+        for layer in range(w.layers):
+            st = lib.duo_append_kv(h, layer, ks[layer][s].data_ptr(), vs[layer][s].data_ptr(), 1, sh)
+            if st:
+                raise B.DuoError(st, "duo_append_kv")
+            if timed_idx is not None:
+                ev_s[timed_idx * w.layers + layer].record(stream)
+            st = lib.duo_decode_attn(h, layer, qs[layer][s].data_ptr(), outs[layer].data_ptr(),
+                                     0.0, ws, wsb, sh)
+            if st:
+                raise B.DuoError(st, "duo_decode_attn")
+            if timed_idx is not None:
+                ev_e[timed_idx * w.layers + layer].record(stream)
+
+    for s in range(W):
+        step(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    n_first = cache.seq_len(0) + 1
+    splits = cache.decode_splits(0)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(clock_gpu) as clk:
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(K):
+            step(W + i, timed_idx=i)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    kern_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+    if B.duo_poll_device_error() != 0:
+        raise RuntimeError("a bounded device wait gave up during the benchmark")
+
+    step_bytes = 0
+    launch_bytes = []
+    for i in range(K):
+        n = n_first + i
+        for layer in range(w.layers):
+            lb = decode_bytes_per_layer(w, batch, n, n_ret[layer], n_str[layer])
+            launch_bytes.append(lb)
+            step_bytes += lb + append_bytes(w, batch)
+    step_bytes /= K
+
+    # ---- end to end through the public API: pinned host inputs in, outputs out
+    host_q = [q[W + K:W + 2 * K].cpu().pin_memory() for q in qs]
+    host_k = [k[W + K:W + 2 * K].cpu().pin_memory() for k in ks]
+    host_v = [v[W + K:W + 2 * K].cpu().pin_memory() for v in vs]
+    host_o = [torch.empty((K,) + tuple(o.shape), dtype=o.dtype).pin_memory() for o in outs]
+    dq = [torch.empty_like(q[0]) for q in qs]
+    dk = [torch.empty_like(k[0]) for k in ks]
+    dv = [torch.empty_like(v[0]) for v in vs]
+    h2d = sum(x[0].numel() * x[0].element_size() for x in host_q + host_k + host_v)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        for layer in range(w.layers):
+            dq[layer].copy_(host_q[layer][i], non_blocking=True)
+            dk[layer].copy_(host_k[layer][i], non_blocking=True)
+            dv[layer].copy_(host_v[layer][i], non_blocking=True)
+            B.duo_append_kv(h, layer, dk[layer].data_ptr(), dv[layer].data_ptr(), 1, sh)
+            B.duo_decode_attn(h, layer, dq[layer].data_ptr(), outs[layer].data_ptr(), 0.0, ws, wsb, sh)
+            host_o[layer][i].copy_(outs[layer], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = t.tolist()
+
+    avg_kern_ms = sum(kern_ms) / len(kern_ms)
+    avg_launch_bytes = sum(launch_bytes) / len(launch_bytes)
+    achieved = avg_launch_bytes / (avg_kern_ms * 1e-3) / 1e9
+    res = {
+        "ms_per_step": ms / K,
+        "value": world * step_bytes / (ms / K * 1e-3) / 1e9,
+        "e2e_value": world * step_bytes / (e2e_ms / K * 1e-3) / 1e9,
+        "h2d": h2d, "d2h": d2h,
+        "step_bytes": step_bytes,
+        "kernel": {"name": "decode_kernel", "avg_ms": avg_kern_ms, "launches": len(kern_ms),
+                   "bytes_per_launch": avg_launch_bytes, "achieved_gbs": achieved},
+        "splits": splits,
+        "fill_s": fill_s,
+        "clocks": clk.summary(),
+        "context": n_first,
+        "gpu_launches": K * w.layers * 2,
+    }
+    del cache
+    torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------------------------- prefill
+
+
+def prefill_tile_flops(w, C, c0, retrieval, tile=128):
+    """Tile-counted flops of one chunk for one query head (4*d per visited
+    128x128 tile element pair), matching the kernel's tile visits."""
+    n_q_tiles = C // tile
+    total = 0
+    for qt in range(n_q_tiles):
+        q_lo = c0 + qt * tile
+        q_hi = q_lo + tile - 1
+        if retrieval:
+            keys = q_hi + 1
+            total += math.ceil(keys / tile) * tile
+        else:
+            vis = set()
+            for kt in range(math.ceil((q_hi + 1) / tile)):
+                k_lo, k_hi = kt * tile, kt * tile + tile - 1
+                if k_lo < w.S or k_hi > q_lo - w.R:
+                    vis.add(kt)
+            total += len(vis) * tile
+    return 4 * w.head_dim * tile * total
+
+
+def prefill_exact_flops(w, C, c0, retrieval):
+    total = 0
+    for i in range(c0, c0 + C):
+        total += (i + 1) if retrieval else min(i + 1, w.S + max(0, min(w.R, i + 1 - w.S)))
+    return 4 * w.head_dim * total
+
+
+def run_prefill(args, w, rank, world, peaks):
+    from head_split_kv_decode_b200.cache import DuoCache
+
+    mask = synth.workload_mask(w)[:1]
+    C = w.chunk
+    n_chunks = w.context // C
+    cache = DuoCache(1, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, "bf16", w.context, mask, w.S, w.R)
+    dt = torch.bfloat16
+    b_ids = [rank]
+    pos = range(w.context)
+    K = synth.history(w, 0, "k", b_ids, pos, device="cuda").to(dt)
+    V = synth.history(w, 0, "v", b_ids, pos, device="cuda").to(dt)
+    Q = synth.queries(w, 0, b_ids, pos, device="cuda").to(dt)
+    chunks = [(Q[:, c * C:(c + 1) * C].contiguous(), K[:, c * C:(c + 1) * C].contiguous(),
+               V[:, c * C:(c + 1) * C].contiguous()) for c in range(n_chunks)]
+    out = torch.empty_like(chunks[0][0])
+    lib = B.lib()
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+
+    def one_prompt(events=None):
+        cache.reset()
+        for c, (q, k, v) in enumerate(chunks):
+            if events is not None:
+                events[c][0].record(stream)
+            st = lib.duo_prefill_attn(cache.handle, 0, q.data_ptr(), k.data_ptr(), v.data_ptr(), C,
+                                      out.data_ptr(), 0.0, None, 0, sh)
+            if st:
+                raise B.DuoError(st, "duo_prefill_attn")
+            if events is not None:
+                events[c][1].record(stream)
+            st = lib.duo_append_kv(cache.handle, 0, k.data_ptr(), v.data_ptr(), C, sh)
+            if st:
+                raise B.DuoError(st, "duo_append_kv")
+
+    for _ in range(max(1, args.warmup)):
+        one_prompt()
+    torch.cuda.synchronize()
+    reps = max(1, min(args.steps, 8))
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_chunks)]
+           for _ in range(reps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for r in range(reps):
+        one_prompt(evs[r])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if B.duo_poll_device_error() != 0:
+        raise RuntimeError("a bounded device wait gave up during pre-fill")
+    attn_ms = sum(a.elapsed_time(b) for rep in evs for a, b in rep) / reps
+    n_ret = int(mask[0].sum())
+    G = w.group
+    tile_fl = exact_fl = 0
+    for c in range(n_chunks):
+        for kvh in range(w.n_kv_heads):
+            ret = bool(mask[0, kvh])
+            tile_fl += G * prefill_tile_flops(w, C, c * C, ret)
+            exact_fl += G * prefill_exact_flops(w, C, c * C, ret)
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tflops = tile_fl / (attn_ms * 1e-3) / 1e12
+    return {
+        "metric": "prefill attn TFLOP/s (tile-counted, 128x128 tiles)",
+        "value": tflops,
+        "unit": "TFLOP/s",
+        "exact_tflops": exact_fl / (attn_ms * 1e-3) / 1e12,
+        "ms_per_layer": attn_ms,
+        "ms_per_prompt_incl_append": e0.elapsed_time(e1) / reps,
+        "workload": w.name,
+        "retrieval_kv_heads": n_ret,
+        "tile_flops_per_layer": tile_fl,
+        "exact_flops_per_layer": exact_fl,
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None},
+        "gpu_launches": reps * n_chunks * 2,
+    }
+
+
+# --------------------------------------------------------------------------- oracle
+
+
+def oracle_decode_sample(w, batch, n, mask_row):
+    """Inputs for the CPU oracle: one decode step of layer 0 at context n for one
+    retrieval and one streaming KV head of batch row 0 (generated untimed)."""
+    ret = [h for h in range(w.n_kv_heads) if mask_row[h]][:1]
+    strm = [h for h in range(w.n_kv_heads) if not mask_row[h]][:1]
+    heads = ret + strm
+    dt = synth.io_dtype(w)
+    k = synth.history(w, 0, "k", [0], range(n), heads=heads, mask_row=mask_row).to(dt).double().numpy()
+    v = synth.history(w, 0, "v", [0], range(n), heads=heads, mask_row=mask_row).to(dt).double().numpy()
+    qh = [hq for h in heads for hq in range(h * w.group, (h + 1) * w.group)]
+    q = synth.queries(w, 0, [0], [n - 1], heads=qh).to(dt).double().numpy()[:, 0]
+    sub_mask = [1] * len(ret) + [0] * len(strm)
+    per_tok = 4 * w.head_dim
+    nbytes = (len(ret) * n + len(strm) * min(n, w.S + w.R)) * per_tok + \
+        2 * len(qh) * w.head_dim * 2
+    return (q, k, v, sub_mask), nbytes, "layer 0, one decode step at context %d, batch row 0, " \
+        "KV heads %s (retrieval) + %s (streaming)" % (n, ret, strm)
+
+
+def time_oracle(sample, w):
+    from oracle import attention as OA
+    q, k, v, sub_mask = sample
+    t = time.perf_counter()
+    OA.decode_reference(q, k, v, sub_mask, w.S, w.R)
+    return time.perf_counter() - t
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, batch):
+    mask = synth.workload_mask(w)
+    sample, nbytes, desc = oracle_decode_sample(w, batch, w.context + 1, mask[0])
+    reps, secs = 0, 0.0
+    while secs < 10.0 or reps < 2:
+        secs += time_oracle(sample, w)
+        reps += 1
+    return {"value": reps * nbytes / secs / 1e9, "unit": "GB/s", "cores": cpu_cores(),
+            "kind": "oracle",
+            "sample": desc + "; numpy fp64, repeated %d times (%.1f s)" % (reps, secs)}
+
+
+def reference_arm(args, w, batch):
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return 0
+    mask = synth.workload_mask(w)
+    sample, nbytes, desc = oracle_decode_sample(w, batch, w.context + 1, mask[0])
+    for _ in range(args.warmup):
+        time_oracle(sample, w)
+    secs = [time_oracle(sample, w) for _ in range(args.steps)]
+    total = sum(secs)
+    value = nbytes * args.steps / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, batch, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, batch, n_gpus):
+    return {"workload": w.name, "batch": batch, "context": w.context, "layers": w.layers,
+            "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+            "S": w.S, "R": w.R, "retrieval_frac": w.retrieval_frac,
+            "l2": "inputs larger than L2 (every step streams each layer's KV cache from HBM)",
+            "parallelism": "replicas x%d" % n_gpus}
+
+
+# --------------------------------------------------------------------------- main
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["duo", "reference"], default="duo")
+    ap.add_argument("--workload", default="llama3_8b_gqa_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--extra", action="store_true",
+                    help="also time batch 4 at 128K and the MHA 32K workload")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w, args.batch)
+
+    world, rank, local = dist_info()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    B.lib()
+    peaks, peak_kind = load_peaks()
+    clock_gpu = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x for x in vis.split(",") if x.strip()]
+        if local < len(ids) and ids[local].strip().isdigit():
+            clock_gpu = int(ids[local])
+
+    res = run_decode(args, w, args.batch, rank, world, peaks, peak_kind, clock_gpu)
+    extra = {}
+    if args.extra:
+        r4 = run_decode(args, w, 4, rank, world, peaks, peak_kind, clock_gpu)
+        extra["batch4"] = {"value": r4["value"], "unit": "GB/s", "ms_per_step": r4["ms_per_step"],
+                           "kernel_achieved_gbs": r4["kernel"]["achieved_gbs"],
+                           "frac": r4["kernel"]["achieved_gbs"] / peaks["hbm_gbs"]}
+        w2 = synth.WORKLOADS["llama2_7b_mha_32k"]
+        r2 = run_decode(args, w2, 1, rank, world, peaks, peak_kind, clock_gpu)
+        extra["llama2_7b_mha_32k"] = {"value": r2["value"], "unit": "GB/s",
+                                      "ms_per_step": r2["ms_per_step"],
+                                      "kernel_achieved_gbs": r2["kernel"]["achieved_gbs"],
+                                      "frac": r2["kernel"]["achieved_gbs"] / peaks["hbm_gbs"]}
+    prefill = None
+    if not args.no_prefill:
+        try:
+            prefill = run_prefill(args, synth.WORKLOADS["llama3_8b_gqa_prefill_32k"], rank, world, peaks)
+            prefill["roofline"]["peak_kind"] = peak_kind
+        except B.DuoError as e:
+            prefill = {"unavailable": str(e)}
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return 0
+    peak = peaks["hbm_gbs"]
+    kern = res["kernel"]
+    line = {
+        "metric": METRIC,
+        "value": res["value"],
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": workload_config(w, args.batch, world),
+        "pct_of_8tbs": 100.0 * res["value"] / world / 8000.0,
+        "roofline": {"bound": "hbm", "achieved": kern["achieved_gbs"], "peak": peak,
+                     "unit": "GB/s", "frac": kern["achieved_gbs"] / peak, "traffic": None,
+                     "kernel": kern["name"], "avg_launch_ms": kern["avg_ms"],
+                     "bytes_per_launch": kern["bytes_per_launch"], "peak_kind": peak_kind},
+        "e2e": {"value": res["e2e_value"], "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["gpu_launches"] + (prefill or {}).get("gpu_launches", 0),
+        "clocks": res["clocks"],
+        "decode_splits": res["splits"],
+        "prefill": prefill,
+    }
+    line.update(extra)
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.batch)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -12,9 +12,15 @@
 
 namespace duo {
 
-// An mbarrier wait gives up after this many polls (each poll may suspend the
-// thread for a short hardware-defined time), sets the error word and returns.
-constexpr uint32_t kWaitPolls = 1u << 24;
+// An mbarrier wait gives up after about kWaitNs nanoseconds of polling (read
+// from the global timer), records its code in the error word and returns false.
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -50,10 +56,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns false
-// (and records `code` in the error word) if it did not within kWaitPolls polls.
+// (and records `code` in the error word) if it did not within kWaitNs.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err, int code) {
-  for (uint32_t i = 0; i < kWaitPolls; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 256; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) break;
+  }
   if (err) atomicOr(err, code);
   return false;
 }

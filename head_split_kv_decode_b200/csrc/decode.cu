@@ -3,8 +3,8 @@
 // One launch covers a whole layer:
 //  * retrieval KV heads (full KV cache, causal attention over every token) run
 //    split-K flash decoding: CTA (b, head, split) streams its key range of the
-//    page into shared memory with 1-D bulk copies (the TMA engine, no
-//    multicast), computes the G query heads' logits and an online softmax, and
+//    page into its own shared memory with 1-D bulk copies (the TMA engine),
+//    computes the G query heads' logits and an online softmax, and
 //    writes a (normalised partial output, log-sum-exp) pair; the CTA that
 //    finishes last for a head merges all splits (an atomic ticket; no CTA ever
 //    waits for another);

@@ -42,6 +42,8 @@ struct duo_cache {
   int row_bytes;
   uint8_t *base;
   int forced_splits;
+  bool have_cfg;           // decode launch facts, queried once per cache
+  duo::DecodeConfig cfg;
 };
 
 namespace {
@@ -104,6 +106,19 @@ int choose_splits(const duo_cache *c, int layer, int64_t n, const duo::DecodeCon
   return (int)want;
 }
 
+// Occupancy and tile facts of the decode kernel for this cache's dtype, head
+// size and group size; queried from the runtime on first use only.
+cudaError_t cached_decode_config(duo_cache *c, duo::DecodeConfig *out) {
+  if (!c->have_cfg) {
+    const duo_cache_desc &d = c->desc;
+    cudaError_t e = duo::decode_config(d.kv_dtype, d.head_dim, d.n_q_heads / d.n_kv_heads, &c->cfg);
+    if (e != cudaSuccess) return e;
+    c->have_cfg = true;
+  }
+  *out = c->cfg;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -147,6 +162,7 @@ duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc, const u
   c->seq_len.assign(d.layers, 0);
   c->base = nullptr;
   c->forced_splits = 0;
+  c->have_cfg = false;
   c->row_bytes = d.kv_dtype == DUO_INT4 ? d.head_dim / 2 : d.head_dim * elem_bytes(d.kv_dtype);
   const bool q4 = d.kv_dtype == DUO_INT4;
 
@@ -260,7 +276,7 @@ duo_status duo_decode_attn(duo_cache *c, int32_t layer, const void *q, void *out
   const duo_cache_desc &d = c->desc;
   const int G = d.n_q_heads / d.n_kv_heads;
   duo::DecodeConfig cfg{};
-  cudaError_t e = duo::decode_config(d.kv_dtype, d.head_dim, G, &cfg);
+  cudaError_t e = cached_decode_config(c, &cfg);
   if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return DUO_ERR_CUDA;
   const int nsplit = choose_splits(c, layer, n, cfg);
@@ -403,9 +419,8 @@ duo_status duo_set_decode_splits(duo_cache *c, int32_t splits) {
 
 duo_status duo_decode_splits(const duo_cache *c, int32_t layer, int32_t *splits) {
   if (!c || !splits || layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
-  const duo_cache_desc &d = c->desc;
   duo::DecodeConfig cfg{};
-  cudaError_t e = duo::decode_config(d.kv_dtype, d.head_dim, d.n_q_heads / d.n_kv_heads, &cfg);
+  cudaError_t e = cached_decode_config(const_cast<duo_cache *>(c), &cfg);
   if (e != cudaSuccess) return e == cudaErrorInvalidValue ? DUO_ERR_UNSUPPORTED : DUO_ERR_CUDA;
   const int64_t n = c->seq_len[layer] > 0 ? c->seq_len[layer] : 1;
   const int want = choose_splits(c, layer, n, cfg);

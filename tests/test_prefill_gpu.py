@@ -1,0 +1,103 @@
+"""Chunked pre-fill parity: the tcgen05 kernel (through the C ABI) against the
+fp64 oracle, causal for retrieval heads and Lambda-masked for streaming heads.
+
+Covers chunks starting at 0 and in the middle of a prompt, ragged chunk
+lengths (not multiples of the 128-row tile), windows smaller and larger than a
+tile, the sink edge inside a chunk, MHA and GQA, batch > 1, and a whole prompt
+fed chunk by chunk with the append between chunks.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as OA
+from head_split_kv_decode_b200 import synth
+from head_split_kv_decode_b200.cache import DuoCache
+
+from _util import assert_parity, f64, seeded_mask
+
+pytestmark = pytest.mark.gpu
+
+BF = torch.bfloat16
+
+
+def _prompt(seed, B, n, Hq, Hkv, D=128):
+    K = synth.kv_field(seed * 10 + 1, range(B), range(n), Hkv, D, device="cuda").to(BF)
+    V = synth.kv_field(seed * 10 + 2, range(B), range(n), Hkv, D, device="cuda").to(BF)
+    Q = synth.kv_field(seed * 10 + 3, range(B), range(n), Hq, D, device="cuda").to(BF)
+    return Q, K, V
+
+
+def _run_chunks(cache, Q, K, V, bounds, check_rows=None):
+    """Feed [c0, c1) chunks: attend, then append.  Returns [(c0, out)]."""
+    outs = []
+    for c0, c1 in bounds:
+        q = Q[:, c0:c1].contiguous()
+        k = K[:, c0:c1].contiguous()
+        v = V[:, c0:c1].contiguous()
+        assert cache.seq_len(0) == c0
+        o = cache.prefill(0, q, k, v)
+        cache.append(0, k, v)
+        outs.append((c0, o.clone()))
+    torch.cuda.synchronize()
+    return outs
+
+
+@pytest.mark.parametrize("B,Hq,Hkv", [(1, 8, 2), (2, 4, 4)])
+@pytest.mark.parametrize("S,R", [(4, 64), (64, 256), (0, 1), (200, 50)])
+@pytest.mark.parametrize("bounds", [[(0, 128)], [(0, 300)], [(0, 257), (257, 700)],
+                                    [(0, 100), (100, 612), (612, 1000)]])
+def test_prefill_parity_small(B, Hq, Hkv, S, R, bounds):
+    n = bounds[-1][1]
+    seed = n + 7 * S + R + Hq
+    Q, K, V = _prompt(seed, B, n, Hq, Hkv)
+    mask = seeded_mask(seed, Hkv, max(1, Hkv // 2))
+    cache = DuoCache(1, B, Hq, Hkv, 128, "bf16", n, mask[None], S, R)
+    outs = _run_chunks(cache, Q, K, V, bounds)
+    Kd, Vd = f64(K), f64(V)
+    for (c0, o), (_, c1) in zip(outs, bounds):
+        ref = OA.prefill_reference(f64(Q[:, c0:c1]), Kd, Vd, c0, mask.numpy(), S, R)
+        assert_parity(o, ref, "bf16", "chunk [%d,%d) S=%d R=%d" % (c0, c1, S, R))
+
+
+def test_prefill_all_heads_one_kind():
+    B, Hq, Hkv, n = 1, 4, 2, 600
+    for bits in ([1, 1], [0, 0]):
+        Q, K, V = _prompt(31 + bits[0], B, n, Hq, Hkv)
+        mask = torch.tensor(bits, dtype=torch.uint8)
+        cache = DuoCache(1, B, Hq, Hkv, 128, "bf16", n, mask[None], 64, 256)
+        outs = _run_chunks(cache, Q, K, V, [(0, 300), (300, 600)])
+        for c0, o in outs:
+            ref = OA.prefill_reference(f64(Q[:, c0:c0 + 300]), f64(K), f64(V), c0, mask.numpy(), 64, 256)
+            assert_parity(o, ref, "bf16", "mask %s c0=%d" % (bits, c0))
+
+
+def test_prefill_then_decode_continues_the_same_cache():
+    """Pre-fill a prompt in chunks, then decode: the decode sees exactly what the
+    pre-fill appended (one consistent cache for both paths)."""
+    B, Hq, Hkv, n = 1, 8, 2, 900
+    S, R = 16, 128
+    Q, K, V = _prompt(77, B, n + 1, Hq, Hkv)
+    mask = torch.tensor([0, 1], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, 128, "bf16", n + 1, mask[None], S, R)
+    _run_chunks(cache, Q, K, V, [(0, 512), (512, n)])
+    cache.append(0, K[:, n:n + 1].contiguous(), V[:, n:n + 1].contiguous())
+    out = cache.decode(0, Q[:, n].contiguous())
+    ref = OA.decode_reference(f64(Q[:, n]), f64(K), f64(V), mask.numpy(), S, R)
+    assert_parity(out, ref, "bf16", "decode after prefill")
+
+
+def test_prefill_rejects_unsupported_and_capacity():
+    from head_split_kv_decode_b200.binding import DuoError
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    c32 = DuoCache(1, 1, 2, 2, 128, "f32", 256, mask[None], 4, 64)
+    q = torch.zeros(1, 128, 2, 128, device="cuda")
+    with pytest.raises(DuoError) as e:
+        c32.prefill(0, q, q, q)
+    assert e.value.name == "DUO_ERR_UNSUPPORTED"
+    cb = DuoCache(1, 1, 2, 2, 128, "bf16", 100, mask[None], 4, 64)
+    qb = torch.zeros(1, 128, 2, 128, device="cuda", dtype=BF)
+    with pytest.raises(DuoError) as e:
+        cb.prefill(0, qb, qb, qb)
+    assert e.value.name == "DUO_ERR_CAPACITY"
