@@ -314,29 +314,71 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ Dec
   if (!s_last) return;
   __threadfence();
   const int64_t part0 = ((int64_t)b * P.n_ret + pidx) * P.nsplit;
-  float *s_lse = reinterpret_cast<float *>(smem);  // [nsplit][G]
-  float *s_max = s_lse + P.nsplit * G;             // [G]
-  float *s_den = s_max + G;                        // [G]
-  for (int i = tid; i < P.nsplit * G; i += NT) s_lse[i] = __ldcg(P.ws_lse + part0 * G + i);
+  // weights w_s = 2^(lse_s - max) per (split, query head)
+  float *s_w = reinterpret_cast<float *>(smem);     // [nsplit][G]
+  float *s_den = s_w + P.nsplit * G;                // [G]
+  float *s_acc = s_w + ((P.nsplit * G + G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
+  for (int i = tid; i < P.nsplit * G; i += NT) s_w[i] = __ldcg(P.ws_lse + part0 * G + i);
   __syncthreads();
   if (tid < G) {
     float M = -INFINITY;
-    for (int sp = 0; sp < P.nsplit; ++sp) M = fmaxf(M, s_lse[sp * G + tid]);
+    for (int sp = 0; sp < P.nsplit; ++sp) M = fmaxf(M, s_w[sp * G + tid]);
     float den = 0.f;
     for (int sp = 0; sp < P.nsplit; ++sp) {
-      const float w = fast_exp2(s_lse[sp * G + tid] - M);
-      s_lse[sp * G + tid] = w;
+      const float w = fast_exp2(s_w[sp * G + tid] - M);
+      s_w[sp * G + tid] = w;
       den += w;
     }
-    s_max[tid] = M;
     s_den[tid] = den;
+  }
+  __syncthreads();
+  // warp w sums splits w, w+NWARPS, ...; lane l owns channels [4l, 4l+4) of
+  // every query head (D/4 float4 per head row, so lanes cover D = 128; for
+  // D = 64 the upper lanes idle).  Four splits' loads are kept in flight.
+  constexpr int L4 = D / 4;
+  float4 acc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane < L4) {
+    const float4 *src = reinterpret_cast<const float4 *>(P.ws_o + part0 * G * D) + lane;
+    int sp = warp;
+    for (; sp + 3 * NWARPS < P.nsplit; sp += 4 * NWARPS) {
+      float4 v[4][G];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int g = 0; g < G; ++g) v[u][g] = __ldcg(src + ((sp + u * NWARPS) * G + g) * L4);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float w = s_w[(sp + u * NWARPS) * G + g];
+          acc[g].x += w * v[u][g].x;
+          acc[g].y += w * v[u][g].y;
+          acc[g].z += w * v[u][g].z;
+          acc[g].w += w * v[u][g].w;
+        }
+    }
+    for (; sp < P.nsplit; sp += NWARPS)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4 v = __ldcg(src + (sp * G + g) * L4);
+        const float w = s_w[sp * G + g];
+        acc[g].x += w * v.x;
+        acc[g].y += w * v.y;
+        acc[g].z += w * v.z;
+        acc[g].w += w * v.w;
+      }
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      reinterpret_cast<float4 *>(s_acc + (warp * G + g) * D)[lane] = acc[g];
   }
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += NT) {
     const int g = idx / D, c = idx % D;
     float num = 0.f;
-    for (int sp = 0; sp < P.nsplit; ++sp)
-      num += s_lse[sp * G + g] * __ldcg(P.ws_o + ((part0 + sp) * G + g) * D + c);
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) num += s_acc[(w * G + g) * D + c];
     store_out(out + g * D + c, num / s_den[g]);
   }
   if (tid == 0) *cnt = 0u;  // leave the ticket ready for the next call

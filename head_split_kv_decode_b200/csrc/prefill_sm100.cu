@@ -41,8 +41,8 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr int kQA = 0, kQB = TILE;
 constexpr int kK0 = 2 * TILE, kV0 = 3 * TILE, kK1 = 4 * TILE, kV1 = 5 * TILE;
 constexpr int kBars = 6 * TILE;
-enum Bar { Q_FULL = 0, K_FULL0, K_FULL1, V_FULL0, V_FULL1, KV_EMPTY0, KV_EMPTY1,
-           S_FULL_A, S_FULL_B, P_FULL_A, P_FULL_B, O_FULL_A, O_FULL_B, DRAIN, NBARS };
+enum Bar { Q_FULL = 0, K_FULL0, K_FULL1, V_FULL0, V_FULL1, K_EMPTY0, K_EMPTY1, V_EMPTY0,
+           V_EMPTY1, S_FULL_A, S_FULL_B, P_FULL_A, P_FULL_B, O_FULL_A, O_FULL_B, DRAIN, NBARS };
 constexpr int kTmemSlot = kBars + NBARS * 8;
 constexpr int kAbort = kTmemSlot + 4;
 constexpr int kSmemBytes = kAbort + 4 + 1024;  // + alignment slack
@@ -103,6 +103,40 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Same load without the completion wait: issue several, then tmem_wait_ld().
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float *v) {
+  uint32_t *r = reinterpret_cast<uint32_t *>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Bits c in [0,32) set where first + 32*ch + c lies in [lo, hi).
+__device__ __forceinline__ uint32_t range_bits(int64_t lo, int64_t hi, int64_t first, int ch) {
+  const int64_t a = max(lo - (first + 32 * ch), (int64_t)0);
+  const int64_t b = min(hi - (first + 32 * ch), (int64_t)32);
+  if (b <= a) return 0u;
+  const uint32_t upto_b = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  const uint32_t below_a = (1u << a) - 1u;
+  return upto_b & ~below_a;
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
@@ -197,13 +231,20 @@ struct Sched {
     return kt <= ks_max || kt >= kb_lo;
   }
   __device__ int count() const {
+    if (ret) return n_pre + kt_max + 1;
     int n = 0;
     for (int t = 0; t < n_pre; ++t) n += pre_needed(t);
     for (int kt = 0; kt <= kt_max; ++kt) n += chunk_needed(kt);
     return n;
   }
-  // j-th visited tile -> (segment, tile index)
+  // j-th visited tile -> (segment, tile index); retrieval heads visit every
+  // tile, streaming heads walk their short candidate list.
   __device__ void get(int j, int &seg, int &idx) const {
+    if (ret) {
+      seg = j < n_pre ? 0 : 1;
+      idx = j < n_pre ? j : j - n_pre;
+      return;
+    }
     for (int t = 0; t < n_pre; ++t)
       if (pre_needed(t)) {
         if (j == 0) { seg = 0; idx = t; return; }
@@ -304,40 +345,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap *pk = retrieval ? &M.kr : &M.ks;
       const CUtensorMap *pv = retrieval ? &M.vr : &M.vs;
       const int pz = b * (retrieval ? P.n_ret : P.n_str) + pidx;
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
+      int issued_k = 0, issued_v = 0;
+      auto issue = [&](int j, bool is_v) -> bool {
         const int st = j & 1;
-        if (j >= 2 && !mbar_wait(bar(KV_EMPTY0 + st), (uint32_t)(((j - 2) >> 1) & 1), P.err,
-                                 kErrWaitPrefillLoad)) {
-          *abort_flag = 1;
-          break;
-        }
-        if (abort_set(abort_flag)) break;
+        if (j >= 2 && !mbar_wait(bar((is_v ? V_EMPTY0 : K_EMPTY0) + st), (uint32_t)(((j - 2) >> 1) & 1),
+                                 P.err, kErrWaitPrefillLoad))
+          return false;
         int seg, idx;
         sc.get(j, seg, idx);
-        const uint32_t kd = base + (st ? kK1 : kK0), vd = base + (st ? kV1 : kV0);
-        mbar_arrive_expect_tx(bar(K_FULL0 + st), TILE);
-        mbar_arrive_expect_tx(bar(V_FULL0 + st), TILE);
+        const uint32_t dst = base + (is_v ? (st ? kV1 : kV0) : (st ? kK1 : kK0));
+        const uint32_t fb = bar((is_v ? V_FULL0 : K_FULL0) + st);
+        mbar_arrive_expect_tx(fb, TILE);
         if (seg == 0) {
-          tma_load3(kd, pk, 0, idx * BN, pz, bar(K_FULL0 + st));
-          tma_load3(kd + BOX, pk, 64, idx * BN, pz, bar(K_FULL0 + st));
-          tma_load3(vd, pv, 0, idx * BN, pz, bar(V_FULL0 + st));
-          tma_load3(vd + BOX, pv, 64, idx * BN, pz, bar(V_FULL0 + st));
+          const CUtensorMap *m = is_v ? pv : pk;
+          tma_load3(dst, m, 0, idx * BN, pz, fb);
+          tma_load3(dst + BOX, m, 64, idx * BN, pz, fb);
         } else {
+          const CUtensorMap *m = is_v ? &M.vc : &M.kc;
           const int z = b * P.C + idx * BN;
-          tma_load3(kd, &M.kc, 0, kvh, z, bar(K_FULL0 + st));
-          tma_load3(kd + BOX, &M.kc, 64, kvh, z, bar(K_FULL0 + st));
-          tma_load3(vd, &M.vc, 0, kvh, z, bar(V_FULL0 + st));
-          tma_load3(vd + BOX, &M.vc, 64, kvh, z, bar(V_FULL0 + st));
+          tma_load3(dst, m, 0, kvh, z, fb);
+          tma_load3(dst + BOX, m, 64, kvh, z, fb);
         }
-        issued = j + 1;
+        return true;
+      };
+      for (int j = 0; j <= n_tiles; ++j) {
+        if (abort_set(abort_flag)) break;
+        if (j < n_tiles) {
+          if (!issue(j, false)) { *abort_flag = 1; break; }
+          issued_k = j + 1;
+        }
+        if (j >= 1) {
+          if (!issue(j - 1, true)) { *abort_flag = 1; break; }
+          issued_v = j;
+        }
       }
       // Copies still in flight land before the CTA can exit (bounded waits;
       // an already completed phase returns at once).
-      for (int jj = max(0, issued - 2); jj < issued; ++jj) {
+      for (int jj = max(0, issued_k - 2); jj < issued_k; ++jj)
         mbar_wait(bar(K_FULL0 + (jj & 1)), (uint32_t)((jj >> 1) & 1), P.err, kErrWaitPrefillLoad);
+      for (int jj = max(0, issued_v - 2); jj < issued_v; ++jj)
         mbar_wait(bar(V_FULL0 + (jj & 1)), (uint32_t)((jj >> 1) & 1), P.err, kErrWaitPrefillLoad);
-      }
     }
   } else if (warp == 9) {
     // =============================================================== MMA issuer
@@ -367,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(bar(S_FULL_A));
         issue_s(1, 0);
         mma_commit(bar(S_FULL_B));
+        mma_commit(bar(K_EMPTY0));
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j & 1;
@@ -389,10 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         issue_pv(1, st, j);
-        mma_commit(bar(KV_EMPTY0 + st));
+        mma_commit(bar(V_EMPTY0 + st));
         if (more) {
           issue_s(1, st ^ 1);
           mma_commit(bar(S_FULL_B));
+          mma_commit(bar(K_EMPTY0 + (st ^ 1)));
         } else {
           mma_commit(bar(O_FULL_B));
         }
@@ -416,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int p_bar = x ? P_FULL_B : P_FULL_A;
     const int o_bar = x ? O_FULL_B : O_FULL_A;
     const float sl2 = P.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f);
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = mbar_wait(bar(s_bar), (uint32_t)(j & 1), P.err, kErrWaitMma);
@@ -427,47 +477,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       int seg, idx;
       sc.get(j, seg, idx);
-      // key positions of this tile: column c -> (valid, position)
+
+      // Visible columns of this row as bit masks, one per 32 columns.  Every
+      // visible set here is a union of at most three position ranges.
       const int64_t first = (int64_t)idx * BN;
-      bool full;  // every column visible to this row
-      if (seg == 1)
-        full = retrieval && (first + BN - 1 < P.C) && (P.c0 + first + BN - 1 <= ipos);
-      else
-        full = retrieval && (first + BN - 1 < P.c0);
-      auto visible = [&](int c) -> bool {
-        int64_t pos;
-        if (seg == 1) {
-          const int64_t kr = first + c;
-          if (kr >= P.C) return false;
-          pos = P.c0 + kr;
-        } else if (retrieval) {
-          pos = first + c;
-          if (pos >= P.c0) return false;
-        } else {
-          const int64_t slot = first + c;
-          if (slot >= sc.filled) return false;
-          if (slot < P.S) {
-            pos = slot;
+      uint32_t vis[BN / 32];
+      if (seg == 1) {
+        // chunk keys: kr in [0, C), kr <= crow, and (streaming) sink or band
+        const int64_t hi = min((int64_t)P.C, (int64_t)crow + 1);
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          if (retrieval) {
+            vis[ch] = range_bits(0, hi, first, ch);
           } else {
-            const int64_t k = slot - P.S, last = P.c0 - 1 - P.S;
-            pos = P.S + k + ((last - k) / P.R) * P.R;
+            vis[ch] = range_bits(0, min(hi, (int64_t)P.S - P.c0), first, ch) |
+                      range_bits((int64_t)crow - P.R + 1, hi, first, ch);
           }
         }
-        if (pos > ipos) return false;
-        return retrieval || pos < P.S || ipos - pos < P.R;
+      } else if (retrieval) {
+        // page rows are positions; all below c0 are visible
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) vis[ch] = range_bits(0, P.c0, first, ch);
+      } else {
+        // slot buffer: sinks, plus the ring slots of positions in
+        // [max(S, ipos-R+1), c0) (a cyclic slot range)
+        const int64_t filled = sc.filled;
+        const int64_t p_lo = max((int64_t)P.S, ipos - P.R + 1), p_hi = P.c0;  // [p_lo, p_hi)
+        int64_t r1lo = 0, r1hi = 0, r2lo = 0, r2hi = 0;
+        if (p_lo < p_hi) {
+          const int64_t cnt = p_hi - p_lo;
+          const int64_t s_lo = P.S + (p_lo - P.S) % P.R;
+          r1lo = s_lo;
+          r1hi = min(s_lo + cnt, (int64_t)P.S + P.R);
+          const int64_t spill = s_lo + cnt - ((int64_t)P.S + P.R);
+          if (spill > 0) {
+            r2lo = P.S;
+            r2hi = P.S + spill;
+          }
+        }
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch)
+          vis[ch] = (range_bits(0, min((int64_t)P.S, filled), first, ch) |
+                     range_bits(r1lo, min(r1hi, filled), first, ch) |
+                     range_bits(r2lo, min(r2hi, filled), first, ch));
+      }
+      // Two passes over S in 64-column halves (register budget: ten warps on
+      // four schedulers leave 168 registers per thread): the row max, then the
+      // probabilities.  Masked logits become -inf.
+      constexpr int HALF = 64;
+      auto load_half = [&](int h, float (&v)[HALF]) {
+        tmem_ld32_async(tS + (uint32_t)(HALF * h), v);
+        tmem_ld32_async(tS + (uint32_t)(HALF * h + 32), v + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t bits = vis[2 * h + k];
+          if (bits != 0xffffffffu) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (!((bits >> i) & 1u)) v[32 * k + i] = -INFINITY;
+          }
+        }
       };
-      // pass 1: row max of this tile (log2 units)
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        float v[32];
-        tmem_ld32(tS + 32u * cc, v);
+      for (int h = 0; h < BN / HALF; ++h) {
+        float v[HALF];
+        load_half(h, v);
+        float t[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float t = v[i] * sl2;
-          if (full || visible(cc * 32 + i)) mx = fmaxf(mx, t);
-        }
+        for (int i = 0; i < 8; ++i)
+          t[i] = max3f(max3f(v[8 * i], v[8 * i + 1], v[8 * i + 2]),
+                       max3f(v[8 * i + 3], v[8 * i + 4], v[8 * i + 5]), fmaxf(v[8 * i + 6], v[8 * i + 7]));
+        mx = max3f(mx, max3f(t[0], t[1], t[2]), max3f(max3f(t[3], t[4], t[5]), t[6], t[7]));
       }
+      mx *= sl2;
       const float m_new = fmaxf(m, mx);
       const bool grow = m_new > m + kRescaleLog2 || (m == -INFINITY && m_new > -INFINITY);
       if (__any_sync(0xffffffffu, grow)) {
@@ -484,56 +568,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         if (grow) {
-          l *= alpha;
+          l2.x *= alpha;
+          l2.y *= alpha;
           m = m_new;
         }
       }
-      // pass 2: probabilities, written over S as packed bf16 (column c/2)
+      // probabilities 2^(s*scale*log2e - m), summed in fp32 and written over S
+      // as packed bf16 (column c/2 holds keys c, c+1)
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        float v[32];
-        tmem_ld32(tS + 32u * cc, v);
-        uint32_t pk[16];
+      for (int h = 0; h < BN / HALF; ++h) {
+        float v[HALF];
+        load_half(h, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = cc * 32 + 2 * i;
-          float p0 = 0.f, p1 = 0.f;
-          if (m != -INFINITY) {
-            if (full || visible(c)) p0 = fast_exp2(v[2 * i] * sl2 - m);
-            if (full || visible(c + 1)) p1 = fast_exp2(v[2 * i + 1] * sl2 - m);
+        for (int cc = 0; cc < HALF / 32; ++cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float2 t = ffma2(make_float2(v[32 * cc + 2 * i], v[32 * cc + 2 * i + 1]), sc2, nm2);
+            t.x = fast_exp2(t.x);
+            t.y = fast_exp2(t.y);
+            l2 = __fadd2_rn(l2, t);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(t.x, t.y);
+            pk[i] = *reinterpret_cast<uint32_t *>(&h2);
           }
-          l += p0 + p1;
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[i] = *reinterpret_cast<uint32_t *>(&h2);
+          tmem_st16(tS + (uint32_t)(HALF / 2 * h + 16 * cc), pk);
         }
-        tmem_st16(tS + 16u * cc, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(p_bar));
     }
+    const float l = l2.x + l2.y;
     if (ok) ok = mbar_wait(bar(o_bar), 0, P.err, kErrWaitMma);
     if (__all_sync(0xffffffffu, ok) && !abort_set(abort_flag)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out) +
                            (((int64_t)b * P.C + crow) * P.Hq + hq) * HD;
-#pragma unroll 1
-      for (int cc = 0; cc < HD / 32; ++cc) {
-        float o[32];
-        tmem_ld32(tO + 32u * cc, o);
-        if (crow < P.C) {
-          uint4 pk[4];
-          uint32_t *w = reinterpret_cast<uint32_t *>(pk);
+      float o[HD];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
-            w[i] = *reinterpret_cast<uint32_t *>(&h2);
+      for (int cc = 0; cc < HD / 32; ++cc) tmem_ld32_async(tO + 32u * cc, o + 32 * cc);
+      tmem_wait_ld();
+      if (crow < P.C) {
+        uint4 *dst = reinterpret_cast<uint4 *>(out);
+#pragma unroll
+        for (int i = 0; i < HD / 8; ++i) {
+          uint4 pk;
+          uint32_t *w = reinterpret_cast<uint32_t *>(&pk);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * i + 2 * k] * inv, o[8 * i + 2 * k + 1] * inv);
+            w[k] = *reinterpret_cast<uint32_t *>(&h2);
           }
-          uint4 *dst = reinterpret_cast<uint4 *>(out + cc * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = pk[i];
+          dst[i] = pk;
         }
       }
     } else {
