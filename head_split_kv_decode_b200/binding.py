@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libduo.so")
 
 MAX_KV_HEADS = 64
 MAX_SPLITS = 512
+DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
 DUO_OK = 0
 STATUS_NAMES = {
@@ -71,6 +72,7 @@ SIGNATURES = {
     "duo_cache_reset": (_I32, [_P]),
     "duo_append_kv": (_I32, [_P, _I32, _P, _P, _I32, _P]),
     "duo_decode_attn": (_I32, [_P, _I32, _P, _P, _F, _P, _SZ, _P]),
+    "duo_decode_attn_static": (_I32, [_P, _I32, _P, _P, _F, _P]),
     "duo_prefill_attn": (_I32, [_P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
     "duo_seq_len": (_I32, [_P, _I32, ctypes.POINTER(_I64)]),
     "duo_kv_bytes": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
@@ -151,6 +153,13 @@ def duo_append_kv(handle, layer, k_ptr, v_ptr, n_tokens, stream=0):
 def duo_decode_attn(handle, layer, q_ptr, out_ptr, softmax_scale, ws_ptr, ws_bytes, stream=0):
     _check(lib().duo_decode_attn(handle, layer, q_ptr, out_ptr, softmax_scale, ws_ptr,
                                  ws_bytes, stream), "duo_decode_attn")
+
+
+def duo_decode_attn_static(handle, layer, q_ptr, out_ptr, softmax_scale, stream=0):
+    """Decode without a workspace: the library's own fixed scratch array is used
+    (see include/duo.h for its limit and the serialisation rule)."""
+    _check(lib().duo_decode_attn_static(handle, layer, q_ptr, out_ptr, softmax_scale, stream),
+           "duo_decode_attn_static")
 
 
 def duo_prefill_attn(handle, layer, q_ptr, k_ptr, v_ptr, C, out_ptr, softmax_scale,

@@ -23,6 +23,7 @@
 
 static_assert(DUO_MAX_KV_HEADS == duo::kMaxKvHeads, "head table size");
 static_assert(DUO_MAX_SPLITS == duo::kMaxSplits, "split limit");
+static_assert(DUO_DECODE_STATIC_SCRATCH_BYTES == (8u << 20), "static decode scratch size");
 
 struct duo_cache {
   duo_cache_desc desc;
@@ -314,6 +315,70 @@ duo_status duo_decode_attn(duo_cache *c, int32_t layer, const void *q, void *out
   p.ws_cnt = need_ws ? reinterpret_cast<unsigned *>(wsb + w.cnt) : nullptr;
   p.ws_lse = need_ws ? reinterpret_cast<float *>(wsb + w.lse) : nullptr;
   p.ws_o = need_ws ? reinterpret_cast<float *>(wsb + w.o) : nullptr;
+  p.err = duo::device_error_word();
+  e = duo::launch_decode(p, d.kv_dtype, (cudaStream_t)stream);
+  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, void *out,
+                                  float scale, duo_stream stream) {
+  if (!c || !q || !out) return DUO_ERR_ARG;
+  if (layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
+  if (!c->base) return DUO_ERR_STATE;
+  if (!std::isfinite(scale)) return DUO_ERR_ARG;
+  const int64_t n = c->seq_len[layer];
+  if (n <= 0) return DUO_ERR_STATE;
+  const auto &L = c->layers[layer];
+  const duo_cache_desc &d = c->desc;
+  const int G = d.n_q_heads / d.n_kv_heads;
+  duo::DecodeConfig cfg{};
+  cudaError_t e = cached_decode_config(c, &cfg);
+  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return DUO_ERR_CUDA;
+  const int want = choose_splits(c, layer, n, cfg);
+  const int64_t split_len = round_up((n + want - 1) / want, cfg.tile_rows);
+  const int nsplit = (int)((n + split_len - 1) / split_len);
+  // Compact scratch layout for exactly this launch: tickets, lse, partial O.
+  const int64_t units = (int64_t)d.batch * L.n_ret;
+  const int64_t off_lse = round_up(units * 4, kAlign);
+  const int64_t off_o = off_lse + round_up(units * nsplit * G * 4, kAlign);
+  const int64_t need = off_o + units * nsplit * G * (int64_t)d.head_dim * 4;
+  const bool need_ws = L.n_ret > 0 && nsplit > 1;
+  if (need_ws && need > (int64_t)duo::decode_static_scratch_bytes()) return DUO_ERR_WORKSPACE;
+  uint8_t *scratch = nullptr;
+  if (need_ws) {
+    void *p = nullptr;
+    if (duo::decode_static_scratch(&p) != cudaSuccess) return DUO_ERR_CUDA;
+    scratch = static_cast<uint8_t *>(p);
+    // tickets start at zero for this launch (the array keeps earlier calls' bytes)
+    if (cudaMemsetAsync(scratch, 0, (size_t)(units * 4), (cudaStream_t)stream) != cudaSuccess)
+      return DUO_ERR_CUDA;
+  }
+  duo::DecodeParams p{};
+  p.q = q;
+  p.out = out;
+  p.p = layer_ptrs(c, layer);
+  p.h = L.h;
+  p.B = d.batch;
+  p.Hq = d.n_q_heads;
+  p.Hkv = d.n_kv_heads;
+  p.G = G;
+  p.D = d.head_dim;
+  p.n_ret = L.n_ret;
+  p.n_str = L.n_str;
+  p.S = c->S;
+  p.R = c->R;
+  p.W = c->W;
+  p.cap = d.capacity;
+  p.n = n;
+  p.nsplit = nsplit;
+  p.split_len = split_len;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d.head_dim);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.ws_cnt = need_ws ? reinterpret_cast<unsigned *>(scratch) : nullptr;
+  p.ws_lse = need_ws ? reinterpret_cast<float *>(scratch + off_lse) : nullptr;
+  p.ws_o = need_ws ? reinterpret_cast<float *>(scratch + off_o) : nullptr;
   p.err = duo::device_error_word();
   e = duo::launch_decode(p, d.kv_dtype, (cudaStream_t)stream);
   if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;

@@ -9,6 +9,7 @@ namespace duo {
 
 constexpr int kMaxKvHeads = 64;
 constexpr int kMaxSplits = 512;
+constexpr int kMaxDevices = 64;
 
 enum KvType : int { kF32 = 0, kBF16 = 1, kINT4 = 2 };
 
@@ -82,5 +83,9 @@ cudaError_t launch_append(const AppendParams &a, int kv_type, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &d, int kv_type, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s);
 int *device_error_word();  // device address of the error word
+
+// Library-owned decode scratch for duo_decode_attn_static (decode_static.cu).
+size_t decode_static_scratch_bytes();
+cudaError_t decode_static_scratch(void **ptr);
 
 }  // namespace duo

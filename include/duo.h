@@ -152,6 +152,30 @@ duo_status duo_decode_attn(duo_cache *cache, int32_t layer, const void *q,
                            void *out, float softmax_scale, void *workspace,
                            size_t workspace_bytes, duo_stream stream);
 
+/* Decode attention like duo_decode_attn, but with no workspace argument and
+ * no allocation of any kind: the split-K scratch (partial outputs, log-sum-exp
+ * values, merge tickets) lives in a fixed array inside the library,
+ * DUO_DECODE_STATIC_SCRATCH_BYTES in size, that every GPU loading the library
+ * holds until the process exits.  The paper has no counterpart to this call.
+ * It is for callers that cannot call cudaMalloc (or any allocator) to get a
+ * workspace: a serving loop that must never stall, since cudaMalloc and
+ * cudaFree can synchronise the device; a host program whose device memory is
+ * entirely reserved by another allocator it may not call into; a plugin given
+ * only the input and output pointers.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array: calls that may overlap on the GPU (other
+ *    streams, other threads, other caches) race and must be serialised by the
+ *    caller.  The merge tickets are cleared on the stream before each launch.
+ *  - If the scratch this layer needs (batch x retrieval heads x splits x
+ *    group x (head_dim + 1) x 4 bytes, plus tickets) exceeds the array, the
+ *    call returns DUO_ERR_WORKSPACE before enqueuing anything.
+ * Results equal duo_decode_attn's for the same cache state. */
+#define DUO_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+duo_status duo_decode_attn_static(duo_cache *cache, int32_t layer, const void *q,
+                                  void *out, float softmax_scale, duo_stream stream);
+
 /* Chunked pre-fill attention for one layer: C queries at positions
  * seq_len .. seq_len+C-1 attend to the cache as it stands (positions below
  * seq_len) plus the chunk's own k/v: causal for retrieval heads, Lambda mask
