@@ -47,7 +47,8 @@ class duo_cache_desc(ctypes.Structure):
 
 class duo_layout_view(ctypes.Structure):
     _fields_ = [("n_retrieval", ctypes.c_int32), ("n_streaming", ctypes.c_int32),
-                ("window", ctypes.c_int32), ("row_bytes", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("window_stride", ctypes.c_int32),
+                ("row_bytes", ctypes.c_int32),
                 ("capacity", ctypes.c_int64), ("seq_len", ctypes.c_int64),
                 ("ret_k", ctypes.c_int64), ("ret_v", ctypes.c_int64),
                 ("str_k", ctypes.c_int64), ("str_v", ctypes.c_int64),

@@ -131,7 +131,7 @@ class DuoCache:
         if off < 0:
             return None
         heads = lv.n_retrieval if name.startswith("ret") else lv.n_streaming
-        rows = lv.capacity if name.startswith("ret") else lv.window
+        rows = lv.capacity if name.startswith("ret") else lv.window_stride
         width = 4 if name.endswith("_sz") else lv.row_bytes
         nbytes = self.batch * heads * rows * width
         return self.storage[off:off + nbytes].view(self.batch, heads, rows, width)

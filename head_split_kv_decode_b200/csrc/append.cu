@@ -38,7 +38,7 @@ __global__ void append_kernel(const __grid_constant__ AppendParams a, int row_by
     } else {
       if (!(p < a.S || p >= end - a.R)) continue;
       const int64_t slot = p < a.S ? p : a.S + (p - a.S) % a.R;
-      off = (((int64_t)b * a.n_str + idx) * a.W + slot) * row_bytes;
+      off = (((int64_t)b * a.n_str + idx) * a.Ws + slot) * row_bytes;
       dk = a.p.str_k;
       dv = a.p.str_v;
     }
@@ -82,7 +82,7 @@ __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
     } else {
       if (!(p < a.S || p >= end - a.R)) continue;
       const int64_t slot = p < a.S ? p : a.S + (p - a.S) % a.R;
-      row = ((int64_t)b * a.n_str + idx) * a.W + slot;
+      row = ((int64_t)b * a.n_str + idx) * a.Ws + slot;
       codes = which ? a.p.str_v : a.p.str_k;
       sz = which ? a.p.str_v_sz : a.p.str_k_sz;
     }

@@ -28,6 +28,7 @@ static_assert(DUO_DECODE_STATIC_SCRATCH_BYTES == (8u << 20), "static decode scra
 struct duo_cache {
   duo_cache_desc desc;
   int S, R, W;
+  int Ws;                     // rows per streaming head buffer
   std::vector<uint8_t> mask;  // [layers][Hkv]
   struct Layer {
     int n_ret, n_str;
@@ -159,6 +160,10 @@ duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc, const u
   c->S = S;
   c->R = R;
   c->W = S + R;
+  // INT4 keeps scale/zero rows in 16-byte groups of four tokens, so its row
+  // counts per head are rounded up to a multiple of 4.
+  c->Ws = d.kv_dtype == DUO_INT4 ? (int)round_up(c->W, 4) : c->W;
+  if (d.kv_dtype == DUO_INT4) c->desc.capacity = round_up(d.capacity, 4);
   c->mask.assign(head_mask, head_mask + (size_t)d.layers * d.n_kv_heads);
   c->seq_len.assign(d.layers, 0);
   c->base = nullptr;
@@ -188,8 +193,8 @@ duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc, const u
         L.h.str_heads[L.n_str++] = (int8_t)h;
       }
     }
-    const int64_t ret_rows = (int64_t)d.batch * L.n_ret * d.capacity;
-    const int64_t str_rows = (int64_t)d.batch * L.n_str * c->W;
+    const int64_t ret_rows = (int64_t)d.batch * L.n_ret * c->desc.capacity;
+    const int64_t str_rows = (int64_t)d.batch * L.n_str * c->Ws;
     L.off_ret_k = L.n_ret ? take(ret_rows * c->row_bytes) : -1;
     L.off_ret_v = L.n_ret ? take(ret_rows * c->row_bytes) : -1;
     L.off_str_k = L.n_str ? take(str_rows * c->row_bytes) : -1;
@@ -202,7 +207,7 @@ duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc, const u
     c->layers.push_back(L);
   }
   c->cache_bytes = (size_t)off;
-  c->ws_bytes = (size_t)ws_layout(d, c->n_ret_max).total;
+  c->ws_bytes = (size_t)ws_layout(c->desc, c->n_ret_max).total;
   *out = c;
   return DUO_OK;
 }
@@ -257,6 +262,7 @@ duo_status duo_append_kv(duo_cache *c, int32_t layer, const void *k, const void 
   a.S = c->S;
   a.R = c->R;
   a.W = c->W;
+  a.Ws = c->Ws;
   a.cap = c->desc.capacity;
   a.n_cur = n_cur;
   a.n_tok = n_tokens;
@@ -305,6 +311,7 @@ duo_status duo_decode_attn(duo_cache *c, int32_t layer, const void *q, void *out
   p.S = c->S;
   p.R = c->R;
   p.W = c->W;
+  p.Ws = c->Ws;
   p.cap = d.capacity;
   p.n = n;
   p.nsplit = (int)((n + split_len - 1) / split_len);
@@ -370,6 +377,7 @@ duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, vo
   p.S = c->S;
   p.R = c->R;
   p.W = c->W;
+  p.Ws = c->Ws;
   p.cap = d.capacity;
   p.n = n;
   p.nsplit = nsplit;
@@ -458,6 +466,7 @@ duo_status duo_layout_info(const duo_cache *c, int32_t layer, duo_layout_view *o
   o->n_retrieval = L.n_ret;
   o->n_streaming = L.n_str;
   o->window = c->W;
+  o->window_stride = c->Ws;
   o->row_bytes = c->row_bytes;
   o->capacity = c->desc.capacity;
   o->seq_len = c->seq_len[layer];

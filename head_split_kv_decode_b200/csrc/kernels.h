@@ -40,6 +40,7 @@ struct AppendParams {
   LayerPtrs p;
   HeadTables h;
   int B, Hkv, D, n_ret, n_str, S, R, W;
+  int Ws;              // rows per streaming head buffer (W, or W rounded up to 4 for int4)
   int64_t cap, n_cur, n_tok;
 };
 
@@ -49,6 +50,7 @@ struct DecodeParams {
   LayerPtrs p;
   HeadTables h;
   int B, Hq, Hkv, G, D, n_ret, n_str, S, R, W;
+  int Ws;              // rows per streaming head buffer
   int64_t cap;
   int64_t n;           // tokens in the cache, the query is at position n-1
   int nsplit;          // splits per retrieval head

@@ -87,7 +87,7 @@ typedef struct duo_cache_desc {
   int32_t n_kv_heads;  /* <= DUO_MAX_KV_HEADS, divides n_q_heads */
   int32_t head_dim;    /* 64 or 128 */
   int32_t kv_dtype;    /* duo_kv_dtype */
-  int64_t capacity;    /* max tokens a retrieval page holds */
+  int64_t capacity;    /* max tokens a retrieval page holds (INT4: rounded up to 4) */
 } duo_cache_desc;
 
 typedef struct duo_cache duo_cache;
@@ -98,11 +98,12 @@ typedef struct duo_layout_view {
   int32_t n_retrieval;   /* retrieval KV heads in this layer */
   int32_t n_streaming;   /* streaming KV heads in this layer */
   int32_t window;        /* S + R */
+  int32_t window_stride; /* rows per streaming head buffer: window, rounded up to 4 for INT4 */
   int32_t row_bytes;     /* bytes of one token of one head: d*4 (f32), d*2 (bf16), d/2 (int4 codes) */
   int64_t capacity;
   int64_t seq_len;       /* tokens appended so far */
   int64_t ret_k, ret_v;  /* [batch][n_retrieval][capacity][row] */
-  int64_t str_k, str_v;  /* [batch][n_streaming][window][row] */
+  int64_t str_k, str_v;  /* [batch][n_streaming][window_stride][row] */
   int64_t ret_k_sz, ret_v_sz, str_k_sz, str_v_sz; /* int4 only: fp16 (scale, zero) per token, same indexing */
   int32_t kind[DUO_MAX_KV_HEADS];         /* 1 retrieval, 0 streaming, per KV head */
   int32_t packed_index[DUO_MAX_KV_HEADS]; /* index among heads of the same kind */

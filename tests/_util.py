@@ -10,21 +10,27 @@ import numpy as np
 import torch
 
 TOL = {
-    "f32": dict(max=1e-5, mean=None),
-    "bf16": dict(max=2e-2, mean=2e-3),
-    "int4": dict(max=2e-2, mean=None),
+    "f32": dict(max=1e-5, mean=None, rel_above_one=False),
+    "bf16": dict(max=2e-2, mean=2e-3, rel_above_one=False),
+    # INT4 outputs are bf16 and, with the x10 outlier channels of the INT4
+    # workload, short contexts give |O| up to ~40, where bf16's own half-ulp
+    # (2^-9 relative, 0.0625 at 32) exceeds 2e-2.  So for INT4 the 2e-2 bound
+    # is applied to |err| / max(1, |ref|): absolute below 1, relative above.
+    "int4": dict(max=2e-2, mean=None, rel_above_one=True),
 }
 
 
-def parity_errors(got, ref):
+def parity_errors(got, ref, rel_above_one=False):
     g = got.detach().to("cpu", torch.float64).numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
     r = np.asarray(ref, dtype=np.float64)
     err = np.abs(g - r)
+    if rel_above_one:
+        err = err / np.maximum(1.0, np.abs(r))
     return float(err.max()), float(err.mean())
 
 
 def assert_parity(got, ref, kind, what=""):
-    mx, mean = parity_errors(got, ref)
+    mx, mean = parity_errors(got, ref, TOL[kind]["rel_above_one"])
     tol = TOL[kind]
     assert np.isfinite(mx), "%s: non-finite output" % what
     assert mx <= tol["max"], "%s: max |err| %.3g > %.3g" % (what, mx, tol["max"])

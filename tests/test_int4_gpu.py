@@ -1,0 +1,125 @@
+"""INT4 KV cache: quantise-on-append bit for bit, and decode against an oracle
+fed the identically dequantised K/V (max |err| <= 2e-2)."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as OA
+from oracle import cache as OC
+from oracle import int4 as OQ
+from head_split_kv_decode_b200 import synth
+from head_split_kv_decode_b200.cache import DuoCache
+
+from _util import assert_parity, f64, seeded_mask
+
+pytestmark = pytest.mark.gpu
+
+BF = torch.bfloat16
+
+
+def _inputs(seed, B, n, Hq, Hkv, D, outliers=True):
+    K = synth.kv_field(seed * 10 + 1, range(B), range(n), Hkv, D, device="cuda")
+    V = synth.kv_field(seed * 10 + 2, range(B), range(n), Hkv, D, device="cuda")
+    if outliers:  # a few channels x10, fixed across tokens (as in the 1M-context workload)
+        ch = synth.outlier_channels(seed, D, 0.02).cuda()
+        K[..., ch] *= 10.0
+        V[..., ch] *= 10.0
+    q = synth.kv_field(seed * 10 + 3, range(B), [n - 1], Hq, D, device="cuda")[:, 0]
+    return K.to(BF), V.to(BF), q.to(BF)
+
+
+def _dequant_history(X):
+    """Oracle side: fp32 mirror of the encoder on the exact bf16 inputs, then
+    the exact dequantisation.  Returns (x_hat float64, codes, sc, zp)."""
+    x = X.detach().cpu().float().numpy()
+    codes, sc, zp = OQ.quantize_int4(x)
+    return OQ.dequantize_int4(codes, sc, zp), codes, sc, zp
+
+
+def _fill(cache, K, V, chunks):
+    n = K.shape[1]
+    pos = 0
+    sizes = list(chunks)
+    while pos < n - 1:
+        c = min(sizes.pop(0) if sizes else n - 1 - pos, n - 1 - pos)
+        cache.append(0, K[:, pos:pos + c].contiguous(), V[:, pos:pos + c].contiguous())
+        pos += c
+    cache.append(0, K[:, n - 1:].contiguous(), V[:, n - 1:].contiguous())
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(1, 8, 2, 128), (2, 4, 4, 64), (1, 8, 8, 128)])
+@pytest.mark.parametrize("n", [1, 3, 70, 333, 2049])
+def test_int4_append_bit_exact_and_decode(B, Hq, Hkv, D, n):
+    S, R = 4, 64
+    seed = n + D + Hkv
+    K, V, q = _inputs(seed, B, n, Hq, Hkv, D)
+    mask = seeded_mask(seed, Hkv, max(1, Hkv // 2))
+    cache = DuoCache(1, B, Hq, Hkv, D, "int4", n, mask[None], S, R)
+    _fill(cache, K, V, [2, 31, 500])
+    out = cache.decode(0, q)
+    torch.cuda.synchronize()
+
+    Kh, Kc, Ks, Kz = _dequant_history(K)
+    Vh, Vc, Vs, Vz = _dequant_history(V)
+    ref = OA.decode_reference(f64(q), Kh, Vh, mask.numpy(), S, R)
+    assert_parity(out, ref, "int4", "int4 decode n=%d" % n)
+
+    # cache bytes: packed codes and (scale, zero) pairs, bit for bit
+    lv = cache.layout(0)
+    for name, codes, sc, zp in (("k", Kc, Ks, Kz), ("v", Vc, Vs, Vz)):
+        packed = OQ.pack_nibbles(codes)                                  # [B, n, Hkv, D/2]
+        szb = np.stack([sc, zp], axis=-1).view(np.uint8).reshape(B, n, Hkv, 4)
+        ret = cache.region(0, "ret_" + name)
+        ret_sz = cache.region(0, "ret_%s_sz" % name)
+        st = cache.region(0, "str_" + name)
+        st_sz = cache.region(0, "str_%s_sz" % name)
+        for h in range(Hkv):
+            idx = lv.packed_index[h]
+            for b in range(B):
+                if mask[h]:
+                    np.testing.assert_array_equal(ret[b, idx, :n].cpu().numpy(), packed[b, :, h])
+                    np.testing.assert_array_equal(ret_sz[b, idx, :n].cpu().numpy(), szb[b, :, h])
+                else:
+                    exp, filled = OC.expected_streaming_buffer(packed[b, :, h], S, R)
+                    np.testing.assert_array_equal(st[b, idx, :S + R].cpu().numpy()[filled], exp[filled])
+                    exp, filled = OC.expected_streaming_buffer(szb[b, :, h], S, R)
+                    np.testing.assert_array_equal(st_sz[b, idx, :S + R].cpu().numpy()[filled], exp[filled])
+    kept, full = cache.kv_bytes()
+    assert (kept, full) == OC.kv_bytes(mask[None].numpy(), B, n, S, R, D, "int4")
+
+
+def test_int4_split_counts_agree():
+    B, Hq, Hkv, D, n, S, R = 1, 8, 2, 128, 20000, 64, 256
+    K, V, q = _inputs(7, B, n, Hq, Hkv, D)
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, D, "int4", n, mask[None], S, R)
+    _fill(cache, K, V, [8192, 8192])
+    Kh = _dequant_history(K)[0]
+    Vh = _dequant_history(V)[0]
+    ref = OA.decode_reference(f64(q), Kh, Vh, mask.numpy(), S, R)
+    for splits in (1, 3, 64, 0):
+        cache.set_decode_splits(splits)
+        assert_parity(cache.decode(0, q), ref, "int4", "splits=%d" % splits)
+
+
+def test_int4_constant_rows_and_prefill_unsupported():
+    """A (token, head) row of identical values has scale 0: codes 0, x_hat = zp."""
+    from head_split_kv_decode_b200.binding import DuoError
+    B, Hq, Hkv, D, n = 1, 2, 2, 128, 40
+    K = torch.full((B, n, Hkv, D), 0.75, dtype=BF, device="cuda")
+    V = synth.kv_field(3, range(B), range(n), Hkv, D, device="cuda").to(BF)
+    q = synth.kv_field(4, range(B), [n - 1], Hq, D, device="cuda")[:, 0].to(BF)
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, D, "int4", n, mask[None], 2, 8)
+    cache.append(0, K, V)
+    out = cache.decode(0, q)
+    Kh = _dequant_history(K)[0]
+    assert (Kh == 0.75).all()
+    ref = OA.decode_reference(f64(q), Kh, _dequant_history(V)[0], mask.numpy(), 2, 8)
+    assert_parity(out, ref, "int4", "constant rows")
+    with pytest.raises(DuoError) as e:
+        cache.prefill(0, torch.zeros(B, 8, Hq, D, dtype=BF, device="cuda"),
+                      torch.zeros(B, 8, Hkv, D, dtype=BF, device="cuda"),
+                      torch.zeros(B, 8, Hkv, D, dtype=BF, device="cuda"))
+    assert e.value.name == "DUO_ERR_UNSUPPORTED"
