@@ -60,6 +60,27 @@ def dist_info():
     return world, rank, local
 
 
+def replica_batch_ids(rank, batch):
+    """Sequences one rank's replica decodes: rank r owns batch rows
+    [r*batch, (r+1)*batch) of the synthetic stream, so no two ranks repeat work."""
+    return [rank * batch + b for b in range(batch)]
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of per-rank timings (ms) across the process group."""
+    if world == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_rate(bytes_per_rank_step, world, steps, max_ms):
+    """Whole-job GB/s: the bytes every rank processed in `steps` steps over the
+    slowest rank's time."""
+    return world * bytes_per_rank_step * steps / (max_ms * 1e-3) / 1e9
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
 
@@ -168,7 +189,7 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
 
     K, W = args.steps, args.warmup
     mask = synth.workload_mask(w)
-    b_ids = [rank * batch + b for b in range(batch)]
+    b_ids = replica_batch_ids(rank, batch)
     total_steps = W + 2 * K
     cache = DuoCache(w.layers, batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.kv_dtype,
                      w.context + total_steps + 1, mask, w.S, w.R)
@@ -260,18 +281,15 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = t.tolist()
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, "cuda")
 
     avg_kern_ms = sum(kern_ms) / len(kern_ms)
     avg_launch_bytes = sum(launch_bytes) / len(launch_bytes)
     achieved = avg_launch_bytes / (avg_kern_ms * 1e-3) / 1e9
     res = {
         "ms_per_step": ms / K,
-        "value": world * step_bytes / (ms / K * 1e-3) / 1e9,
-        "e2e_value": world * step_bytes / (e2e_ms / K * 1e-3) / 1e9,
+        "value": aggregate_rate(step_bytes, world, K, ms),
+        "e2e_value": aggregate_rate(step_bytes, world, K, e2e_ms),
         "h2d": h2d, "d2h": d2h,
         "step_bytes": step_bytes,
         "kernel": {"name": "decode_kernel", "avg_ms": avg_kern_ms, "launches": len(kern_ms),
@@ -521,14 +539,19 @@ def main(argv=None):
     if args.extra:
         r4 = run_decode(args, w, 4, rank, world, peaks, peak_kind, clock_gpu)
         extra["batch4"] = {"value": r4["value"], "unit": "GB/s", "ms_per_step": r4["ms_per_step"],
+                           "kernel_avg_launch_ms": r4["kernel"]["avg_ms"],
                            "kernel_achieved_gbs": r4["kernel"]["achieved_gbs"],
-                           "frac": r4["kernel"]["achieved_gbs"] / peaks["hbm_gbs"]}
-        w2 = synth.WORKLOADS["llama2_7b_mha_32k"]
-        r2 = run_decode(args, w2, 1, rank, world, peaks, peak_kind, clock_gpu)
-        extra["llama2_7b_mha_32k"] = {"value": r2["value"], "unit": "GB/s",
-                                      "ms_per_step": r2["ms_per_step"],
-                                      "kernel_achieved_gbs": r2["kernel"]["achieved_gbs"],
-                                      "frac": r2["kernel"]["achieved_gbs"] / peaks["hbm_gbs"]}
+                           "frac": r4["kernel"]["achieved_gbs"] / peaks["hbm_gbs"],
+                           "decode_splits": r4["splits"], "gpu_launches": r4["gpu_launches"]}
+        for key in ("llama2_7b_mha_32k", "llama3_8b_gqa_int4_1m"):
+            wx = synth.WORKLOADS[key]
+            rx = run_decode(args, wx, 1, rank, world, peaks, peak_kind, clock_gpu)
+            extra[key] = {"workload": wx.name, "value": rx["value"], "unit": "GB/s",
+                          "ms_per_step": rx["ms_per_step"],
+                          "kernel_avg_launch_ms": rx["kernel"]["avg_ms"],
+                          "kernel_achieved_gbs": rx["kernel"]["achieved_gbs"],
+                          "frac": rx["kernel"]["achieved_gbs"] / peaks["hbm_gbs"],
+                          "decode_splits": rx["splits"], "gpu_launches": rx["gpu_launches"]}
     prefill = None
     if not args.no_prefill:
         try:

@@ -294,14 +294,21 @@ static cudaError_t dispatch(const DecodeParams &d, int kv_type, int D, int G, cu
 
 cudaError_t decode_int4_config(int D, int G, DecodeConfig *cfg);
 cudaError_t launch_decode_int4(const DecodeParams &d, cudaStream_t s);
+bool decode_mma_supported(int kv_type, int D, int G);
+cudaError_t decode_mma_config(int kv_type, int G, DecodeConfig *cfg);
+cudaError_t launch_decode_mma(const DecodeParams &d, int kv_type, cudaStream_t s);
 
+// head_dim 128 with a bf16 or 4-bit cache runs the tensor-core decode
+// (decode_mma.cu); fp32 caches and head_dim 64 run the CUDA-core kernels.
 cudaError_t decode_config(int kv_type, int D, int G, DecodeConfig *cfg) {
+  if (decode_mma_supported(kv_type, D, G)) return decode_mma_config(kv_type, G, cfg);
   if (kv_type == kINT4) return decode_int4_config(D, G, cfg);
   DecodeParams dummy{};
   return dispatch(dummy, kv_type, D, G, nullptr, cfg);
 }
 
 cudaError_t launch_decode(const DecodeParams &d, int kv_type, cudaStream_t s) {
+  if (decode_mma_supported(kv_type, d.D, d.G)) return launch_decode_mma(d, kv_type, s);
   if (kv_type == kINT4) return launch_decode_int4(d, s);
   return dispatch(d, kv_type, d.D, d.G, s, nullptr);
 }

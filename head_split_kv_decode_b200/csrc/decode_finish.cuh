@@ -9,60 +9,21 @@
 
 namespace duo {
 
-// State layout expected: each 8-lane group of a warp holds m[g], l[g] and NP
-// fp32 pairs of the output row of query head g; chan(li, j) gives the channel
-// of pair j's first element for lane li of the group.
-template <typename T, int D, int G, int NWARPS, int NP, typename ChanFn>
-__device__ __forceinline__ void decode_finish(const DecodeParams &P, uint8_t *smem, int *s_last_p,
-                                              float (&m)[G], float (&l)[G], float2 (&of)[G][NP],
-                                              ChanFn chan, bool retrieval, int b, int kvh, int pidx,
-                                              int split) {
+// Second half of the epilogue: the per-warp states of the CTA are staged in
+// shared memory as red_m [NWARPS][G], red_l [NWARPS][G] (log2 units) and
+// red_o [NWARPS][G][D] (unnormalised), all starting at `smem`.  Combines them,
+// writes the output (single split) or this split's normalised partial and
+// log-sum-exp, and lets the last split of the head merge every partial.
+template <typename T, int D, int G, int NWARPS>
+__device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8_t *smem,
+                                                    int *s_last_p, bool retrieval, int b, int kvh,
+                                                    int pidx, int split) {
   constexpr int NT = NWARPS * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int grp = lane >> 3, li = lane & 7;
   int &s_last = *s_last_p;
-  // ---- combine the four 8-lane groups of each warp
-#pragma unroll
-  for (int off = 8; off <= 16; off <<= 1)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[g], off);
-      const float mn = fmaxf(m[g], mo);
-      const float a = (m[g] == -INFINITY) ? 0.f : fast_exp2(m[g] - mn);
-      const float c = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
-      l[g] = l[g] * a + lo * c;
-#pragma unroll
-      for (int j = 0; j < NP; ++j) {
-        const float ox = __shfl_xor_sync(0xffffffffu, of[g][j].x, off);
-        const float oy = __shfl_xor_sync(0xffffffffu, of[g][j].y, off);
-        of[g][j].x = of[g][j].x * a + ox * c;
-        of[g][j].y = of[g][j].y * a + oy * c;
-      }
-      m[g] = mn;
-    }
-
-  // ---- combine warps through shared memory (the pipeline stages are idle now)
-  float *red_m = reinterpret_cast<float *>(smem);       // [NWARPS][G]
-  float *red_l = red_m + NWARPS * G;                    // [NWARPS][G]
-  float *red_o = red_l + NWARPS * G;                    // [NWARPS][G][D]
-  if (grp == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      if (li == 0) {
-        red_m[warp * G + g] = m[g];
-        red_l[warp * G + g] = l[g];
-      }
-#pragma unroll
-      for (int j = 0; j < NP; ++j) {
-        const int e = chan(li, j);
-        red_o[(warp * G + g) * D + e] = of[g][j].x;
-        red_o[(warp * G + g) * D + e + 1] = of[g][j].y;
-      }
-    }
-  }
-  __syncthreads();
-
+  const float *red_m = reinterpret_cast<const float *>(smem);
+  const float *red_l = red_m + NWARPS * G;
+  const float *red_o = red_l + NWARPS * G;
   const bool direct = !retrieval || P.nsplit == 1;
   T *out = reinterpret_cast<T *>(P.out) + ((int64_t)b * P.Hq + (int64_t)kvh * G) * D;
   const int64_t part = ((int64_t)b * P.n_ret + (retrieval ? pidx : 0)) * P.nsplit + split;
@@ -165,6 +126,61 @@ __device__ __forceinline__ void decode_finish(const DecodeParams &P, uint8_t *sm
     store_out(out + g * D + c, num / s_den[g]);
   }
   if (tid == 0) *cnt = 0u;  // leave the ticket ready for the next call
+}
+
+// State layout expected: each 8-lane group of a warp holds m[g], l[g] and NP
+// fp32 pairs of the output row of query head g; chan(li, j) gives the channel
+// of pair j's first element for lane li of the group.
+template <typename T, int D, int G, int NWARPS, int NP, typename ChanFn>
+__device__ __forceinline__ void decode_finish(const DecodeParams &P, uint8_t *smem, int *s_last_p,
+                                              float (&m)[G], float (&l)[G], float2 (&of)[G][NP],
+                                              ChanFn chan, bool retrieval, int b, int kvh, int pidx,
+                                              int split) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int grp = lane >> 3, li = lane & 7;
+  // ---- combine the four 8-lane groups of each warp
+#pragma unroll
+  for (int off = 8; off <= 16; off <<= 1)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[g], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[g], off);
+      const float mn = fmaxf(m[g], mo);
+      const float a = (m[g] == -INFINITY) ? 0.f : fast_exp2(m[g] - mn);
+      const float c = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
+      l[g] = l[g] * a + lo * c;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        const float ox = __shfl_xor_sync(0xffffffffu, of[g][j].x, off);
+        const float oy = __shfl_xor_sync(0xffffffffu, of[g][j].y, off);
+        of[g][j].x = of[g][j].x * a + ox * c;
+        of[g][j].y = of[g][j].y * a + oy * c;
+      }
+      m[g] = mn;
+    }
+
+  // ---- combine warps through shared memory (the pipeline stages are idle now)
+  float *red_m = reinterpret_cast<float *>(smem);       // [NWARPS][G]
+  float *red_l = red_m + NWARPS * G;                    // [NWARPS][G]
+  float *red_o = red_l + NWARPS * G;                    // [NWARPS][G][D]
+  if (grp == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (li == 0) {
+        red_m[warp * G + g] = m[g];
+        red_l[warp * G + g] = l[g];
+      }
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        const int e = chan(li, j);
+        red_o[(warp * G + g) * D + e] = of[g][j].x;
+        red_o[(warp * G + g) * D + e + 1] = of[g][j].y;
+      }
+    }
+  }
+  __syncthreads();
+
+  decode_reduce_store<T, D, G, NWARPS>(P, smem, s_last_p, retrieval, b, kvh, pidx, split);
 }
 
 }  // namespace duo

@@ -1,0 +1,445 @@
+// Single-token decode attention with warp-level tensor-core MMAs
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate), for head_dim 128 and a bf16
+// or 4-bit KV cache.
+//
+// Same work split as the CUDA-core decode (split-K over retrieval pages, one
+// CTA per streaming slot buffer, last split merges); what changes is the inner
+// product.  Per warp and per 16 keys:
+//   S[16 x 8]  = Q[16 x 128] . K^T      two key tiles of 8, 8 k-steps each
+//   O[16 x 8] += P[16 x 16] . V         one per 8-channel output tile (16)
+// Rows 0..G-1 of the 16-row operands are the G query heads sharing the KV head
+// (the rest are zero).  The accumulator fragment of S is, element for element,
+// the A fragment of P for the next product, so probabilities never leave
+// registers.  Because a dot product does not depend on the order of its terms,
+// the head-dim positions behind each k-slot are chosen so that every thread's
+// B fragment of K is one contiguous 16-byte load of its key row (the query
+// fragment follows the same order), and output channels are assigned so that
+// a thread's V operand comes from 32 contiguous bytes per key.  K and V are
+// loaded straight from global memory into registers; nothing is staged in
+// shared memory except the final cross-warp combine.
+//
+// 4-bit cache: a nibble u becomes the bf16 128 + u by masking it under the bf16
+// pattern of 128 and is then reduced by 128 (exact), and the per-token scale
+// and zero are applied outside the products: s = sc*(q.u) + zp*sum(q),
+// sum p*v_hat = sum (p*sc)*u + (sum p*zp).
+//
+// Pages: "DuoAttention: Efficient Long-Context LLM Inference with Retrieval and
+// Streaming Heads" (hotpaper.ai), abstract and section "기술적 접근법".
+#include "common.cuh"
+#include "decode_finish.cuh"
+
+namespace duo {
+
+namespace dm {
+
+constexpr int D = 128;
+constexpr int NWARPS = 8;
+constexpr int KEYS = 16;               // keys per warp iteration
+constexpr int STEP = NWARPS * KEYS;    // keys per CTA iteration
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1) {
+  // rows g+8 of A are zero (a1 = a3 = 0)
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg128(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint2 ldg64(const void *p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Two 4-bit codes (at bit s and bit s+16 of x) -> bf16x2 of their values.
+__device__ __forceinline__ uint32_t nib2(uint32_t x, int s) {
+  const uint32_t v = ((x >> s) & 0x000F000Fu) | 0x43004300u;  // bf16 128 + u in each half
+  __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&v);
+  h = __hsub2(h, __floats2bfloat162_rn(128.f, 128.f));
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool Q4, int G>
+__global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid_constant__ DecodeParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
+
+  // ---- work item
+  const int n_ret_ctas = P.B * P.n_ret * P.nsplit;
+  int b, kvh, pidx, split;
+  bool retrieval;
+  int64_t row0, k0, k1;
+  const uint8_t *Kb, *Vb, *Ks = nullptr, *Vs = nullptr;
+  if ((int)blockIdx.x < n_ret_ctas) {
+    split = blockIdx.x % P.nsplit;
+    const int r = blockIdx.x / P.nsplit;
+    pidx = r % P.n_ret;
+    b = r / P.n_ret;
+    kvh = P.h.ret_heads[pidx];
+    retrieval = true;
+    row0 = ((int64_t)b * P.n_ret + pidx) * P.cap;
+    Kb = P.p.ret_k;
+    Vb = P.p.ret_v;
+    if (Q4) {
+      Ks = P.p.ret_k_sz;
+      Vs = P.p.ret_v_sz;
+    }
+    k0 = (int64_t)split * P.split_len;
+    k1 = min(P.n, k0 + P.split_len);
+  } else {
+    const int r = blockIdx.x - n_ret_ctas;
+    pidx = r % P.n_str;
+    b = r / P.n_str;
+    kvh = P.h.str_heads[pidx];
+    retrieval = false;
+    split = 0;
+    row0 = ((int64_t)b * P.n_str + pidx) * P.Ws;
+    Kb = P.p.str_k;
+    Vb = P.p.str_v;
+    if (Q4) {
+      Ks = P.p.str_k_sz;
+      Vs = P.p.str_v_sz;
+    }
+    k0 = 0;
+    k1 = min(P.n, (int64_t)P.W);
+  }
+  constexpr int RB = Q4 ? D / 2 : D * 2;  // bytes per key row
+  Kb += row0 * RB;
+  Vb += row0 * RB;
+  if (Q4) {
+    Ks += row0 * 4;
+    Vs += row0 * 4;
+  }
+
+  // ---- query fragments (rows g < G), k-step order matching the K loads
+  uint32_t qa[8][2];
+  float qsum = 0.f;  // sum of the query's channels (4-bit zero-point term)
+  const bool live = g < G;
+  {
+    const __nv_bfloat16 *qrow =
+        reinterpret_cast<const __nv_bfloat16 *>(P.q) + ((int64_t)b * P.Hq + (int64_t)kvh * G + g) * D;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      int c0, c1, c2, c3;  // channels behind k-slots 2t, 2t+1, 2t+8, 2t+9
+      if (Q4) {
+        const int w = k >> 1, tt = k & 1;
+        c0 = 32 * t + 8 * w + 2 * tt;
+        c1 = c0 + 4;
+        c2 = c0 + 1;
+        c3 = c0 + 5;
+      } else {
+        const int s = k >> 1, tt = k & 1;
+        c0 = 32 * s + 8 * t + 4 * tt;
+        c1 = c0 + 1;
+        c2 = c0 + 2;
+        c3 = c0 + 3;
+      }
+      const float q0 = live ? __bfloat162float(qrow[c0]) : 0.f;
+      const float q1 = live ? __bfloat162float(qrow[c1]) : 0.f;
+      const float q2 = live ? __bfloat162float(qrow[c2]) : 0.f;
+      const float q3 = live ? __bfloat162float(qrow[c3]) : 0.f;
+      qa[k][0] = pack_bf16(q0, q1);  // exact: the inputs are bf16
+      qa[k][1] = pack_bf16(q2, q3);
+      qsum += (q0 + q1) + (q2 + q3);
+    }
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+  }
+  const float sl2 = P.scale_log2;
+
+  // O^T accumulators: tile mt holds channels 16g + 2mt (rows g) and
+  // 16g + 2mt + 1 (rows g+8) for queries 2t and 2t+1.
+  float o[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  // softmax state of query g (identical in the four threads of a row)
+  float m = -INFINITY, l = 0.f, z = 0.f;
+
+  for (int64_t kb = k0 + (int64_t)warp * KEYS; kb < k1; kb += STEP) {
+    // ------------------------------------------------------------ loads (all up front)
+    // K: key kb + 8*nt + g (this thread's column of S); V: keys kA..kD behind
+    // the k-slots 2t, 2t+1, 2t+8, 2t+9 of the P^T fragment, channels [16g, 16g+16).
+    const int64_t kA = kb + 2 * t, kB = kA + 1, kC = kA + 8, kD = kA + 9;
+    uint4 kr[2][Q4 ? 1 : 4];
+    uint2 ksz[2], vsz[2];
+    uint4 vr[4][Q4 ? 1 : 2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int64_t key = kb + 8 * nt + g;
+      const bool ok = key < k1;
+      if (Q4) {
+        kr[nt][0] = ok ? ldg128(Kb + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
+      } else {
+#pragma unroll
+        for (int sp = 0; sp < 4; ++sp)
+          kr[nt][sp] = ok ? ldg128(Kb + key * RB + (32 * sp + 8 * t) * 2) : make_uint4(0, 0, 0, 0);
+      }
+      if (Q4) {
+        const int64_t key2 = kb + 8 * nt + 2 * t;
+        ksz[nt] = key2 < k1 ? ldg64(Ks + key2 * 4) : make_uint2(0, 0);
+        vsz[nt] = key2 < k1 ? ldg64(Vs + key2 * 4) : make_uint2(0, 0);
+      }
+    }
+    {
+      const int64_t keys[4] = {kA, kB, kC, kD};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool ok = keys[i] < k1;
+        if (Q4) {
+          const uint2 x = ok ? ldg64(Vb + keys[i] * RB + 8 * g) : make_uint2(0, 0);
+          vr[i][0] = make_uint4(x.x, x.y, 0, 0);
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            vr[i][h] = ok ? ldg128(Vb + keys[i] * RB + 32 * g + 16 * h) : make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+    // ------------------------------------------------------------ S = Q K^T
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+      if (Q4) {
+        const uint32_t w4[4] = {kr[nt][0].x, kr[nt][0].y, kr[nt][0].z, kr[nt][0].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          mma16816(s[nt], qa[2 * w][0], qa[2 * w][1], nib2(w4[w], 0), nib2(w4[w], 4));
+          mma16816(s[nt], qa[2 * w + 1][0], qa[2 * w + 1][1], nib2(w4[w], 8), nib2(w4[w], 12));
+        }
+      } else {
+#pragma unroll
+        for (int sp = 0; sp < 4; ++sp) {
+          mma16816(s[nt], qa[2 * sp][0], qa[2 * sp][1], kr[nt][sp].x, kr[nt][sp].y);
+          mma16816(s[nt], qa[2 * sp + 1][0], qa[2 * sp + 1][1], kr[nt][sp].z, kr[nt][sp].w);
+        }
+      }
+    }
+    // scores of query g at keys kb + 8*nt + 2t + e
+    float sc[2][2], vscale[2][2], vzero[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int64_t key = kb + 8 * nt + 2 * t;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float raw = s[nt][e];
+        vscale[nt][e] = 1.f;
+        vzero[nt][e] = 0.f;
+        if (Q4) {
+          const __half2 kp = *reinterpret_cast<const __half2 *>(e ? &ksz[nt].y : &ksz[nt].x);
+          const __half2 vp = *reinterpret_cast<const __half2 *>(e ? &vsz[nt].y : &vsz[nt].x);
+          raw = __low2float(kp) * raw + __high2float(kp) * qsum;
+          vscale[nt][e] = __low2float(vp);
+          vzero[nt][e] = __high2float(vp);
+        }
+        sc[nt][e] = (live && key + e < k1) ? raw * sl2 : -INFINITY;
+      }
+    }
+    // ------------------------------------------------------------ online softmax
+    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    // Rescale only when the running max grows by more than 2^8 (numerator and
+    // denominator scale together, so the result is unchanged).
+    const bool grow = mx > m + 8.f || (m == -INFINITY && mx > -INFINITY);
+    float alpha = 1.f;
+    if (grow) {
+      alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
+      l *= alpha;
+      z *= alpha;
+      m = mx;
+    }
+    if (__any_sync(0xffffffffu, grow)) {
+      // O^T columns are queries 2t and 2t+1: take their factors from the
+      // threads that own those rows of S.
+      const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * t) << 2);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) << 2);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i][0] *= a0;
+        o[i][2] *= a0;
+        o[i][1] *= a1;
+        o[i][3] *= a1;
+      }
+    }
+    float p[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        p[nt][e] = (sc[nt][e] == -INFINITY) ? 0.f : fast_exp2(sc[nt][e] - m);
+        l += p[nt][e];
+        if (Q4) {
+          z += p[nt][e] * vzero[nt][e];
+          p[nt][e] *= vscale[nt][e];
+        }
+      }
+    // P^T fragment: b0 = keys 2t, 2t+1 (tile 0), b1 = keys 8+2t, 9+2t (tile 1)
+    const uint32_t pb0 = pack_bf16(p[0][0], p[0][1]);
+    const uint32_t pb1 = pack_bf16(p[1][0], p[1][1]);
+    // 4-bit cache: p*sc multiplies codes up to 15 whose sum is offset by the
+    // zero point, so bf16's 8-bit mantissa alone is too coarse; the residual
+    // p*sc - bf16(p*sc) goes through a second product (16 mantissa bits).
+    uint32_t pl0 = 0u, pl1 = 0u;
+    if (Q4) {
+      const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162 *>(&pb0);
+      const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162 *>(&pb1);
+      pl0 = pack_bf16(p[0][0] - __low2float(h0), p[0][1] - __high2float(h0));
+      pl1 = pack_bf16(p[1][0] - __low2float(h1), p[1][1] - __high2float(h1));
+    }
+    // ------------------------------------------------------------ O^T += V^T P^T
+    if (Q4) {
+#pragma unroll
+      for (int wi = 0; wi < 2; ++wi) {
+        const uint32_t xa = wi ? vr[0][0].y : vr[0][0].x, xb = wi ? vr[1][0].y : vr[1][0].x;
+        const uint32_t xc = wi ? vr[2][0].y : vr[2][0].x, xd = wi ? vr[3][0].y : vr[3][0].x;
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+          const uint32_t sel = j ? 0x7632u : 0x5410u;
+          const uint32_t ab = __byte_perm(xa, xb, sel);  // [A_j, A_j+1, B_j, B_j+1]
+          const uint32_t cd = __byte_perm(xc, xd, sel);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int mt = 4 * wi + j + h;  // code byte 8g + mt: channels 16g + 2mt, +1
+            const uint32_t a0 = nib2(ab, 8 * h), a1 = nib2(ab, 8 * h + 4);
+            const uint32_t a2 = nib2(cd, 8 * h), a3 = nib2(cd, 8 * h + 4);
+            mma16816_full(o[mt], a0, a1, a2, a3, pb0, pb1);
+            mma16816_full(o[mt], a0, a1, a2, a3, pl0, pl1);
+          }
+        }
+      }
+    } else {
+      const uint32_t wa[8] = {vr[0][0].x, vr[0][0].y, vr[0][0].z, vr[0][0].w,
+                              vr[0][1].x, vr[0][1].y, vr[0][1].z, vr[0][1].w};
+      const uint32_t wb[8] = {vr[1][0].x, vr[1][0].y, vr[1][0].z, vr[1][0].w,
+                              vr[1][1].x, vr[1][1].y, vr[1][1].z, vr[1][1].w};
+      const uint32_t wc[8] = {vr[2][0].x, vr[2][0].y, vr[2][0].z, vr[2][0].w,
+                              vr[2][1].x, vr[2][1].y, vr[2][1].z, vr[2][1].w};
+      const uint32_t wd[8] = {vr[3][0].x, vr[3][0].y, vr[3][0].z, vr[3][0].w,
+                              vr[3][1].x, vr[3][1].y, vr[3][1].z, vr[3][1].w};
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)  // word mt holds channels 16g + 2mt, +1
+        mma16816_full(o[mt], __byte_perm(wa[mt], wb[mt], 0x5410u), __byte_perm(wa[mt], wb[mt], 0x7632u),
+                      __byte_perm(wc[mt], wd[mt], 0x5410u), __byte_perm(wc[mt], wd[mt], 0x7632u), pb0,
+                      pb1);
+    }
+  }
+
+  // ---- per-warp state -> shared memory (queries < G only)
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  if (Q4) {
+    z += __shfl_xor_sync(0xffffffffu, z, 1);
+    z += __shfl_xor_sync(0xffffffffu, z, 2);
+  }
+  float *red_m = reinterpret_cast<float *>(smem);
+  float *red_l = red_m + NWARPS * G;
+  float *red_o = red_l + NWARPS * G;
+  // the zero-point sums of this thread's two O^T columns (queries 2t, 2t+1)
+  const float z0 = __shfl_sync(0xffffffffu, z, (2 * t) << 2);
+  const float z1 = __shfl_sync(0xffffffffu, z, (2 * t + 1) << 2);
+  if (live && t == 0) {
+    red_m[warp * G + g] = m;
+    red_l[warp * G + g] = l;
+  }
+  const int q0 = 2 * t, q1 = 2 * t + 1;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int ch = 16 * g + 2 * mt;
+    if (q0 < G) {
+      red_o[(warp * G + q0) * D + ch] = o[mt][0] + z0;
+      red_o[(warp * G + q0) * D + ch + 1] = o[mt][2] + z0;
+    }
+    if (q1 < G) {
+      red_o[(warp * G + q1) * D + ch] = o[mt][1] + z1;
+      red_o[(warp * G + q1) * D + ch + 1] = o[mt][3] + z1;
+    }
+  }
+  __syncthreads();
+  decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(P, smem, &s_last, retrieval, b, kvh, pidx, split);
+}
+
+template <bool Q4, int G>
+cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
+  auto kern = decode_mma_kernel<Q4, G>;
+  // staging: 2*NWARPS*G + NWARPS*G*D floats; merge: nsplit*G + G (+align) + NWARPS*G*D floats
+  const int smem = (int)sizeof(float) * (kMaxSplits * G + 8 + NWARPS * G * D + 2 * NWARPS * G);
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  if (cfg) {
+    int occ = 0, dev = 0, sms = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NWARPS * 32, smem);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cfg->tile_rows = STEP;
+    cfg->ctas_per_sm = occ;
+    cfg->num_sms = sms;
+    return cudaSuccess;
+  }
+  const int grid = d.B * d.n_ret * d.nsplit + d.B * d.n_str;
+  if (grid == 0) return cudaSuccess;
+  kern<<<grid, NWARPS * 32, smem, s>>>(d);
+  return cudaGetLastError();
+}
+
+template <bool Q4>
+cudaError_t dispatch(const DecodeParams &d, int G, cudaStream_t s, DecodeConfig *cfg) {
+  switch (G) {
+    case 1: return run<Q4, 1>(d, s, cfg);
+    case 2: return run<Q4, 2>(d, s, cfg);
+    case 4: return run<Q4, 4>(d, s, cfg);
+    case 8: return run<Q4, 8>(d, s, cfg);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dm
+
+// head_dim 128, bf16 or 4-bit cache: the tensor-core decode.
+bool decode_mma_supported(int kv_type, int D, int G) {
+  return D == 128 && (kv_type == kBF16 || kv_type == kINT4) && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
+cudaError_t decode_mma_config(int kv_type, int G, DecodeConfig *cfg) {
+  DecodeParams dummy{};
+  return kv_type == kINT4 ? dm::dispatch<true>(dummy, G, nullptr, cfg)
+                          : dm::dispatch<false>(dummy, G, nullptr, cfg);
+}
+
+cudaError_t launch_decode_mma(const DecodeParams &d, int kv_type, cudaStream_t s) {
+  return kv_type == kINT4 ? dm::dispatch<true>(d, d.G, s, nullptr)
+                          : dm::dispatch<false>(d, d.G, s, nullptr);
+}
+
+}  // namespace duo
