@@ -209,17 +209,27 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K * w.layers)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K * w.layers)]
 
+    # bf16 head_dim-128 caches decode each layer in one fused launch
+    # (duo_decode_step: append + attend); other caches append, then attend.
+    fused = w.kv_dtype == "bf16" and w.head_dim == 128
+
     def step(s, timed_idx=None):
         for layer in range(w.layers):
-            st = lib.duo_append_kv(h, layer, ks[layer][s].data_ptr(), vs[layer][s].data_ptr(), 1, sh)
-            if st:
-                raise B.DuoError(st, "duo_append_kv")
+            kp, vp = ks[layer][s].data_ptr(), vs[layer][s].data_ptr()
+            if not fused:
+                st = lib.duo_append_kv(h, layer, kp, vp, 1, sh)
+                if st:
+                    raise B.DuoError(st, "duo_append_kv")
             if timed_idx is not None:
                 ev_s[timed_idx * w.layers + layer].record(stream)
-            st = lib.duo_decode_attn(h, layer, qs[layer][s].data_ptr(), outs[layer].data_ptr(),
-                                     0.0, ws, wsb, sh)
+            if fused:
+                st = lib.duo_decode_step(h, layer, qs[layer][s].data_ptr(), kp, vp,
+                                         outs[layer].data_ptr(), 0.0, ws, wsb, sh)
+            else:
+                st = lib.duo_decode_attn(h, layer, qs[layer][s].data_ptr(), outs[layer].data_ptr(),
+                                         0.0, ws, wsb, sh)
             if st:
-                raise B.DuoError(st, "duo_decode_attn")
+                raise B.DuoError(st, "duo_decode_step" if fused else "duo_decode_attn")
             if timed_idx is not None:
                 ev_e[timed_idx * w.layers + layer].record(stream)
 
@@ -251,7 +261,8 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
         n = n_first + i
         for layer in range(w.layers):
             lb = decode_bytes_per_layer(w, batch, n, n_ret[layer], n_str[layer])
-            launch_bytes.append(lb)
+            # the fused launch also reads the new K/V and writes them to the cache
+            launch_bytes.append(lb + (append_bytes(w, batch) if fused else 0))
             step_bytes += lb + append_bytes(w, batch)
     step_bytes /= K
 
@@ -275,8 +286,13 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
             dq[layer].copy_(host_q[layer][i], non_blocking=True)
             dk[layer].copy_(host_k[layer][i], non_blocking=True)
             dv[layer].copy_(host_v[layer][i], non_blocking=True)
-            B.duo_append_kv(h, layer, dk[layer].data_ptr(), dv[layer].data_ptr(), 1, sh)
-            B.duo_decode_attn(h, layer, dq[layer].data_ptr(), outs[layer].data_ptr(), 0.0, ws, wsb, sh)
+            if fused:
+                B.duo_decode_step(h, layer, dq[layer].data_ptr(), dk[layer].data_ptr(),
+                                  dv[layer].data_ptr(), outs[layer].data_ptr(), 0.0, ws, wsb, sh)
+            else:
+                B.duo_append_kv(h, layer, dk[layer].data_ptr(), dv[layer].data_ptr(), 1, sh)
+                B.duo_decode_attn(h, layer, dq[layer].data_ptr(), outs[layer].data_ptr(), 0.0, ws,
+                                  wsb, sh)
             host_o[layer][i].copy_(outs[layer], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -292,13 +308,14 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
         "e2e_value": aggregate_rate(step_bytes, world, K, e2e_ms),
         "h2d": h2d, "d2h": d2h,
         "step_bytes": step_bytes,
-        "kernel": {"name": "decode_kernel", "avg_ms": avg_kern_ms, "launches": len(kern_ms),
+        "kernel": {"name": "decode_mma_kernel (fused append + attention)" if fused else
+                   "decode_mma_kernel", "avg_ms": avg_kern_ms, "launches": len(kern_ms),
                    "bytes_per_launch": avg_launch_bytes, "achieved_gbs": achieved},
         "splits": splits,
         "fill_s": fill_s,
         "clocks": clk.summary(),
         "context": n_first,
-        "gpu_launches": K * w.layers * 2,
+        "gpu_launches": K * w.layers * (1 if fused else 2),
     }
     del cache
     torch.cuda.empty_cache()

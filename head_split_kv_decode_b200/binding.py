@@ -73,6 +73,7 @@ SIGNATURES = {
     "duo_cache_reset": (_I32, [_P]),
     "duo_append_kv": (_I32, [_P, _I32, _P, _P, _I32, _P]),
     "duo_decode_attn": (_I32, [_P, _I32, _P, _P, _F, _P, _SZ, _P]),
+    "duo_decode_step": (_I32, [_P, _I32, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "duo_decode_attn_static": (_I32, [_P, _I32, _P, _P, _F, _P]),
     "duo_prefill_attn": (_I32, [_P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
     "duo_seq_len": (_I32, [_P, _I32, ctypes.POINTER(_I64)]),
@@ -154,6 +155,12 @@ def duo_append_kv(handle, layer, k_ptr, v_ptr, n_tokens, stream=0):
 def duo_decode_attn(handle, layer, q_ptr, out_ptr, softmax_scale, ws_ptr, ws_bytes, stream=0):
     _check(lib().duo_decode_attn(handle, layer, q_ptr, out_ptr, softmax_scale, ws_ptr,
                                  ws_bytes, stream), "duo_decode_attn")
+
+
+def duo_decode_step(handle, layer, q_ptr, k_new_ptr, v_new_ptr, out_ptr, softmax_scale, ws_ptr,
+                    ws_bytes, stream=0):
+    _check(lib().duo_decode_step(handle, layer, q_ptr, k_new_ptr, v_new_ptr, out_ptr, softmax_scale,
+                                 ws_ptr, ws_bytes, stream), "duo_decode_step")
 
 
 def duo_decode_attn_static(handle, layer, q_ptr, out_ptr, softmax_scale, stream=0):

@@ -86,6 +86,22 @@ class DuoCache:
                           self.ws_ptr, self.ws_bytes, _stream_handle(stream, self.device))
         return out
 
+    def step(self, layer, q, k_new, v_new, out=None, scale=0.0, stream=None):
+        """Append one token (k_new, v_new: [batch, n_kv_heads, head_dim]) and
+        attend with q at its position, in one launch where possible."""
+        kv_shape = (self.batch, self.n_kv_heads, self.head_dim)
+        shape = (self.batch, self.n_q_heads, self.head_dim)
+        self._check(q, shape, "q")
+        self._check(k_new, kv_shape, "k_new")
+        self._check(v_new, kv_shape, "v_new")
+        if out is None:
+            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
+        self._check(out, shape, "out")
+        B.duo_decode_step(self.handle, layer, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
+                          out.data_ptr(), float(scale), self.ws_ptr, self.ws_bytes,
+                          _stream_handle(stream, self.device))
+        return out
+
     def prefill(self, layer, q, k, v, out=None, scale=0.0, stream=None):
         """q: [batch, C, n_q_heads, d]; k, v: [batch, C, n_kv_heads, d].  Attends only."""
         C = q.shape[1]

@@ -34,8 +34,13 @@ namespace dm {
 
 constexpr int D = 128;
 constexpr int NWARPS = 8;
-constexpr int KEYS = 16;               // keys per warp iteration
-constexpr int STEP = NWARPS * KEYS;    // keys per CTA iteration
+// Key groups of 16 per warp iteration: the 4-bit rows are 4x smaller, so a
+// warp takes two groups to keep as many bytes in flight as the bf16 path.
+template <bool Q4>
+struct Keys {
+  static constexpr int KG = Q4 ? 2 : 1;
+  static constexpr int STEP = NWARPS * 16 * KG;  // keys per CTA iteration
+};
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
                                          uint32_t b1) {
@@ -66,12 +71,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Two 4-bit codes (at bit s and bit s+16 of x) -> bf16x2 of their values.
+// Two 4-bit codes u (at bit s and bit s+16 of x) -> bf16x2 of 128 + u (exact):
+// the code is masked under the bit pattern of 128.0, whose mantissa is zero.
+// The offset of 128 is removed after the products (see the callers).
 __device__ __forceinline__ uint32_t nib2(uint32_t x, int s) {
-  const uint32_t v = ((x >> s) & 0x000F000Fu) | 0x43004300u;  // bf16 128 + u in each half
-  __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&v);
-  h = __hsub2(h, __floats2bfloat162_rn(128.f, 128.f));
-  return *reinterpret_cast<uint32_t *>(&h);
+  return ((x >> s) & 0x000F000Fu) | 0x43004300u;
 }
 
 __device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -136,6 +140,24 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
     Ks += row0 * 4;
     Vs += row0 * 4;
   }
+  // Launched with programmatic dependent launch: everything above overlapped
+  // the previous kernel; nothing it may have written is read before this.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // Fused append (bf16 cache): the token at position n-1 is not in the cache
+  // yet.  The CTA whose key range holds its row writes it there, skips that
+  // row in the main pass, and adds it in a one-key pass that reads the inputs.
+  const bool fused = !Q4 && P.knew != nullptr;
+  const int64_t newk = retrieval ? P.n - 1 : P.new_slot;  // its row in this head's buffer
+  const bool owns_new = fused && newk >= k0 && newk < k1;
+  if (owns_new && warp == 0) {
+    const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB;
+    const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + off;
+    uint8_t *dst = const_cast<uint8_t *>(lane < 16 ? Kb : Vb) + newk * RB;
+    reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
+  }
+  const int64_t skip = owns_new ? newk : -1;
 
   // ---- query fragments (rows g < G), k-step order matching the K loads
   uint32_t qa[8][2];
@@ -178,91 +200,100 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   float o[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  // softmax state of query g (identical in the four threads of a row)
-  float m = -INFINITY, l = 0.f, z = 0.f;
+  // softmax state of query g (identical in the four threads of a row); for the
+  // 4-bit cache z = sum p*zp and cs = sum p*sc (as multiplied, see below)
+  float m = -INFINITY, l = 0.f, z = 0.f, cs = 0.f;
 
-  for (int64_t kb = k0 + (int64_t)warp * KEYS; kb < k1; kb += STEP) {
+  constexpr int KG = Keys<Q4>::KG;
+  // Keys [lo, hi) of the buffers Kx/Vx (row index = key), except `skip`.
+  auto pass = [&](const uint8_t *Kx, const uint8_t *Vx, int64_t lo, int64_t hi, int64_t skip_key) {
+  for (int64_t kb0 = lo + (int64_t)warp * 16 * KG; kb0 < hi; kb0 += Keys<Q4>::STEP) {
     // ------------------------------------------------------------ loads (all up front)
-    // K: key kb + 8*nt + g (this thread's column of S); V: keys kA..kD behind
-    // the k-slots 2t, 2t+1, 2t+8, 2t+9 of the P^T fragment, channels [16g, 16g+16).
-    const int64_t kA = kb + 2 * t, kB = kA + 1, kC = kA + 8, kD = kA + 9;
-    uint4 kr[2][Q4 ? 1 : 4];
-    uint2 ksz[2], vsz[2];
-    uint4 vr[4][Q4 ? 1 : 2];
+    // group kg covers keys kb = kb0 + 16*kg ..: K of key kb + 8*nt + g (this
+    // thread's column of S); V of keys kb + {2t, 2t+1, 8+2t, 9+2t} (the k-slots
+    // of the P^T fragment), channels [16g, 16g+16).
+    uint4 kr[KG][2][Q4 ? 1 : 4];
+    uint2 ksz[KG][2], vsz[KG][2];
+    uint4 vr[KG][4][Q4 ? 1 : 2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int64_t key = kb + 8 * nt + g;
-      const bool ok = key < k1;
-      if (Q4) {
-        kr[nt][0] = ok ? ldg128(Kb + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
-      } else {
+    for (int kg = 0; kg < KG; ++kg) {
+      const int64_t kb = kb0 + 16 * kg;
 #pragma unroll
-        for (int sp = 0; sp < 4; ++sp)
-          kr[nt][sp] = ok ? ldg128(Kb + key * RB + (32 * sp + 8 * t) * 2) : make_uint4(0, 0, 0, 0);
+      for (int nt = 0; nt < 2; ++nt) {
+        const int64_t key = kb + 8 * nt + g;
+        const bool ok = key < hi && key != skip_key;
+        if (Q4) {
+          kr[kg][nt][0] = ok ? ldg128(Kb + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
+          const int64_t key2 = kb + 8 * nt + 2 * t;
+          ksz[kg][nt] = key2 < hi ? ldg64(Ks + key2 * 4) : make_uint2(0, 0);
+          vsz[kg][nt] = key2 < hi ? ldg64(Vs + key2 * 4) : make_uint2(0, 0);
+        } else {
+#pragma unroll
+          for (int sp = 0; sp < 4; ++sp)
+            kr[kg][nt][sp] = ok ? ldg128(Kx + key * RB + (32 * sp + 8 * t) * 2) : make_uint4(0, 0, 0, 0);
+        }
       }
-      if (Q4) {
-        const int64_t key2 = kb + 8 * nt + 2 * t;
-        ksz[nt] = key2 < k1 ? ldg64(Ks + key2 * 4) : make_uint2(0, 0);
-        vsz[nt] = key2 < k1 ? ldg64(Vs + key2 * 4) : make_uint2(0, 0);
-      }
-    }
-    {
-      const int64_t keys[4] = {kA, kB, kC, kD};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const bool ok = keys[i] < k1;
+        const int64_t key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
+        const bool ok = key < hi && key != skip_key;
         if (Q4) {
-          const uint2 x = ok ? ldg64(Vb + keys[i] * RB + 8 * g) : make_uint2(0, 0);
-          vr[i][0] = make_uint4(x.x, x.y, 0, 0);
+          const uint2 x = ok ? ldg64(Vb + key * RB + 8 * g) : make_uint2(0, 0);
+          vr[kg][i][0] = make_uint4(x.x, x.y, 0, 0);
         } else {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            vr[i][h] = ok ? ldg128(Vb + keys[i] * RB + 32 * g + 16 * h) : make_uint4(0, 0, 0, 0);
+            vr[kg][i][h] = ok ? ldg128(Vx + key * RB + 32 * g + 16 * h) : make_uint4(0, 0, 0, 0);
         }
       }
     }
     // ------------------------------------------------------------ S = Q K^T
-    float s[2][4];
+    float sc[KG][2][2], vscale[KG][2][2], vzero[KG][2][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-      if (Q4) {
-        const uint32_t w4[4] = {kr[nt][0].x, kr[nt][0].y, kr[nt][0].z, kr[nt][0].w};
+    for (int kg = 0; kg < KG; ++kg) {
+      const int64_t kb = kb0 + 16 * kg;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          mma16816(s[nt], qa[2 * w][0], qa[2 * w][1], nib2(w4[w], 0), nib2(w4[w], 4));
-          mma16816(s[nt], qa[2 * w + 1][0], qa[2 * w + 1][1], nib2(w4[w], 8), nib2(w4[w], 12));
-        }
-      } else {
-#pragma unroll
-        for (int sp = 0; sp < 4; ++sp) {
-          mma16816(s[nt], qa[2 * sp][0], qa[2 * sp][1], kr[nt][sp].x, kr[nt][sp].y);
-          mma16816(s[nt], qa[2 * sp + 1][0], qa[2 * sp + 1][1], kr[nt][sp].z, kr[nt][sp].w);
-        }
-      }
-    }
-    // scores of query g at keys kb + 8*nt + 2t + e
-    float sc[2][2], vscale[2][2], vzero[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int64_t key = kb + 8 * nt + 2 * t;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float raw = s[nt][e];
-        vscale[nt][e] = 1.f;
-        vzero[nt][e] = 0.f;
+      for (int nt = 0; nt < 2; ++nt) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
         if (Q4) {
-          const __half2 kp = *reinterpret_cast<const __half2 *>(e ? &ksz[nt].y : &ksz[nt].x);
-          const __half2 vp = *reinterpret_cast<const __half2 *>(e ? &vsz[nt].y : &vsz[nt].x);
-          raw = __low2float(kp) * raw + __high2float(kp) * qsum;
-          vscale[nt][e] = __low2float(vp);
-          vzero[nt][e] = __high2float(vp);
+          const uint32_t w4[4] = {kr[kg][nt][0].x, kr[kg][nt][0].y, kr[kg][nt][0].z, kr[kg][nt][0].w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            mma16816(s, qa[2 * w][0], qa[2 * w][1], nib2(w4[w], 0), nib2(w4[w], 4));
+            mma16816(s, qa[2 * w + 1][0], qa[2 * w + 1][1], nib2(w4[w], 8), nib2(w4[w], 12));
+          }
+        } else {
+#pragma unroll
+          for (int sp = 0; sp < 4; ++sp) {
+            mma16816(s, qa[2 * sp][0], qa[2 * sp][1], kr[kg][nt][sp].x, kr[kg][nt][sp].y);
+            mma16816(s, qa[2 * sp + 1][0], qa[2 * sp + 1][1], kr[kg][nt][sp].z, kr[kg][nt][sp].w);
+          }
         }
-        sc[nt][e] = (live && key + e < k1) ? raw * sl2 : -INFINITY;
+        // scores of query g at keys kb + 8*nt + 2t + e
+        const int64_t key = kb + 8 * nt + 2 * t;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float raw = s[e];
+          vscale[kg][nt][e] = 1.f;
+          vzero[kg][nt][e] = 0.f;
+          if (Q4) {
+            const __half2 kp = *reinterpret_cast<const __half2 *>(e ? &ksz[kg][nt].y : &ksz[kg][nt].x);
+            const __half2 vp = *reinterpret_cast<const __half2 *>(e ? &vsz[kg][nt].y : &vsz[kg][nt].x);
+            // q.(128 + u) = q.u + 128*sum(q):  s = sc*q.u + zp*sum(q)
+            const float ksc = __low2float(kp);
+            raw = ksc * raw + (__high2float(kp) - 128.f * ksc) * qsum;
+            vscale[kg][nt][e] = __low2float(vp);
+            vzero[kg][nt][e] = __high2float(vp);
+          }
+          sc[kg][nt][e] = (live && key + e < hi && key + e != skip_key) ? raw * sl2 : -INFINITY;
+        }
       }
     }
     // ------------------------------------------------------------ online softmax
-    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    float mx = -INFINITY;
+#pragma unroll
+    for (int kg = 0; kg < KG; ++kg)
+      mx = fmaxf(mx, fmaxf(fmaxf(sc[kg][0][0], sc[kg][0][1]), fmaxf(sc[kg][1][0], sc[kg][1][1])));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     // Rescale only when the running max grows by more than 2^8 (numerator and
@@ -273,6 +304,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
       alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
       l *= alpha;
       z *= alpha;
+      cs *= alpha;
       m = mx;
     }
     if (__any_sync(0xffffffffu, grow)) {
@@ -288,68 +320,85 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
         o[i][3] *= a1;
       }
     }
-    float p[2][2];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int kg = 0; kg < KG; ++kg) {
+      float p[2][2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        p[nt][e] = (sc[nt][e] == -INFINITY) ? 0.f : fast_exp2(sc[nt][e] - m);
-        l += p[nt][e];
-        if (Q4) {
-          z += p[nt][e] * vzero[nt][e];
-          p[nt][e] *= vscale[nt][e];
-        }
-      }
-    // P^T fragment: b0 = keys 2t, 2t+1 (tile 0), b1 = keys 8+2t, 9+2t (tile 1)
-    const uint32_t pb0 = pack_bf16(p[0][0], p[0][1]);
-    const uint32_t pb1 = pack_bf16(p[1][0], p[1][1]);
-    // 4-bit cache: p*sc multiplies codes up to 15 whose sum is offset by the
-    // zero point, so bf16's 8-bit mantissa alone is too coarse; the residual
-    // p*sc - bf16(p*sc) goes through a second product (16 mantissa bits).
-    uint32_t pl0 = 0u, pl1 = 0u;
-    if (Q4) {
-      const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162 *>(&pb0);
-      const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162 *>(&pb1);
-      pl0 = pack_bf16(p[0][0] - __low2float(h0), p[0][1] - __high2float(h0));
-      pl1 = pack_bf16(p[1][0] - __low2float(h1), p[1][1] - __high2float(h1));
-    }
-    // ------------------------------------------------------------ O^T += V^T P^T
-    if (Q4) {
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int wi = 0; wi < 2; ++wi) {
-        const uint32_t xa = wi ? vr[0][0].y : vr[0][0].x, xb = wi ? vr[1][0].y : vr[1][0].x;
-        const uint32_t xc = wi ? vr[2][0].y : vr[2][0].x, xd = wi ? vr[3][0].y : vr[3][0].x;
-#pragma unroll
-        for (int j = 0; j < 4; j += 2) {
-          const uint32_t sel = j ? 0x7632u : 0x5410u;
-          const uint32_t ab = __byte_perm(xa, xb, sel);  // [A_j, A_j+1, B_j, B_j+1]
-          const uint32_t cd = __byte_perm(xc, xd, sel);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int mt = 4 * wi + j + h;  // code byte 8g + mt: channels 16g + 2mt, +1
-            const uint32_t a0 = nib2(ab, 8 * h), a1 = nib2(ab, 8 * h + 4);
-            const uint32_t a2 = nib2(cd, 8 * h), a3 = nib2(cd, 8 * h + 4);
-            mma16816_full(o[mt], a0, a1, a2, a3, pb0, pb1);
-            mma16816_full(o[mt], a0, a1, a2, a3, pl0, pl1);
+        for (int e = 0; e < 2; ++e) {
+          p[nt][e] = (sc[kg][nt][e] == -INFINITY) ? 0.f : fast_exp2(sc[kg][nt][e] - m);
+          l += p[nt][e];
+          if (Q4) {
+            z += p[nt][e] * vzero[kg][nt][e];
+            p[nt][e] *= vscale[kg][nt][e];
           }
         }
+      // P^T fragment: b0 = keys 2t, 2t+1 (tile 0), b1 = keys 8+2t, 9+2t (tile 1)
+      const uint32_t pb0 = pack_bf16(p[0][0], p[0][1]);
+      const uint32_t pb1 = pack_bf16(p[1][0], p[1][1]);
+      // 4-bit cache: p*sc multiplies codes up to 15 whose sum is offset by the
+      // zero point, so bf16's 8-bit mantissa alone is too coarse; the residual
+      // p*sc - bf16(p*sc) goes through a second product (16 mantissa bits).
+      uint32_t pl0 = 0u, pl1 = 0u;
+      if (Q4) {
+        const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162 *>(&pb0);
+        const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162 *>(&pb1);
+        pl0 = pack_bf16(p[0][0] - __low2float(h0), p[0][1] - __high2float(h0));
+        pl1 = pack_bf16(p[1][0] - __low2float(h1), p[1][1] - __high2float(h1));
+        // The V codes enter as 128 + u: remember exactly what was multiplied
+        // so that 128 * sum(p*sc) can be removed from O afterwards.
+        const __nv_bfloat162 l0 = *reinterpret_cast<const __nv_bfloat162 *>(&pl0);
+        const __nv_bfloat162 l1 = *reinterpret_cast<const __nv_bfloat162 *>(&pl1);
+        cs += ((__low2float(h0) + __low2float(l0)) + (__high2float(h0) + __high2float(l0))) +
+              ((__low2float(h1) + __low2float(l1)) + (__high2float(h1) + __high2float(l1)));
       }
-    } else {
-      const uint32_t wa[8] = {vr[0][0].x, vr[0][0].y, vr[0][0].z, vr[0][0].w,
-                              vr[0][1].x, vr[0][1].y, vr[0][1].z, vr[0][1].w};
-      const uint32_t wb[8] = {vr[1][0].x, vr[1][0].y, vr[1][0].z, vr[1][0].w,
-                              vr[1][1].x, vr[1][1].y, vr[1][1].z, vr[1][1].w};
-      const uint32_t wc[8] = {vr[2][0].x, vr[2][0].y, vr[2][0].z, vr[2][0].w,
-                              vr[2][1].x, vr[2][1].y, vr[2][1].z, vr[2][1].w};
-      const uint32_t wd[8] = {vr[3][0].x, vr[3][0].y, vr[3][0].z, vr[3][0].w,
-                              vr[3][1].x, vr[3][1].y, vr[3][1].z, vr[3][1].w};
+      // ---------------------------------------------------------- O^T += V^T P^T
+      if (Q4) {
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt)  // word mt holds channels 16g + 2mt, +1
-        mma16816_full(o[mt], __byte_perm(wa[mt], wb[mt], 0x5410u), __byte_perm(wa[mt], wb[mt], 0x7632u),
-                      __byte_perm(wc[mt], wd[mt], 0x5410u), __byte_perm(wc[mt], wd[mt], 0x7632u), pb0,
-                      pb1);
+        for (int wi = 0; wi < 2; ++wi) {
+          const uint32_t xa = wi ? vr[kg][0][0].y : vr[kg][0][0].x, xb = wi ? vr[kg][1][0].y : vr[kg][1][0].x;
+          const uint32_t xc = wi ? vr[kg][2][0].y : vr[kg][2][0].x, xd = wi ? vr[kg][3][0].y : vr[kg][3][0].x;
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            const uint32_t sel = j ? 0x7632u : 0x5410u;
+            const uint32_t ab = __byte_perm(xa, xb, sel);  // [A_j, A_j+1, B_j, B_j+1]
+            const uint32_t cd = __byte_perm(xc, xd, sel);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int mt = 4 * wi + j + h;  // code byte 8g + mt: channels 16g + 2mt, +1
+              const uint32_t a0 = nib2(ab, 8 * h), a1 = nib2(ab, 8 * h + 4);
+              const uint32_t a2 = nib2(cd, 8 * h), a3 = nib2(cd, 8 * h + 4);
+              mma16816_full(o[mt], a0, a1, a2, a3, pb0, pb1);
+              mma16816_full(o[mt], a0, a1, a2, a3, pl0, pl1);
+            }
+          }
+        }
+      } else {
+        const uint4 *va = vr[kg][0], *vb = vr[kg][1], *vc = vr[kg][2], *vd = vr[kg][3];
+        const uint32_t wa[8] = {va[0].x, va[0].y, va[0].z, va[0].w, va[1].x, va[1].y, va[1].z, va[1].w};
+        const uint32_t wb[8] = {vb[0].x, vb[0].y, vb[0].z, vb[0].w, vb[1].x, vb[1].y, vb[1].z, vb[1].w};
+        const uint32_t wc[8] = {vc[0].x, vc[0].y, vc[0].z, vc[0].w, vc[1].x, vc[1].y, vc[1].z, vc[1].w};
+        const uint32_t wd[8] = {vd[0].x, vd[0].y, vd[0].z, vd[0].w, vd[1].x, vd[1].y, vd[1].z, vd[1].w};
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)  // word mt holds channels 16g + 2mt, +1
+          mma16816_full(o[mt], __byte_perm(wa[mt], wb[mt], 0x5410u), __byte_perm(wa[mt], wb[mt], 0x7632u),
+                        __byte_perm(wc[mt], wd[mt], 0x5410u), __byte_perm(wc[mt], wd[mt], 0x7632u), pb0,
+                        pb1);
+      }
     }
   }
+  };
+  pass(Kb, Vb, k0, k1, skip);
+  if (owns_new) {
+    // the new token: buffers shifted so that row newk is the input row
+    const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB - newk * RB;
+    pass(reinterpret_cast<const uint8_t *>(P.knew) + off, reinterpret_cast<const uint8_t *>(P.vnew) + off,
+         newk, newk + 1, -1);
+  }
+
+  // the next kernel in the stream may start its set-up now
+  asm volatile("griddepcontrol.launch_dependents;");
 
   // ---- per-warp state -> shared memory (queries < G only)
   l += __shfl_xor_sync(0xffffffffu, l, 1);
@@ -357,6 +406,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   if (Q4) {
     z += __shfl_xor_sync(0xffffffffu, z, 1);
     z += __shfl_xor_sync(0xffffffffu, z, 2);
+    cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+    cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+    z -= 128.f * cs;  // the codes were multiplied as 128 + u
   }
   float *red_m = reinterpret_cast<float *>(smem);
   float *red_l = red_m + NWARPS * G;
@@ -402,15 +454,28 @@ cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
     if (e != cudaSuccess) return e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    cfg->tile_rows = STEP;
+    cfg->tile_rows = Keys<Q4>::STEP;
     cfg->ctas_per_sm = occ;
     cfg->num_sms = sms;
     return cudaSuccess;
   }
   const int grid = d.B * d.n_ret * d.nsplit + d.B * d.n_str;
   if (grid == 0) return cudaSuccess;
-  kern<<<grid, NWARPS * 32, smem, s>>>(d);
-  return cudaGetLastError();
+  if (!d.pdl) {
+    kern<<<grid, NWARPS * 32, smem, s>>>(d);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(NWARPS * 32);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kern, d);
 }
 
 template <bool Q4>
@@ -429,6 +494,10 @@ cudaError_t dispatch(const DecodeParams &d, int G, cudaStream_t s, DecodeConfig 
 // head_dim 128, bf16 or 4-bit cache: the tensor-core decode.
 bool decode_mma_supported(int kv_type, int D, int G) {
   return D == 128 && (kv_type == kBF16 || kv_type == kINT4) && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
+bool decode_can_fuse_append(int kv_type, int D, int G) {
+  return kv_type == kBF16 && decode_mma_supported(kv_type, D, G);
 }
 
 cudaError_t decode_mma_config(int kv_type, int G, DecodeConfig *cfg) {

@@ -271,81 +271,126 @@ duo_status duo_append_kv(duo_cache *c, int32_t layer, const void *k, const void 
   return st;
 }
 
-duo_status duo_decode_attn(duo_cache *c, int32_t layer, const void *q, void *out, float scale,
-                           void *ws, size_t ws_bytes, duo_stream stream) {
-  if (!c || !q || !out) return DUO_ERR_ARG;
-  if (layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
-  if (!c->base) return DUO_ERR_STATE;
-  if (!std::isfinite(scale)) return DUO_ERR_ARG;
-  const int64_t n = c->seq_len[layer];
-  if (n <= 0) return DUO_ERR_STATE;
-  const auto &L = c->layers[layer];
-  const duo_cache_desc &d = c->desc;
-  const int G = d.n_q_heads / d.n_kv_heads;
-  duo::DecodeConfig cfg{};
-  cudaError_t e = cached_decode_config(c, &cfg);
-  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
-  if (e != cudaSuccess) return DUO_ERR_CUDA;
-  const int nsplit = choose_splits(c, layer, n, cfg);
-  const bool need_ws = L.n_ret > 0 && nsplit > 1;
-  const WsLayout w = ws_layout(d, c->n_ret_max);
-  if (need_ws) {
-    if (!ws) return DUO_ERR_WORKSPACE;
-    if (ws_bytes < (size_t)w.total) return DUO_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return DUO_ERR_ARG;
-  }
-  int64_t split_len = (n + nsplit - 1) / nsplit;
-  split_len = round_up(split_len, cfg.tile_rows);
-  duo::DecodeParams p{};
-  p.q = q;
-  p.out = out;
-  p.p = layer_ptrs(c, layer);
-  p.h = L.h;
-  p.B = d.batch;
-  p.Hq = d.n_q_heads;
-  p.Hkv = d.n_kv_heads;
-  p.G = G;
-  p.D = d.head_dim;
-  p.n_ret = L.n_ret;
-  p.n_str = L.n_str;
-  p.S = c->S;
-  p.R = c->R;
-  p.W = c->W;
-  p.Ws = c->Ws;
-  p.cap = d.capacity;
-  p.n = n;
-  p.nsplit = (int)((n + split_len - 1) / split_len);
-  p.split_len = split_len;
-  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d.head_dim);
-  p.scale_log2 = sc * 1.4426950408889634f;
-  uint8_t *wsb = static_cast<uint8_t *>(ws);
-  p.ws_cnt = need_ws ? reinterpret_cast<unsigned *>(wsb + w.cnt) : nullptr;
-  p.ws_lse = need_ws ? reinterpret_cast<float *>(wsb + w.lse) : nullptr;
-  p.ws_o = need_ws ? reinterpret_cast<float *>(wsb + w.o) : nullptr;
-  p.err = duo::device_error_word();
-  e = duo::launch_decode(p, d.kv_dtype, (cudaStream_t)stream);
-  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
-  return cuda_status(e);
-}
+namespace {
 
-duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, void *out,
-                                  float scale, duo_stream stream) {
-  if (!c || !q || !out) return DUO_ERR_ARG;
-  if (layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
-  if (!c->base) return DUO_ERR_STATE;
-  if (!std::isfinite(scale)) return DUO_ERR_ARG;
-  const int64_t n = c->seq_len[layer];
-  if (n <= 0) return DUO_ERR_STATE;
+// Everything a decode launch needs except the scratch pointers, for a layer
+// holding n tokens (the query at position n-1).
+duo_status plan_decode(duo_cache *c, int32_t layer, int64_t n, const void *q, void *out, float scale,
+                       duo::DecodeParams *p) {
   const auto &L = c->layers[layer];
   const duo_cache_desc &d = c->desc;
-  const int G = d.n_q_heads / d.n_kv_heads;
   duo::DecodeConfig cfg{};
   cudaError_t e = cached_decode_config(c, &cfg);
   if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return DUO_ERR_CUDA;
   const int want = choose_splits(c, layer, n, cfg);
   const int64_t split_len = round_up((n + want - 1) / want, cfg.tile_rows);
-  const int nsplit = (int)((n + split_len - 1) / split_len);
+  *p = duo::DecodeParams{};
+  p->q = q;
+  p->out = out;
+  p->p = layer_ptrs(c, layer);
+  p->h = L.h;
+  p->B = d.batch;
+  p->Hq = d.n_q_heads;
+  p->Hkv = d.n_kv_heads;
+  p->G = d.n_q_heads / d.n_kv_heads;
+  p->D = d.head_dim;
+  p->n_ret = L.n_ret;
+  p->n_str = L.n_str;
+  p->S = c->S;
+  p->R = c->R;
+  p->W = c->W;
+  p->Ws = c->Ws;
+  p->cap = d.capacity;
+  p->n = n;
+  p->nsplit = (int)((n + split_len - 1) / split_len);
+  p->split_len = split_len;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d.head_dim);
+  p->scale_log2 = sc * 1.4426950408889634f;
+  p->err = duo::device_error_word();
+  return DUO_OK;
+}
+
+// Point the decode at the caller's workspace (layout of ws_layout).
+duo_status use_workspace(const duo_cache *c, const duo::DecodeParams &p, void *ws, size_t ws_bytes,
+                         duo::DecodeParams *out) {
+  *out = p;
+  if (p.n_ret == 0 || p.nsplit == 1) return DUO_OK;
+  const WsLayout w = ws_layout(c->desc, c->n_ret_max);
+  if (!ws || ws_bytes < (size_t)w.total) return DUO_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return DUO_ERR_ARG;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  out->ws_cnt = reinterpret_cast<unsigned *>(wsb + w.cnt);
+  out->ws_lse = reinterpret_cast<float *>(wsb + w.lse);
+  out->ws_o = reinterpret_cast<float *>(wsb + w.o);
+  return DUO_OK;
+}
+
+duo_status launch_status(cudaError_t e) {
+  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+duo_status check_decode_args(const duo_cache *c, int32_t layer, const void *q, void *out, float scale) {
+  if (!c || !q || !out) return DUO_ERR_ARG;
+  if (layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
+  if (!c->base) return DUO_ERR_STATE;
+  if (!std::isfinite(scale)) return DUO_ERR_ARG;
+  return DUO_OK;
+}
+
+}  // namespace
+
+duo_status duo_decode_attn(duo_cache *c, int32_t layer, const void *q, void *out, float scale,
+                           void *ws, size_t ws_bytes, duo_stream stream) {
+  duo_status st = check_decode_args(c, layer, q, out, scale);
+  if (st != DUO_OK) return st;
+  const int64_t n = c->seq_len[layer];
+  if (n <= 0) return DUO_ERR_STATE;
+  duo::DecodeParams plan, p;
+  if ((st = plan_decode(c, layer, n, q, out, scale, &plan)) != DUO_OK) return st;
+  if ((st = use_workspace(c, plan, ws, ws_bytes, &p)) != DUO_OK) return st;
+  return launch_status(duo::launch_decode(p, c->desc.kv_dtype, (cudaStream_t)stream));
+}
+
+duo_status duo_decode_step(duo_cache *c, int32_t layer, const void *q, const void *k_new,
+                           const void *v_new, void *out, float scale, void *ws, size_t ws_bytes,
+                           duo_stream stream) {
+  duo_status st = check_decode_args(c, layer, q, out, scale);
+  if (st != DUO_OK) return st;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return DUO_ERR_ARG;
+  const duo_cache_desc &d = c->desc;
+  const int64_t n_cur = c->seq_len[layer];
+  if (c->layers[layer].n_ret > 0 && n_cur + 1 > d.capacity) return DUO_ERR_CAPACITY;
+  if (!duo::decode_can_fuse_append(d.kv_dtype, d.head_dim, d.n_q_heads / d.n_kv_heads)) {
+    // no fused kernel for this configuration: append, then attend
+    if ((st = duo_append_kv(c, layer, k_new, v_new, 1, stream)) != DUO_OK) return st;
+    return duo_decode_attn(c, layer, q, out, scale, ws, ws_bytes, stream);
+  }
+  const int64_t n = n_cur + 1;
+  duo::DecodeParams plan, p;
+  if ((st = plan_decode(c, layer, n, q, out, scale, &plan)) != DUO_OK) return st;
+  if ((st = use_workspace(c, plan, ws, ws_bytes, &p)) != DUO_OK) return st;
+  p.knew = k_new;
+  p.vnew = v_new;
+  p.new_slot = n_cur < c->S ? n_cur : c->S + (n_cur - c->S) % c->R;
+  p.pdl = 1;
+  st = launch_status(duo::launch_decode(p, d.kv_dtype, (cudaStream_t)stream));
+  if (st == DUO_OK) c->seq_len[layer] = n;
+  return st;
+}
+
+duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, void *out,
+                                  float scale, duo_stream stream) {
+  duo_status st = check_decode_args(c, layer, q, out, scale);
+  if (st != DUO_OK) return st;
+  const int64_t n = c->seq_len[layer];
+  if (n <= 0) return DUO_ERR_STATE;
+  const auto &L = c->layers[layer];
+  const duo_cache_desc &d = c->desc;
+  duo::DecodeParams p;
+  if ((st = plan_decode(c, layer, n, q, out, scale, &p)) != DUO_OK) return st;
+  const int G = p.G, nsplit = p.nsplit;
   // Compact scratch layout for exactly this launch: tickets, lse, partial O.
   const int64_t units = (int64_t)d.batch * L.n_ret;
   const int64_t off_lse = round_up(units * 4, kAlign);
@@ -353,44 +398,18 @@ duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, vo
   const int64_t need = off_o + units * nsplit * G * (int64_t)d.head_dim * 4;
   const bool need_ws = L.n_ret > 0 && nsplit > 1;
   if (need_ws && need > (int64_t)duo::decode_static_scratch_bytes()) return DUO_ERR_WORKSPACE;
-  uint8_t *scratch = nullptr;
   if (need_ws) {
-    void *p = nullptr;
-    if (duo::decode_static_scratch(&p) != cudaSuccess) return DUO_ERR_CUDA;
-    scratch = static_cast<uint8_t *>(p);
+    void *ptr = nullptr;
+    if (duo::decode_static_scratch(&ptr) != cudaSuccess) return DUO_ERR_CUDA;
+    uint8_t *scratch = static_cast<uint8_t *>(ptr);
     // tickets start at zero for this launch (the array keeps earlier calls' bytes)
     if (cudaMemsetAsync(scratch, 0, (size_t)(units * 4), (cudaStream_t)stream) != cudaSuccess)
       return DUO_ERR_CUDA;
+    p.ws_cnt = reinterpret_cast<unsigned *>(scratch);
+    p.ws_lse = reinterpret_cast<float *>(scratch + off_lse);
+    p.ws_o = reinterpret_cast<float *>(scratch + off_o);
   }
-  duo::DecodeParams p{};
-  p.q = q;
-  p.out = out;
-  p.p = layer_ptrs(c, layer);
-  p.h = L.h;
-  p.B = d.batch;
-  p.Hq = d.n_q_heads;
-  p.Hkv = d.n_kv_heads;
-  p.G = G;
-  p.D = d.head_dim;
-  p.n_ret = L.n_ret;
-  p.n_str = L.n_str;
-  p.S = c->S;
-  p.R = c->R;
-  p.W = c->W;
-  p.Ws = c->Ws;
-  p.cap = d.capacity;
-  p.n = n;
-  p.nsplit = nsplit;
-  p.split_len = split_len;
-  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d.head_dim);
-  p.scale_log2 = sc * 1.4426950408889634f;
-  p.ws_cnt = need_ws ? reinterpret_cast<unsigned *>(scratch) : nullptr;
-  p.ws_lse = need_ws ? reinterpret_cast<float *>(scratch + off_lse) : nullptr;
-  p.ws_o = need_ws ? reinterpret_cast<float *>(scratch + off_o) : nullptr;
-  p.err = duo::device_error_word();
-  e = duo::launch_decode(p, d.kv_dtype, (cudaStream_t)stream);
-  if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) return DUO_ERR_UNSUPPORTED;
-  return cuda_status(e);
+  return launch_status(duo::launch_decode(p, d.kv_dtype, (cudaStream_t)stream));
 }
 
 duo_status duo_prefill_attn(duo_cache *c, int32_t layer, const void *q, const void *k,

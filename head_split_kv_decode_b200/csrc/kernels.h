@@ -60,6 +60,12 @@ struct DecodeParams {
   float *ws_lse;       // [B][n_ret][nsplit][G]
   unsigned *ws_cnt;    // [B][n_ret]
   int *err;            // device error word
+  // Fused append (duo_decode_step): the K/V of the token at position n-1,
+  // [B][Hkv][D]; null when it is already in the cache.  The CTA that owns the
+  // token's row reads it from here and writes it to the cache.
+  const void *knew, *vnew;
+  int64_t new_slot;    // streaming slot of position n-1
+  int pdl;             // launched with programmatic dependent launch
 };
 
 struct PrefillParams {
@@ -83,6 +89,8 @@ struct DecodeConfig {
 cudaError_t decode_config(int kv_type, int D, int G, DecodeConfig *cfg);
 cudaError_t launch_append(const AppendParams &a, int kv_type, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &d, int kv_type, cudaStream_t s);
+// True when launch_decode can take the new token's K/V itself (fused append).
+bool decode_can_fuse_append(int kv_type, int D, int G);
 cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s);
 int *device_error_word();  // device address of the error word
 

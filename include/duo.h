@@ -153,6 +153,20 @@ duo_status duo_decode_attn(duo_cache *cache, int32_t layer, const void *q,
                            void *out, float softmax_scale, void *workspace,
                            size_t workspace_bytes, duo_stream stream);
 
+/* One decode step for one layer in a single launch where the kernels allow
+ * it: append the new token (k_new, v_new: [batch, n_kv_heads, head_dim]) at
+ * position seq_len and attend with q at that position, exactly as
+ * duo_append_kv(.., 1, ..) followed by duo_decode_attn.  The CTA that owns the
+ * new token's row takes its K/V from the inputs and writes them to the cache.
+ * Configurations without a fused kernel (fp32 caches, head_dim 64, 4-bit
+ * caches) run the two calls.  Advances the layer length by one.  The launch
+ * uses programmatic dependent launch, so its set-up overlaps the previous
+ * kernel in the stream.  Errors as for the two calls. */
+duo_status duo_decode_step(duo_cache *cache, int32_t layer, const void *q,
+                           const void *k_new, const void *v_new, void *out,
+                           float softmax_scale, void *workspace,
+                           size_t workspace_bytes, duo_stream stream);
+
 /* Decode attention like duo_decode_attn, but with no workspace argument and
  * no allocation of any kind: the split-K scratch (partial outputs, log-sum-exp
  * values, merge tickets) lives in a fixed array inside the library,

@@ -170,3 +170,28 @@ def test_workspace_too_small_is_rejected():
         B.duo_decode_attn(cache.handle, 0, q.data_ptr(), out.data_ptr(), 0.0, cache.ws_ptr, 16)
     assert e.value.name == "DUO_ERR_WORKSPACE"
     assert B.duo_poll_device_error() == 0
+
+
+@pytest.mark.parametrize("kind,D,Hq,Hkv", [("bf16", 128, 8, 2), ("bf16", 128, 4, 4), ("f32", 64, 4, 2)])
+def test_decode_step_fused_append(kind, D, Hq, Hkv):
+    """duo_decode_step = append one token + attend, in one launch where a fused
+    kernel exists; many steps so the ring wraps and the new token lands both in
+    the middle of a split and at a split boundary."""
+    B, S, R = 2, 3, 40
+    n0, steps = 700, 90
+    total = n0 + steps
+    mask = torch.tensor([1] + [0] * (Hkv - 1), dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, D, kind, total, mask[None], S, R)
+    K = synth.kv_field(81, range(B), range(total), Hkv, D, device="cuda").to(DT[kind])
+    V = synth.kv_field(82, range(B), range(total), Hkv, D, device="cuda").to(DT[kind])
+    Q = synth.kv_field(83, range(B), range(total), Hq, D, device="cuda").to(DT[kind])
+    cache.append(0, K[:, :n0].contiguous(), V[:, :n0].contiguous())
+    for t in range(n0, total):
+        if t == n0 + 40:
+            cache.set_decode_splits(3)
+        out = cache.step(0, Q[:, t].contiguous(), K[:, t].contiguous(), V[:, t].contiguous())
+        assert cache.seq_len(0) == t + 1
+        if t % 7 == 0 or t == total - 1:
+            ref = _oracle(K[:, :t + 1], V[:, :t + 1], Q[:, t], mask, S, R)
+            assert_parity(out, ref, kind, "step t=%d" % t)
+    _check_cache_bytes(cache, K, V, mask, S, R)
