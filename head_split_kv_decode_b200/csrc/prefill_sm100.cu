@@ -34,7 +34,12 @@ constexpr int BN = 128;           // keys per tile
 constexpr int HD = 128;           // head dim
 constexpr int BOX = 16384;        // one 64-column x 128-row swizzled box (bytes)
 constexpr int TILE = 2 * BOX;     // a 128 x 128 bf16 tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;       // 3 warpgroups: softmax A, softmax B, TMA + MMA (+2 idle)
+// Register split (setmaxnreg): the TMA/MMA warpgroup drops to kRegsLow and the
+// softmax warpgroups rise to kRegsHigh.  The sum must fit what the CTA was
+// launched with (kThreads x launch registers); the host checks it.
+constexpr int kRegsHigh = 200;
+constexpr int kRegsLow = 96;
 constexpr float kRescaleLog2 = 8.0f;
 
 // shared memory map (offsets from a 1024-aligned base)
@@ -333,6 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + kTmemSlot);
 
+  if (warp >= 8) {
+    // third warpgroup: one TMA warp, one MMA warp, two spare warps
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 8) {
     // =============================================================== TMA producer
     if (lane == 0) {
@@ -391,20 +399,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
       const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
-      const uint32_t qb[2] = {base + kQA, base + kQB};
+      // Descriptors are built once; the start-address field (address >> 4,
+      // 14 bits) is advanced by adding offsets (shared memory < 256 KB, so the
+      // field never carries out).
+      const uint64_t dq[2] = {sdesc(base + kQA, 16, 1024), sdesc(base + kQB, 16, 1024)};
+      const uint64_t dk[2] = {sdesc(base + kK0, 16, 1024), sdesc(base + kK1, 16, 1024)};
+      const uint64_t dv[2] = {sdesc(base + kV0, BOX, 1024), sdesc(base + kV1, BOX, 1024)};
       auto issue_s = [&](int x, int st) {
-        const uint32_t kb = base + (st ? kK1 : kK0);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
-          const uint32_t off = (uint32_t)((k >> 2) * BOX + (k & 3) * 32);
-          mma_ss(tS[x], sdesc(qb[x] + off, 16, 1024), sdesc(kb + off, 16, 1024), kIdescS, k > 0);
+          const uint64_t off = (uint64_t)(((k >> 2) * BOX + (k & 3) * 32) >> 4);
+          mma_ss(tS[x], dq[x] + off, dk[st] + off, kIdescS, k > 0);
         }
       };
       auto issue_pv = [&](int x, int st, int j) {
-        const uint32_t vb = base + (st ? kV1 : kV0);
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_ts(tO[x], tS[x] + 8u * k, sdesc(vb + k * 2048u, BOX, 1024), kIdescPV, (j > 0 || k > 0));
+          mma_ts(tO[x], tS[x] + 8u * k, dv[st] + (uint64_t)((k * 2048) >> 4), kIdescPV, (j > 0 || k > 0));
       };
       bool ok = mbar_wait(bar(Q_FULL), 0, P.err, kErrWaitMma) &&
                 mbar_wait(bar(K_FULL0), 0, P.err, kErrWaitMma);
@@ -451,7 +462,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(DRAIN));
       mbar_wait(bar(DRAIN), 0, P.err, kErrWaitMma);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     // =============================================================== softmax (A: warps 0-3, B: 4-7)
     const int x = warp >> 2;
     const int wq = warp & 3;
@@ -466,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int o_bar = x ? O_FULL_B : O_FULL_A;
     const float sl2 = P.scale_log2;
     float m = -INFINITY;
-    float2 l2 = make_float2(0.f, 0.f);
+    float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = mbar_wait(bar(s_bar), (uint32_t)(j & 1), P.err, kErrWaitMma);
@@ -521,37 +534,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                      range_bits(r1lo, min(r1hi, filled), first, ch) |
                      range_bits(r2lo, min(r2hi, filled), first, ch));
       }
-      // Two passes over S in 64-column halves (register budget: ten warps on
-      // four schedulers leave 168 registers per thread): the row max, then the
-      // probabilities.  Masked logits become -inf.
-      constexpr int HALF = 64;
-      auto load_half = [&](int h, float (&v)[HALF]) {
-        tmem_ld32_async(tS + (uint32_t)(HALF * h), v);
-        tmem_ld32_async(tS + (uint32_t)(HALF * h + 32), v + 32);
-        tmem_wait_ld();
+      // The whole S row in registers: four loads in flight, one wait.
+      float v[BN];
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const uint32_t bits = vis[2 * h + k];
-          if (bits != 0xffffffffu) {
+      for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32_async(tS + 32u * cc, v + 32 * cc);
+      tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (!((bits >> i) & 1u)) v[32 * k + i] = -INFINITY;
-          }
+      for (int k = 0; k < BN / 32; ++k) {
+        const uint32_t bits = vis[k];
+        if (bits != 0xffffffffu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (!((bits >> i) & 1u)) v[32 * k + i] = -INFINITY;
         }
-      };
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int h = 0; h < BN / HALF; ++h) {
-        float v[HALF];
-        load_half(h, v);
-        float t[8];
+      }
+      float mx;
+      {
+        float t[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 16; ++i)
           t[i] = max3f(max3f(v[8 * i], v[8 * i + 1], v[8 * i + 2]),
                        max3f(v[8 * i + 3], v[8 * i + 4], v[8 * i + 5]), fmaxf(v[8 * i + 6], v[8 * i + 7]));
-        mx = max3f(mx, max3f(t[0], t[1], t[2]), max3f(max3f(t[3], t[4], t[5]), t[6], t[7]));
+        const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
+        const float u2 = max3f(t[6], t[7], t[8]), u3 = max3f(t[9], t[10], t[11]);
+        const float u4 = max3f(t[12], t[13], t[14]);
+        mx = max3f(max3f(u0, u1, u2), max3f(u3, u4, t[15]), -INFINITY) * sl2;
       }
-      mx *= sl2;
       const float m_new = fmaxf(m, mx);
       const bool grow = m_new > m + kRescaleLog2 || (m == -INFINITY && m_new > -INFINITY);
       if (__any_sync(0xffffffffu, grow)) {
@@ -568,8 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_st();
         }
         if (grow) {
-          l2.x *= alpha;
-          l2.y *= alpha;
+          l2[0].x *= alpha;
+          l2[0].y *= alpha;
+          l2[1].x *= alpha;
+          l2[1].y *= alpha;
           m = m_new;
         }
       }
@@ -577,31 +587,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // as packed bf16 (column c/2 holds keys c, c+1)
       const float mu = (m == -INFINITY) ? 0.f : m;
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-mu, -mu);
-#pragma unroll 1
-      for (int h = 0; h < BN / HALF; ++h) {
-        float v[HALF];
-        load_half(h, v);
 #pragma unroll
-        for (int cc = 0; cc < HALF / 32; ++cc) {
-          uint32_t pk[16];
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float2 t = ffma2(make_float2(v[32 * cc + 2 * i], v[32 * cc + 2 * i + 1]), sc2, nm2);
-            t.x = fast_exp2(t.x);
-            t.y = fast_exp2(t.y);
-            l2 = __fadd2_rn(l2, t);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(t.x, t.y);
-            pk[i] = *reinterpret_cast<uint32_t *>(&h2);
-          }
-          tmem_st16(tS + (uint32_t)(HALF / 2 * h + 16 * cc), pk);
+        for (int i = 0; i < 16; ++i) {
+          float2 t = ffma2(make_float2(v[32 * cc + 2 * i], v[32 * cc + 2 * i + 1]), sc2, nm2);
+          t.x = fast_exp2(t.x);
+          t.y = fast_exp2(t.y);
+          l2[i & 1] = __fadd2_rn(l2[i & 1], t);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(t.x, t.y);
+          pk[i] = *reinterpret_cast<uint32_t *>(&h2);
         }
+        tmem_st16(tS + 16u * cc, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(p_bar));
     }
-    const float l = l2.x + l2.y;
+    const float l = (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
     if (ok) ok = mbar_wait(bar(o_bar), 0, P.err, kErrWaitMma);
     if (__all_sync(0xffffffffu, ok) && !abort_set(abort_flag)) {
       tc_fence_after();
@@ -699,6 +704,11 @@ cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
+    // The register split must fit the registers the CTA is launched with, or
+    // setmaxnreg.inc would wait for registers that never come.
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, prefill_kernel)) != cudaSuccess) return e;
+    if (128 * (2 * kRegsHigh + kRegsLow) > kThreads * fa.numRegs) return cudaErrorInvalidConfiguration;
     attr = true;
   }
   const int n_pairs = (p.C + 2 * BM - 1) / (2 * BM);
