@@ -195,8 +195,13 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   }
   const float sl2 = P.scale_log2;
 
-  // O^T accumulators: tile mt holds channels 16g + 2mt (rows g) and
-  // 16g + 2mt + 1 (rows g+8) for queries 2t and 2t+1.
+  // O^T accumulators: tile mt holds channels vchan(mt) (rows g) and
+  // vchan(mt) + 1 (rows g+8) for queries 2t and 2t+1.  bf16: the thread's V
+  // channels are the 16-byte chunks g and 8+g of a row (so the eight lanes of
+  // a key read 128 contiguous bytes); 4-bit: code bytes 8g..8g+7.
+  auto vchan = [&](int mt) {
+    return Q4 ? 16 * g + 2 * mt : 64 * (mt >> 2) + 8 * g + 2 * (mt & 3);
+  };
   float o[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
@@ -211,7 +216,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
     // ------------------------------------------------------------ loads (all up front)
     // group kg covers keys kb = kb0 + 16*kg ..: K of key kb + 8*nt + g (this
     // thread's column of S); V of keys kb + {2t, 2t+1, 8+2t, 9+2t} (the k-slots
-    // of the P^T fragment), channels [16g, 16g+16).
+    // of the P^T fragment) at this thread's channels (see vchan below).
     uint4 kr[KG][2][Q4 ? 1 : 4];
     uint2 ksz[KG][2], vsz[KG][2];
     uint4 vr[KG][4][Q4 ? 1 : 2];
@@ -243,7 +248,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
         } else {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            vr[kg][i][h] = ok ? ldg128(Vx + key * RB + 32 * g + 16 * h) : make_uint4(0, 0, 0, 0);
+            vr[kg][i][h] = ok ? ldg128(Vx + key * RB + 16 * (8 * h + g)) : make_uint4(0, 0, 0, 0);
         }
       }
     }
@@ -381,7 +386,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
         const uint32_t wc[8] = {vc[0].x, vc[0].y, vc[0].z, vc[0].w, vc[1].x, vc[1].y, vc[1].z, vc[1].w};
         const uint32_t wd[8] = {vd[0].x, vd[0].y, vd[0].z, vd[0].w, vd[1].x, vd[1].y, vd[1].z, vd[1].w};
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)  // word mt holds channels 16g + 2mt, +1
+        for (int mt = 0; mt < 8; ++mt)  // word mt holds channels vchan(mt), +1
           mma16816_full(o[mt], __byte_perm(wa[mt], wb[mt], 0x5410u), __byte_perm(wa[mt], wb[mt], 0x7632u),
                         __byte_perm(wc[mt], wd[mt], 0x5410u), __byte_perm(wc[mt], wd[mt], 0x7632u), pb0,
                         pb1);
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   const int q0 = 2 * t, q1 = 2 * t + 1;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
-    const int ch = 16 * g + 2 * mt;
+    const int ch = vchan(mt);
     if (q0 < G) {
       red_o[(warp * G + q0) * D + ch] = o[mt][0] + z0;
       red_o[(warp * G + q0) * D + ch + 1] = o[mt][2] + z0;
