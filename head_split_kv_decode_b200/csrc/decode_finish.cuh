@@ -43,8 +43,10 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
     if (direct) {
       store_out(out + g * D + c, O / L);
     } else {
-      P.ws_o[(part * G + g) * D + c] = O / L;
-      if (c == 0) P.ws_lse[part * G + g] = M + fast_log2(L);
+      // a split whose CTA claimed no keys leaves weight zero (lse -inf)
+      const bool empty = L == 0.f;
+      P.ws_o[(part * G + g) * D + c] = empty ? 0.f : O / L;
+      if (c == 0) P.ws_lse[part * G + g] = empty ? -INFINITY : M + fast_log2(L);
     }
   }
   if (direct) return;
@@ -58,64 +60,82 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   if (!s_last) return;
   __threadfence();
   const int64_t part0 = ((int64_t)b * P.n_ret + pidx) * P.nsplit;
-  // weights w_s = 2^(lse_s - max) per (split, query head)
-  float *s_w = reinterpret_cast<float *>(smem);     // [nsplit][G]
-  float *s_den = s_w + P.nsplit * G;                // [G]
+  // weights w_s = 2^(lse_s - max) per (split, query head), then the weighted
+  // sum of the partials.  Warp w sums splits w, w+NWARPS, ... (U at a time,
+  // their loads in flight together); lane l owns channels [4l, 4l+4) of every
+  // query head (D/4 float4 per head row; for D = 64 the upper lanes idle).
+  // The first batch of partials is loaded before the weights are reduced, so
+  // that its latency overlaps that reduction.
+  float *s_w = reinterpret_cast<float *>(smem);        // [nsplit][G]
+  float *s_den = s_w + P.nsplit * G;                   // [G]
   float *s_acc = s_w + ((P.nsplit * G + G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
-  for (int i = tid; i < P.nsplit * G; i += NT) s_w[i] = __ldcg(P.ws_lse + part0 * G + i);
-  __syncthreads();
-  if (tid < G) {
+  constexpr int L4 = D / 4;
+  constexpr int U = G >= 8 ? 2 : 4;
+  const bool owns = lane < L4;
+  const float4 *src = reinterpret_cast<const float4 *>(P.ws_o + part0 * G * D) + (owns ? lane : 0);
+  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 v[U][G];
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int sp = warp + u * NWARPS;
+      v[u][g] = (owns && sp < P.nsplit) ? __ldcg(src + (sp * G + g) * L4) : zero4;
+    }
+  // warp g (and g + NWARPS, ...) reduces query head g over the splits, one
+  // split per lane at a time
+  for (int g = warp; g < G; g += NWARPS) {
     float M = -INFINITY;
-    for (int sp = 0; sp < P.nsplit; ++sp) M = fmaxf(M, s_w[sp * G + tid]);
+    for (int sp = lane; sp < P.nsplit; sp += 32) {
+      const float x = __ldcg(P.ws_lse + (part0 + sp) * G + g);
+      s_w[sp * G + g] = x;
+      M = fmaxf(M, x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float den = 0.f;
-    for (int sp = 0; sp < P.nsplit; ++sp) {
-      const float w = fast_exp2(s_w[sp * G + tid] - M);
-      s_w[sp * G + tid] = w;
+    for (int sp = lane; sp < P.nsplit; sp += 32) {
+      const float x = s_w[sp * G + g];
+      const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);  // a split that claimed no keys
+      s_w[sp * G + g] = w;
       den += w;
     }
-    s_den[tid] = den;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (lane == 0) s_den[g] = den;
   }
   __syncthreads();
-  // warp w sums splits w, w+NWARPS, ...; lane l owns channels [4l, 4l+4) of
-  // every query head (D/4 float4 per head row, so lanes cover D = 128; for
-  // D = 64 the upper lanes idle).  Four splits' loads are kept in flight.
-  constexpr int L4 = D / 4;
   float4 acc[G];
 #pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (lane < L4) {
-    const float4 *src = reinterpret_cast<const float4 *>(P.ws_o + part0 * G * D) + lane;
-    int sp = warp;
-    for (; sp + 3 * NWARPS < P.nsplit; sp += 4 * NWARPS) {
-      float4 v[4][G];
+  for (int g = 0; g < G; ++g) acc[g] = zero4;
+  auto fma4 = [&](float4 &a, float w, const float4 &x) {
+    a.x += w * x.x;
+    a.y += w * x.y;
+    a.z += w * x.z;
+    a.w += w * x.w;
+  };
+  int sp = warp;
+  while (true) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int g = 0; g < G; ++g) v[u][g] = __ldcg(src + ((sp + u * NWARPS) * G + g) * L4);
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float w = s_w[(sp + u * NWARPS) * G + g];
-          acc[g].x += w * v[u][g].x;
-          acc[g].y += w * v[u][g].y;
-          acc[g].z += w * v[u][g].z;
-          acc[g].w += w * v[u][g].w;
-        }
-    }
-    for (; sp < P.nsplit; sp += NWARPS)
+    for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float4 v = __ldcg(src + (sp * G + g) * L4);
-        const float w = s_w[sp * G + g];
-        acc[g].x += w * v.x;
-        acc[g].y += w * v.y;
-        acc[g].z += w * v.z;
-        acc[g].w += w * v.w;
+        const int su = sp + u * NWARPS;
+        if (su < P.nsplit) fma4(acc[g], s_w[su * G + g], v[u][g]);
       }
+    sp += U * NWARPS;
+    if (sp >= P.nsplit) break;
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-      reinterpret_cast<float4 *>(s_acc + (warp * G + g) * D)[lane] = acc[g];
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int su = sp + u * NWARPS;
+        v[u][g] = (owns && su < P.nsplit) ? __ldcg(src + (su * G + g) * L4) : zero4;
+      }
+  }
+  if (owns) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) reinterpret_cast<float4 *>(s_acc + (warp * G + g) * D)[lane] = acc[g];
   }
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += NT) {
@@ -125,7 +145,10 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
     for (int w = 0; w < NWARPS; ++w) num += s_acc[(w * G + g) * D + c];
     store_out(out + g * D + c, num / s_den[g]);
   }
-  if (tid == 0) *cnt = 0u;  // leave the ticket ready for the next call
+  if (tid == 0) {  // leave the ticket (and chunk counter) ready for the next call
+    *cnt = 0u;
+    if (P.ws_next) P.ws_next[((int64_t)b * P.n_ret + pidx) * kChunkCounterStride] = 0u;
+  }
 }
 
 // State layout expected: each 8-lane group of a warp holds m[g], l[g] and NP

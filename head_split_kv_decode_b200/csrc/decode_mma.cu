@@ -66,6 +66,11 @@ __device__ __forceinline__ uint2 ldg64(const void *p) {
   return v;
 }
 
+// Fetch [ptr, ptr + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -140,8 +145,41 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
     Ks += row0 * 4;
     Vs += row0 * 4;
   }
-  // Launched with programmatic dependent launch: everything above overlapped
-  // the previous kernel; nothing it may have written is read before this.
+  constexpr int KG = Keys<Q4>::KG;
+  constexpr int64_t T = 16 * KG;  // keys per warp tile
+  // A retrieval head with several splits balances its splits at run time: a
+  // CTA that gets less memory bandwidth takes fewer of the tiles handed out
+  // at the end (see below), so the splits finish together.  Each CTA still
+  // leaves one partial.  Streaming heads and single-split heads walk their
+  // range [k0, k1) statically.
+  const bool dynamic = retrieval && P.nsplit > 1;
+  const int64_t tiles = (P.n + T - 1) / T;
+  const int64_t ts = dynamic ? (tiles - tiles / 8) / P.nsplit : 0;  // static tiles per split
+  // this warp's first two tiles, [first, first + T) and the one NWARPS tiles on
+  const int64_t first = dynamic ? ((int64_t)split * ts + warp) * T : k0 + (int64_t)warp * T;
+  const int64_t last = dynamic ? (int64_t)(split + 1) * ts * T : k1;
+
+  // Launched with programmatic dependent launch, so this may run while the
+  // previous kernel in the stream finishes.  Bring this warp's first two
+  // tiles into L2 meanwhile: every global write lands in L2, so a line
+  // fetched now cannot be stale when the loads below (after the wait) use it.
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int64_t kb = first + (int64_t)i * NWARPS * T;
+      if (kb < last) {
+        const int64_t rows = min(T, last - kb);
+        prefetch_l2(Kb + kb * RB, (uint32_t)(rows * RB));
+        prefetch_l2(Vb + kb * RB, (uint32_t)(rows * RB));
+        if (Q4) {  // 4-byte (scale, zero) rows; buffers hold a multiple of 4 rows
+          const uint32_t sz = (uint32_t)(((rows + 3) & ~3LL) * 4);
+          prefetch_l2(Ks + kb * 4, sz);
+          prefetch_l2(Vs + kb * 4, sz);
+        }
+      }
+    }
+  }
+  // Nothing the previous kernel may have written is read before this.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Fused append (bf16 cache): the token at position n-1 is not in the cache
@@ -149,15 +187,15 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   // row in the main pass, and adds it in a one-key pass that reads the inputs.
   const bool fused = !Q4 && P.knew != nullptr;
   const int64_t newk = retrieval ? P.n - 1 : P.new_slot;  // its row in this head's buffer
-  const bool owns_new = fused && newk >= k0 && newk < k1;
-  if (owns_new && warp == 0) {
+  const bool owns_new = fused && !dynamic && newk >= k0 && newk < k1;
+  auto write_new = [&]() {  // one warp copies the new K and V rows into the cache
     const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB;
     const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
     const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + off;
     uint8_t *dst = const_cast<uint8_t *>(lane < 16 ? Kb : Vb) + newk * RB;
     reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
-  }
-  const int64_t skip = owns_new ? newk : -1;
+  };
+  if (owns_new && warp == 0) write_new();
 
   // ---- query fragments (rows g < G), k-step order matching the K loads
   uint32_t qa[8][2];
@@ -209,10 +247,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   // 4-bit cache z = sum p*zp and cs = sum p*sc (as multiplied, see below)
   float m = -INFINITY, l = 0.f, z = 0.f, cs = 0.f;
 
-  constexpr int KG = Keys<Q4>::KG;
-  // Keys [lo, hi) of the buffers Kx/Vx (row index = key), except `skip`.
-  auto pass = [&](const uint8_t *Kx, const uint8_t *Vx, int64_t lo, int64_t hi, int64_t skip_key) {
-  for (int64_t kb0 = lo + (int64_t)warp * 16 * KG; kb0 < hi; kb0 += Keys<Q4>::STEP) {
+  // One warp, keys [kb0, kb0 + 16*KG) below hi of the buffers Kx/Vx (row
+  // index = key), except `skip_key`.
+  auto tile = [&](const uint8_t *Kx, const uint8_t *Vx, int64_t kb0, int64_t hi, int64_t skip_key) {
     // ------------------------------------------------------------ loads (all up front)
     // group kg covers keys kb = kb0 + 16*kg ..: K of key kb + 8*nt + g (this
     // thread's column of S); V of keys kb + {2t, 2t+1, 8+2t, 9+2t} (the k-slots
@@ -392,13 +429,47 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
                         pb1);
       }
     }
-  }
   };
-  pass(Kb, Vb, k0, k1, skip);
-  if (owns_new) {
+  bool new_here = owns_new && warp == 0;  // this warp adds the new token at the end
+  if (dynamic) {
+    // Tiles of T keys: each split walks a static share of 7/8 of them (warps
+    // strided as in the static pass); the last eighth is a pool that warps
+    // claim one tile at a time from the head's counter once their share is
+    // done.  The first claim is issued during the warp's last static tile, so
+    // its latency overlaps that tile.
+    const int64_t t1 = (int64_t)(split + 1) * ts, pool0 = (int64_t)P.nsplit * ts;
+    unsigned *next = P.ws_next + ((int64_t)b * P.n_ret + pidx) * kChunkCounterStride;
+    auto visit = [&](int64_t tt) {
+      const int64_t kb0 = tt * T;
+      const bool has_new = fused && newk >= kb0 && newk < kb0 + T;
+      if (has_new) {
+        write_new();
+        new_here = true;
+      }
+      tile(Kb, Vb, kb0, P.n, has_new ? newk : -1);
+    };
+    unsigned c = 0;
+    int64_t tt = (int64_t)split * ts + warp;
+    if (tt >= t1 && lane == 0) c = atomicAdd(next, 1u);
+    for (; tt < t1; tt += NWARPS) {
+      if (tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
+      visit(tt);
+    }
+    c = __shfl_sync(0xffffffffu, c, 0);
+    while (pool0 + (int64_t)c < tiles) {
+      unsigned nx = 0;  // claim the following tile now; needed only after this one
+      if (lane == 0) nx = atomicAdd(next, 1u);
+      visit(pool0 + c);
+      c = __shfl_sync(0xffffffffu, nx, 0);
+    }
+  } else {
+    for (int64_t kb0 = k0 + (int64_t)warp * 16 * KG; kb0 < k1; kb0 += Keys<Q4>::STEP)
+      tile(Kb, Vb, kb0, k1, owns_new ? newk : -1);
+  }
+  if (new_here) {
     // the new token: buffers shifted so that row newk is the input row
     const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB - newk * RB;
-    pass(reinterpret_cast<const uint8_t *>(P.knew) + off, reinterpret_cast<const uint8_t *>(P.vnew) + off,
+    tile(reinterpret_cast<const uint8_t *>(P.knew) + off, reinterpret_cast<const uint8_t *>(P.vnew) + off,
          newk, newk + 1, -1);
   }
 

@@ -66,9 +66,10 @@ duo::LayerPtrs layer_ptrs(const duo_cache *c, int layer) {
                         at(L.off_str_k_sz), at(L.off_str_v_sz)};
 }
 
-// Workspace: [counters: B*n_ret_max u32][lse: B*n_ret_max*MAXS*G f32][o: ...*D f32]
+// Workspace: [merge tickets: B*n_ret_max u32][chunk counters: B*n_ret_max
+//            lines of kChunkCounterStride u32][lse: B*n_ret_max*MAXS*G f32][o: ...*D f32]
 struct WsLayout {
-  int64_t cnt, lse, o, total;
+  int64_t cnt, next, lse, o, total;
 };
 
 WsLayout ws_layout(const duo_cache_desc &d, int n_ret_max) {
@@ -76,7 +77,8 @@ WsLayout ws_layout(const duo_cache_desc &d, int n_ret_max) {
   const int64_t units = (int64_t)d.batch * (n_ret_max > 0 ? n_ret_max : 1);
   WsLayout w;
   w.cnt = 0;
-  w.lse = round_up(units * 4, kAlign);
+  w.next = round_up(units * 4, kAlign);
+  w.lse = w.next + round_up(units * duo::kChunkCounterStride * 4, kAlign);
   w.o = w.lse + round_up(units * duo::kMaxSplits * G * 4, kAlign);
   w.total = w.o + round_up(units * duo::kMaxSplits * G * (int64_t)d.head_dim * 4, kAlign);
   return w;
@@ -321,6 +323,7 @@ duo_status use_workspace(const duo_cache *c, const duo::DecodeParams &p, void *w
   if ((reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return DUO_ERR_ARG;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   out->ws_cnt = reinterpret_cast<unsigned *>(wsb + w.cnt);
+  out->ws_next = reinterpret_cast<unsigned *>(wsb + w.next);
   out->ws_lse = reinterpret_cast<float *>(wsb + w.lse);
   out->ws_o = reinterpret_cast<float *>(wsb + w.o);
   return DUO_OK;
@@ -391,9 +394,11 @@ duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, vo
   duo::DecodeParams p;
   if ((st = plan_decode(c, layer, n, q, out, scale, &p)) != DUO_OK) return st;
   const int G = p.G, nsplit = p.nsplit;
-  // Compact scratch layout for exactly this launch: tickets, lse, partial O.
+  // Compact scratch layout for exactly this launch: tickets, chunk counters,
+  // lse, partial O.
   const int64_t units = (int64_t)d.batch * L.n_ret;
-  const int64_t off_lse = round_up(units * 4, kAlign);
+  const int64_t off_next = round_up(units * 4, kAlign);
+  const int64_t off_lse = off_next + round_up(units * duo::kChunkCounterStride * 4, kAlign);
   const int64_t off_o = off_lse + round_up(units * nsplit * G * 4, kAlign);
   const int64_t need = off_o + units * nsplit * G * (int64_t)d.head_dim * 4;
   const bool need_ws = L.n_ret > 0 && nsplit > 1;
@@ -402,10 +407,12 @@ duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, vo
     void *ptr = nullptr;
     if (duo::decode_static_scratch(&ptr) != cudaSuccess) return DUO_ERR_CUDA;
     uint8_t *scratch = static_cast<uint8_t *>(ptr);
-    // tickets start at zero for this launch (the array keeps earlier calls' bytes)
-    if (cudaMemsetAsync(scratch, 0, (size_t)(units * 4), (cudaStream_t)stream) != cudaSuccess)
+    // tickets and counters start at zero for this launch (the array keeps
+    // earlier calls' bytes)
+    if (cudaMemsetAsync(scratch, 0, (size_t)off_lse, (cudaStream_t)stream) != cudaSuccess)
       return DUO_ERR_CUDA;
     p.ws_cnt = reinterpret_cast<unsigned *>(scratch);
+    p.ws_next = reinterpret_cast<unsigned *>(scratch + off_next);
     p.ws_lse = reinterpret_cast<float *>(scratch + off_lse);
     p.ws_o = reinterpret_cast<float *>(scratch + off_o);
   }

@@ -9,6 +9,10 @@ namespace duo {
 
 constexpr int kMaxKvHeads = 64;
 constexpr int kMaxSplits = 512;
+// u32 slots between the per-head chunk counters of the decode workspace (one
+// 256-byte line each, so that concurrent claims on different heads do not
+// queue on one line)
+constexpr int kChunkCounterStride = 64;
 constexpr int kMaxDevices = 64;
 
 enum KvType : int { kF32 = 0, kBF16 = 1, kINT4 = 2 };
@@ -58,7 +62,8 @@ struct DecodeParams {
   float scale_log2;    // softmax scale * log2(e)
   float *ws_o;         // [B][n_ret][nsplit][G][D]
   float *ws_lse;       // [B][n_ret][nsplit][G]
-  unsigned *ws_cnt;    // [B][n_ret]
+  unsigned *ws_cnt;    // [B][n_ret] merge tickets
+  unsigned *ws_next;   // [B][n_ret][kChunkCounterStride] pool counter of each retrieval head (tensor-core decode)
   int *err;            // device error word
   // Fused append (duo_decode_step): the K/V of the token at position n-1,
   // [B][Hkv][D]; null when it is already in the cache.  The CTA that owns the
