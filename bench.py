@@ -18,6 +18,7 @@ bounded sample of the same workload instead.
 """
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -143,6 +144,32 @@ class ClockSampler:
 # --------------------------------------------------------------------------- decode
 
 
+# DRAM traffic of one fused decode launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from an ncu capture of one layer of the 128K batch-1
+# GQA workload (4 retrieval + 4 streaming KV heads, context 131075), and that
+# launch's algorithmic bytes.  The ratio scales to the benchmark's launches; it
+# is reported only while the kernel's sources hash as they did when the
+# counters were taken (otherwise traffic is null).
+DECODE_TRAFFIC = {
+    "sources": ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h"),
+    "sha256": "249c97faa4c8fbeb90a80da2820e9932755cd0926ccfa1d8cfb9c0120d98a5a4",
+    "dram_bytes": 269760768 + 4478720,
+    "algorithmic_bytes": 269117440,
+}
+
+
+def decode_traffic(bytes_per_launch):
+    """ncu DRAM bytes per launch scaled to this launch size, or None if the
+    kernel changed since the capture."""
+    h = hashlib.sha256()
+    for name in DECODE_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, "head_split_kv_decode_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != DECODE_TRAFFIC["sha256"]:
+        return None
+    return DECODE_TRAFFIC["dram_bytes"] / DECODE_TRAFFIC["algorithmic_bytes"] * bytes_per_launch
+
+
 def decode_bytes_per_layer(w, batch, n, n_ret, n_str):
     """Algorithmic bytes of one decode-attention launch (visible KV + Q + O)."""
     per_tok = 4 * w.head_dim if w.kv_dtype != "int4" else 2 * (w.head_dim // 2 + 4)
@@ -213,6 +240,12 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
     # (duo_decode_step: append + attend); other caches append, then attend.
     fused = w.kv_dtype == "bf16" and w.head_dim == 128
 
+    # The fused path's timed region holds nothing but its decode launches, back
+    # to back (programmatic dependent launch overlaps each one's set-up with
+    # the previous one's tail), so its average launch duration is the region's
+    # time over the launch count; an event between two launches would break
+    # that overlap.  The unfused path brackets each attention launch with
+    # events to separate it from the append before it.
     def step(s, timed_idx=None):
         for layer in range(w.layers):
             kp, vp = ks[layer][s].data_ptr(), vs[layer][s].data_ptr()
@@ -220,7 +253,7 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
                 st = lib.duo_append_kv(h, layer, kp, vp, 1, sh)
                 if st:
                     raise B.DuoError(st, "duo_append_kv")
-            if timed_idx is not None:
+            if timed_idx is not None and not fused:
                 ev_s[timed_idx * w.layers + layer].record(stream)
             if fused:
                 st = lib.duo_decode_step(h, layer, qs[layer][s].data_ptr(), kp, vp,
@@ -230,7 +263,7 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
                                          0.0, ws, wsb, sh)
             if st:
                 raise B.DuoError(st, "duo_decode_step" if fused else "duo_decode_attn")
-            if timed_idx is not None:
+            if timed_idx is not None and not fused:
                 ev_e[timed_idx * w.layers + layer].record(stream)
 
     for s in range(W):
@@ -251,7 +284,10 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
     if world > 1:
         torch.distributed.barrier()
     ms = start.elapsed_time(end)
-    kern_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+    if fused:
+        kern_ms = [ms / (K * w.layers)] * (K * w.layers)
+    else:
+        kern_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
     if B.duo_poll_device_error() != 0:
         raise RuntimeError("a bounded device wait gave up during the benchmark")
 
@@ -266,34 +302,41 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
             step_bytes += lb + append_bytes(w, batch)
     step_bytes /= K
 
-    # ---- end to end through the public API: pinned host inputs in, outputs out
-    host_q = [q[W + K:W + 2 * K].cpu().pin_memory() for q in qs]
-    host_k = [k[W + K:W + 2 * K].cpu().pin_memory() for k in ks]
-    host_v = [v[W + K:W + 2 * K].cpu().pin_memory() for v in vs]
-    host_o = [torch.empty((K,) + tuple(o.shape), dtype=o.dtype).pin_memory() for o in outs]
-    dq = [torch.empty_like(q[0]) for q in qs]
-    dk = [torch.empty_like(k[0]) for k in ks]
-    dv = [torch.empty_like(v[0]) for v in vs]
-    h2d = sum(x[0].numel() * x[0].element_size() for x in host_q + host_k + host_v)
-    d2h = sum(o.numel() * o.element_size() for o in outs)
+    # ---- end to end through the public API: each step copies that token's
+    # q/k/v for every layer in from one pinned host buffer, runs the layers,
+    # and copies every layer's output back to pinned host memory.
+    nq, nk = qs[0][0].numel(), ks[0][0].numel()
+    per_layer = nq + 2 * nk
+    host_in = torch.empty((K, w.layers, per_layer), dtype=qs[0].dtype).pin_memory()
+    for layer in range(w.layers):
+        host_in[:, layer, :nq] = qs[layer][W + K:W + 2 * K].reshape(K, nq).cpu()
+        host_in[:, layer, nq:nq + nk] = ks[layer][W + K:W + 2 * K].reshape(K, nk).cpu()
+        host_in[:, layer, nq + nk:] = vs[layer][W + K:W + 2 * K].reshape(K, nk).cpu()
+    dev_in = torch.empty((w.layers, per_layer), dtype=host_in.dtype, device="cuda")
+    dev_out = torch.empty((w.layers,) + tuple(outs[0].shape), dtype=outs[0].dtype, device="cuda")
+    host_out = torch.empty((K,) + tuple(dev_out.shape), dtype=dev_out.dtype).pin_memory()
+    esz = host_in.element_size()
+    qp = [dev_in[layer].data_ptr() for layer in range(w.layers)]
+    kp = [p + nq * esz for p in qp]
+    vp = [p + (nq + nk) * esz for p in qp]
+    op = [dev_out[layer].data_ptr() for layer in range(w.layers)]
+    h2d = host_in[0].numel() * esz
+    d2h = dev_out.numel() * dev_out.element_size()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(K):
+        dev_in.copy_(host_in[i], non_blocking=True)
         for layer in range(w.layers):
-            dq[layer].copy_(host_q[layer][i], non_blocking=True)
-            dk[layer].copy_(host_k[layer][i], non_blocking=True)
-            dv[layer].copy_(host_v[layer][i], non_blocking=True)
             if fused:
-                B.duo_decode_step(h, layer, dq[layer].data_ptr(), dk[layer].data_ptr(),
-                                  dv[layer].data_ptr(), outs[layer].data_ptr(), 0.0, ws, wsb, sh)
-            else:
-                B.duo_append_kv(h, layer, dk[layer].data_ptr(), dv[layer].data_ptr(), 1, sh)
-                B.duo_decode_attn(h, layer, dq[layer].data_ptr(), outs[layer].data_ptr(), 0.0, ws,
+                B.duo_decode_step(h, layer, qp[layer], kp[layer], vp[layer], op[layer], 0.0, ws,
                                   wsb, sh)
-            host_o[layer][i].copy_(outs[layer], non_blocking=True)
+            else:
+                B.duo_append_kv(h, layer, kp[layer], vp[layer], 1, sh)
+                B.duo_decode_attn(h, layer, qp[layer], op[layer], 0.0, ws, wsb, sh)
+        host_out[i].copy_(dev_out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -316,6 +359,7 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
         "clocks": clk.summary(),
         "context": n_first,
         "gpu_launches": K * w.layers * (1 if fused else 2),
+        "fused": fused,
     }
     del cache
     torch.cuda.empty_cache()
@@ -601,7 +645,8 @@ def main(argv=None):
         "config": workload_config(w, args.batch, world),
         "pct_of_8tbs": 100.0 * res["value"] / world / 8000.0,
         "roofline": {"bound": "hbm", "achieved": kern["achieved_gbs"], "peak": peak,
-                     "unit": "GB/s", "frac": kern["achieved_gbs"] / peak, "traffic": None,
+                     "unit": "GB/s", "frac": kern["achieved_gbs"] / peak,
+                     "traffic": decode_traffic(kern["bytes_per_launch"]) if res["fused"] else None,
                      "kernel": kern["name"], "avg_launch_ms": kern["avg_ms"],
                      "bytes_per_launch": kern["bytes_per_launch"], "peak_kind": peak_kind},
         "e2e": {"value": res["e2e_value"], "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],

@@ -80,6 +80,7 @@ SIGNATURES = {
     "duo_kv_bytes": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
     "duo_layout_info": (_I32, [_P, _I32, ctypes.POINTER(duo_layout_view)]),
     "duo_set_decode_splits": (_I32, [_P, _I32]),
+    "duo_set_decode_reproducible": (_I32, [_P, _I32]),
     "duo_decode_splits": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "duo_poll_device_error": (_I32, [ctypes.POINTER(_I32)]),
     "duo_status_string": (ctypes.c_char_p, [_I32]),
@@ -196,6 +197,10 @@ def duo_layout_info(handle, layer):
 
 def duo_set_decode_splits(handle, splits):
     _check(lib().duo_set_decode_splits(handle, splits), "duo_set_decode_splits")
+
+
+def duo_set_decode_reproducible(handle, on):
+    _check(lib().duo_set_decode_reproducible(handle, 1 if on else 0), "duo_set_decode_reproducible")
 
 
 def duo_decode_splits(handle, layer):

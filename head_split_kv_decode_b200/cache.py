@@ -129,6 +129,10 @@ class DuoCache:
     def set_decode_splits(self, splits):
         B.duo_set_decode_splits(self.handle, splits)
 
+    def set_decode_reproducible(self, on=True):
+        """Fixed key shares per decode split: bit-identical repeated calls."""
+        B.duo_set_decode_reproducible(self.handle, on)
+
     def decode_splits(self, layer):
         return B.duo_decode_splits(self.handle, layer)
 

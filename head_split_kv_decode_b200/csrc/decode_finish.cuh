@@ -27,19 +27,23 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   const bool direct = !retrieval || P.nsplit == 1;
   T *out = reinterpret_cast<T *>(P.out) + ((int64_t)b * P.Hq + (int64_t)kvh * G) * D;
   const int64_t part = ((int64_t)b * P.n_ret + (retrieval ? pidx : 0)) * P.nsplit + split;
+  // One output element per thread and step; D is a multiple of 32, so the
+  // query head g is the same across a warp and lane w < NWARPS can hold warp
+  // w's weight 2^(m_w - M) for all lanes to fetch.
+  static_assert(D % 32 == 0 && NWARPS <= 32, "warp-uniform query head");
   for (int idx = tid; idx < G * D; idx += NT) {
     const int g = idx / D, c = idx % D;
-    float M = -INFINITY;
+    const float mw = lane < NWARPS ? red_m[lane * G + g] : -INFINITY;
+    float M = mw;
 #pragma unroll
-    for (int w = 0; w < NWARPS; ++w) M = fmaxf(M, red_m[w * G + g]);
-    float L = 0.f, O = 0.f;
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float sw = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+    float L = lane < NWARPS ? red_l[lane * G + g] * sw : 0.f;
 #pragma unroll
-    for (int w = 0; w < NWARPS; ++w) {
-      const float mw = red_m[w * G + g];
-      const float sw = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-      L += red_l[w * G + g] * sw;
-      O += red_o[(w * G + g) * D + c] * sw;
-    }
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < NWARPS; ++w) O += red_o[(w * G + g) * D + c] * __shfl_sync(0xffffffffu, sw, w);
     if (direct) {
       store_out(out + g * D + c, O / L);
     } else {
@@ -51,14 +55,20 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   }
   if (direct) return;
 
-  // ---- the last split of this head to finish merges all splits
-  __threadfence();
+  // ---- the last split of this head to finish merges all splits.  The
+  // barrier orders the CTA's partial stores before thread 0's fence, which
+  // (being cumulative) publishes them before the ticket; the CTA that draws
+  // the last ticket fences again before the barrier that lets its threads
+  // read the other splits' partials.
   __syncthreads();
   unsigned *cnt = P.ws_cnt + (int64_t)b * P.n_ret + pidx;
-  if (tid == 0) s_last = (atomicAdd(cnt, 1u) == (unsigned)(P.nsplit - 1));
+  if (tid == 0) {
+    __threadfence();
+    s_last = (atomicAdd(cnt, 1u) == (unsigned)(P.nsplit - 1));
+    if (s_last) __threadfence();
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   const int64_t part0 = ((int64_t)b * P.n_ret + pidx) * P.nsplit;
   // weights w_s = 2^(lse_s - max) per (split, query head), then the weighted
   // sum of the partials.  Warp w sums splits w, w+NWARPS, ... (U at a time,

@@ -33,7 +33,7 @@ namespace duo {
 namespace dm {
 
 constexpr int D = 128;
-constexpr int NWARPS = 8;
+constexpr int NWARPS = 16;
 // Key groups of 16 per warp iteration: the 4-bit rows are 4x smaller, so a
 // warp takes two groups to keep as many bytes in flight as the bf16 path.
 template <bool Q4>
@@ -93,7 +93,7 @@ __device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32
 }
 
 template <bool Q4, int G>
-__global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid_constant__ DecodeParams P) {
+__global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid_constant__ DecodeParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,17 +147,22 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   }
   constexpr int KG = Keys<Q4>::KG;
   constexpr int64_t T = 16 * KG;  // keys per warp tile
-  // A retrieval head with several splits balances its splits at run time: a
-  // CTA that gets less memory bandwidth takes fewer of the tiles handed out
-  // at the end (see below), so the splits finish together.  Each CTA still
-  // leaves one partial.  Streaming heads and single-split heads walk their
-  // range [k0, k1) statically.
-  const bool dynamic = retrieval && P.nsplit > 1;
+  // A retrieval head with several splits is cut into tiles of T keys.  Each
+  // split walks a fixed share of them; with P.pool the shares cover 7/8 of
+  // the tiles and the rest is claimed one tile at a time by warps that have
+  // finished (see below), so a CTA that gets less memory bandwidth takes
+  // fewer tiles and the splits finish together.  Each CTA leaves one
+  // partial.  Streaming heads and single-split heads walk [k0, k1).
+  const bool split_head = retrieval && P.nsplit > 1;
+  const bool pooled = split_head && P.pool;
   const int64_t tiles = (P.n + T - 1) / T;
-  const int64_t ts = dynamic ? (tiles - tiles / 8) / P.nsplit : 0;  // static tiles per split
+  const int64_t ts = !split_head ? 0
+                     : pooled    ? (tiles - tiles / 8) / P.nsplit
+                                 : (tiles + P.nsplit - 1) / P.nsplit;  // tiles per split share
+  const int64_t t1 = min(tiles, (int64_t)(split + 1) * ts);           // end of this split's share
   // this warp's first two tiles, [first, first + T) and the one NWARPS tiles on
-  const int64_t first = dynamic ? ((int64_t)split * ts + warp) * T : k0 + (int64_t)warp * T;
-  const int64_t last = dynamic ? (int64_t)(split + 1) * ts * T : k1;
+  const int64_t first = split_head ? ((int64_t)split * ts + warp) * T : k0 + (int64_t)warp * T;
+  const int64_t last = split_head ? min(P.n, t1 * T) : k1;
 
   // Launched with programmatic dependent launch, so this may run while the
   // previous kernel in the stream finishes.  Bring this warp's first two
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
   // row in the main pass, and adds it in a one-key pass that reads the inputs.
   const bool fused = !Q4 && P.knew != nullptr;
   const int64_t newk = retrieval ? P.n - 1 : P.new_slot;  // its row in this head's buffer
-  const bool owns_new = fused && !dynamic && newk >= k0 && newk < k1;
+  const bool owns_new = fused && !split_head && newk >= k0 && newk < k1;
   auto write_new = [&]() {  // one warp copies the new K and V rows into the cache
     const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB;
     const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
@@ -431,13 +436,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
     }
   };
   bool new_here = owns_new && warp == 0;  // this warp adds the new token at the end
-  if (dynamic) {
-    // Tiles of T keys: each split walks a static share of 7/8 of them (warps
-    // strided as in the static pass); the last eighth is a pool that warps
-    // claim one tile at a time from the head's counter once their share is
-    // done.  The first claim is issued during the warp's last static tile, so
-    // its latency overlaps that tile.
-    const int64_t t1 = (int64_t)(split + 1) * ts, pool0 = (int64_t)P.nsplit * ts;
+  if (split_head) {
+    // The first pool claim is issued during the warp's last tile of its
+    // share, so that its latency overlaps that tile.
+    const int64_t pool0 = pooled ? (int64_t)P.nsplit * ts : tiles;
     unsigned *next = P.ws_next + ((int64_t)b * P.n_ret + pidx) * kChunkCounterStride;
     auto visit = [&](int64_t tt) {
       const int64_t kb0 = tt * T;
@@ -450,9 +452,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 2) decode_mma_kernel(const __grid
     };
     unsigned c = 0;
     int64_t tt = (int64_t)split * ts + warp;
-    if (tt >= t1 && lane == 0) c = atomicAdd(next, 1u);
+    if (pooled && tt >= t1 && lane == 0) c = atomicAdd(next, 1u);
     for (; tt < t1; tt += NWARPS) {
-      if (tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
+      if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
       visit(tt);
     }
     c = __shfl_sync(0xffffffffu, c, 0);

@@ -44,6 +44,7 @@ struct duo_cache {
   int row_bytes;
   uint8_t *base;
   int forced_splits;
+  bool reproducible;       // decode splits take fixed key shares only
   bool have_cfg;           // decode launch facts, queried once per cache
   duo::DecodeConfig cfg;
 };
@@ -170,6 +171,7 @@ duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc, const u
   c->seq_len.assign(d.layers, 0);
   c->base = nullptr;
   c->forced_splits = 0;
+  c->reproducible = false;
   c->have_cfg = false;
   c->row_bytes = d.kv_dtype == DUO_INT4 ? d.head_dim / 2 : d.head_dim * elem_bytes(d.kv_dtype);
   const bool q4 = d.kv_dtype == DUO_INT4;
@@ -310,6 +312,7 @@ duo_status plan_decode(duo_cache *c, int32_t layer, int64_t n, const void *q, vo
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d.head_dim);
   p->scale_log2 = sc * 1.4426950408889634f;
   p->err = duo::device_error_word();
+  p->pool = c->reproducible ? 0 : 1;
   return DUO_OK;
 }
 
@@ -514,6 +517,12 @@ duo_status duo_layout_info(const duo_cache *c, int32_t layer, duo_layout_view *o
 duo_status duo_set_decode_splits(duo_cache *c, int32_t splits) {
   if (!c || splits < 0 || splits > DUO_MAX_SPLITS) return DUO_ERR_ARG;
   c->forced_splits = splits;
+  return DUO_OK;
+}
+
+duo_status duo_set_decode_reproducible(duo_cache *c, int32_t on) {
+  if (!c || (on != 0 && on != 1)) return DUO_ERR_ARG;
+  c->reproducible = on == 1;
   return DUO_OK;
 }
 

@@ -71,6 +71,9 @@ struct DecodeParams {
   const void *knew, *vnew;
   int64_t new_slot;    // streaming slot of position n-1
   int pdl;             // launched with programmatic dependent launch
+  int pool;            // tensor-core decode: the last eighth of a split head's
+                       // tiles is claimed at run time (0: every split gets an
+                       // even, fixed share)
 };
 
 struct PrefillParams {

@@ -221,6 +221,19 @@ duo_status duo_layout_info(const duo_cache *cache, int32_t layer,
  * depends on it beyond rounding. */
 duo_status duo_set_decode_splits(duo_cache *cache, int32_t splits);
 
+/* How the tensor-core decode (bf16 and 4-bit caches, head_dim 128) shares a
+ * split retrieval head's keys among its splits.  By default (on = 0) each
+ * split takes a fixed share of 7/8 of the key tiles and the last eighth goes,
+ * one tile at a time, to whichever warps finish first, so that splits running
+ * on SMs that get less memory bandwidth do less work and all finish together.
+ * Which keys each split sums then varies between calls, and outputs can differ
+ * in the last bits.  on = 1 gives every split an even fixed share instead:
+ * repeated calls on the same cache state return bit-identical outputs, at
+ * about 1-2% more time per call at long contexts.  Applies to duo_decode_attn,
+ * duo_decode_step and duo_decode_attn_static.  Errors: DUO_ERR_ARG for a null
+ * cache or on outside {0, 1}. */
+duo_status duo_set_decode_reproducible(duo_cache *cache, int32_t on);
+
 /* Split count the next decode of this layer will use. */
 duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
                              int32_t *splits);

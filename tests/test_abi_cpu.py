@@ -121,6 +121,10 @@ def test_calls_before_bind_fail_cleanly(lib):
             B.duo_set_decode_splits(h, B.MAX_SPLITS + 1)
         B.duo_set_decode_splits(h, 7)
         B.duo_set_decode_splits(h, 0)
+        assert B.STATUS_NAMES[lib.duo_set_decode_reproducible(h, 2)] == "DUO_ERR_ARG"
+        assert B.STATUS_NAMES[lib.duo_set_decode_reproducible(None, 1)] == "DUO_ERR_ARG"
+        B.duo_set_decode_reproducible(h, True)
+        B.duo_set_decode_reproducible(h, False)
     finally:
         B.duo_cache_destroy(h)
 

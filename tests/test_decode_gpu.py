@@ -195,3 +195,25 @@ def test_decode_step_fused_append(kind, D, Hq, Hkv):
             ref = _oracle(K[:, :t + 1], V[:, :t + 1], Q[:, t], mask, S, R)
             assert_parity(out, ref, kind, "step t=%d" % t)
     _check_cache_bytes(cache, K, V, mask, S, R)
+
+
+@pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
+def test_reproducible_mode(kind, D):
+    """Fixed split shares: repeated decodes of one cache state are bit-identical;
+    the default (pooled) mode agrees with them within rounding; both match the
+    oracle."""
+    B, Hq, Hkv, n, S, R = 2, 8, 2, 20000, 16, 128
+    cache, K, V, q, mask = _build(B, Hq, Hkv, D, kind, n, S, R, n_ret=1, seed=123,
+                                  chunks=[8192, 8192])
+    assert cache.decode_splits(0) > 1
+    ref = _oracle(K, V, q, mask, S, R)
+    cache.set_decode_reproducible(True)
+    outs = [cache.decode(0, q).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+    assert_parity(outs[0], ref, kind, "reproducible")
+    cache.set_decode_reproducible(False)
+    pooled = cache.decode(0, q)
+    assert_parity(pooled, ref, kind, "pooled")
+    assert (pooled.float() - outs[0].float()).abs().max().item() <= 2e-2

@@ -55,8 +55,9 @@ def test_static_decode_matches_workspace_decode_twice():
 
 def test_static_decode_refuses_oversized_layer():
     # 16 batch rows x 1 retrieval head x 313 splits x G=4 x 129 floats x 4 B
-    # = 10.3 MB > 8 MiB
-    batch, n = 16, 40000
+    # = 10.3 MB > 8 MiB (80000 keys in at most 512 splits rounded up to whole
+    # tiles of 128 or 256 keys: 313 splits of 256)
+    batch, n = 16, 80000
     cache, K, V, Q = _cache(batch, n, 900)
     cache.set_decode_splits(512)
     q = Q[:, n - 1].contiguous()
