@@ -18,6 +18,7 @@ bounded sample of the same workload instead.
 """
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -566,6 +567,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["duo", "reference"], default="duo")
     ap.add_argument("--workload", default="llama3_8b_gqa_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=0,
+                    help="decode only the first N layers of the workload (a small case for "
+                         "profiling; 0 = all layers)")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--extra", action="store_true",
                     help="also time batch 4 at 128K and the MHA 32K workload")
@@ -575,6 +579,8 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = dataclasses.replace(w, layers=min(args.layers, w.layers))
     if args.impl == "reference":
         return reference_arm(args, w, args.batch)
 
