@@ -367,6 +367,93 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
     return res
 
 
+def run_paged_mixed(args, w, rank, world, peaks):
+    """Decode of a mixed-length batch on the paged layout: every row (one
+    sequence, w.row_lengths tokens of context) takes one fused step per layer,
+    all rows in one launch, each at its own position."""
+    from head_split_kv_decode_b200.cache import DuoCache
+
+    K, Wm = min(args.steps, w.steps), args.warmup
+    lens = list(w.row_lengths)
+    B_ = len(lens)
+    mask = synth.workload_mask(w)
+    b_ids = replica_batch_ids(rank, B_)  # distinct sequences on every rank
+    total_steps = Wm + K
+    pool = sum((n + total_steps + 1 + B.PAGE_TOKENS - 1) // B.PAGE_TOKENS for n in lens)
+    cache = DuoCache(w.layers, B_, w.n_q_heads, w.n_kv_heads, w.head_dim, "bf16",
+                     max(lens) + total_steps + 1, mask, w.S, w.R, pool_blocks=pool)
+    dt = torch.bfloat16
+    t0 = time.time()
+    for layer in range(w.layers):
+        for r, n in enumerate(lens):
+            for p0 in range(0, n, 16384):
+                pos = range(p0, min(n, p0 + 16384))
+                k = synth.history(w, layer, "k", [b_ids[r]], pos, device="cuda", mask_row=mask[layer])
+                v = synth.history(w, layer, "v", [b_ids[r]], pos, device="cuda", mask_row=mask[layer])
+                cache.append_rows(layer, [r], k.to(dt).contiguous(), v.to(dt).contiguous())
+        torch.cuda.synchronize()
+    fill_s = time.time() - t0
+    # per layer and step: q [B, Hq, d], k/v [B, Hkv, d], row r at position lens[r] + step
+    qs, ks, vs = [], [], []
+    for layer in range(w.layers):
+        qr, kr, vr = [], [], []
+        for r, n in enumerate(lens):
+            pos = range(n, n + total_steps)
+            qr.append(synth.queries(w, layer, [b_ids[r]], pos, device="cuda")[0])
+            kr.append(synth.history(w, layer, "k", [b_ids[r]], pos, device="cuda", mask_row=mask[layer])[0])
+            vr.append(synth.history(w, layer, "v", [b_ids[r]], pos, device="cuda", mask_row=mask[layer])[0])
+        qs.append(torch.stack(qr, 1).to(dt).contiguous())  # [steps, B, Hq, d]
+        ks.append(torch.stack(kr, 1).to(dt).contiguous())
+        vs.append(torch.stack(vr, 1).to(dt).contiguous())
+    out = torch.empty(B_, w.n_q_heads, w.head_dim, dtype=dt, device="cuda")
+    lib = B.lib()
+    h, sh = cache.handle, torch.cuda.current_stream().cuda_stream
+    ws, wsb = cache.ws_ptr, cache.ws_bytes
+
+    def step(s):
+        for layer in range(w.layers):
+            st = lib.duo_decode_step(h, layer, qs[layer][s].data_ptr(), ks[layer][s].data_ptr(),
+                                     vs[layer][s].data_ptr(), out.data_ptr(), 0.0, ws, wsb, sh)
+            if st:
+                raise B.DuoError(st, "duo_decode_step")
+
+    for s in range(Wm):
+        step(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        step(Wm + i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks([ms], world, "cuda")[0]
+    if B.duo_poll_device_error() != 0:
+        raise RuntimeError("a bounded device wait gave up during the benchmark")
+    n_ret = [int(mask[layer].sum()) for layer in range(w.layers)]
+    step_bytes = 0
+    for i in range(K):
+        for layer in range(w.layers):
+            for n in lens:
+                step_bytes += decode_bytes_per_layer(w, 1, n + Wm + i + 1, n_ret[layer],
+                                                     w.n_kv_heads - n_ret[layer])
+                step_bytes += append_bytes(w, 1)
+    step_bytes /= K
+    launches = K * w.layers
+    res = {"workload": w.name, "row_lengths": lens, "pool_blocks": pool,
+           "value": aggregate_rate(step_bytes, world, K, ms), "unit": "GB/s",
+           "ms_per_step": ms / K, "kernel_avg_launch_ms": ms / launches,
+           "bytes_per_launch": step_bytes / w.layers, "gpu_launches": launches,
+           "decode_splits": cache.decode_splits(0), "fill_s": fill_s}
+    res["kernel_achieved_gbs"] = res["bytes_per_launch"] / (res["kernel_avg_launch_ms"] * 1e-3) / 1e9
+    res["frac"] = res["kernel_achieved_gbs"] / peaks["hbm_gbs"]
+    del cache
+    torch.cuda.empty_cache()
+    return res
+
+
 # --------------------------------------------------------------------------- prefill
 
 
@@ -619,6 +706,8 @@ def main(argv=None):
                           "kernel_achieved_gbs": rx["kernel"]["achieved_gbs"],
                           "frac": rx["kernel"]["achieved_gbs"] / peaks["hbm_gbs"],
                           "decode_splits": rx["splits"], "gpu_launches": rx["gpu_launches"]}
+        extra["llama3_8b_gqa_paged_mixed"] = run_paged_mixed(
+            args, synth.WORKLOADS["llama3_8b_gqa_paged_mixed"], rank, world, peaks)
     prefill = None
     if not args.no_prefill:
         try:

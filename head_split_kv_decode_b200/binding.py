@@ -16,6 +16,8 @@ LIB_PATH = os.path.join(_HERE, "libduo.so")
 MAX_KV_HEADS = 64
 MAX_SPLITS = 512
 DECODE_STATIC_SCRATCH_BYTES = 8 << 20
+PAGE_TOKENS = 256
+MAX_LAUNCH_ROWS = 128
 
 DUO_OK = 0
 STATUS_NAMES = {
@@ -25,6 +27,7 @@ STATUS_NAMES = {
 }
 DUO_F32, DUO_BF16, DUO_INT4 = 0, 1, 2
 DUO_LAYOUT_PACKED = 0
+DUO_LAYOUT_PAGED = 1
 KV_DTYPES = {"f32": DUO_F32, "bf16": DUO_BF16, "int4": DUO_INT4}
 
 
@@ -55,7 +58,10 @@ class duo_layout_view(ctypes.Structure):
                 ("ret_k_sz", ctypes.c_int64), ("ret_v_sz", ctypes.c_int64),
                 ("str_k_sz", ctypes.c_int64), ("str_v_sz", ctypes.c_int64),
                 ("kind", ctypes.c_int32 * MAX_KV_HEADS),
-                ("packed_index", ctypes.c_int32 * MAX_KV_HEADS)]
+                ("packed_index", ctypes.c_int32 * MAX_KV_HEADS),
+                ("layout", ctypes.c_int32), ("page_tokens", ctypes.c_int32),
+                ("table_stride", ctypes.c_int32),
+                ("pool_blocks", ctypes.c_int64), ("block_table", ctypes.c_int64)]
 
 
 _P = ctypes.c_void_p
@@ -67,16 +73,25 @@ _F = ctypes.c_float
 # name -> (restype, argtypes); every function of include/duo.h
 SIGNATURES = {
     "duo_cache_create": (_I32, [ctypes.POINTER(_P), ctypes.POINTER(duo_cache_desc), _P, _I32, _I32, _I32]),
+    "duo_cache_create_paged": (_I32, [ctypes.POINTER(_P), ctypes.POINTER(duo_cache_desc), _P, _I32, _I32, _I64]),
     "duo_cache_destroy": (None, [_P]),
     "duo_cache_required_bytes": (_I32, [_P, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]),
     "duo_cache_bind": (_I32, [_P, _P, _SZ]),
     "duo_cache_reset": (_I32, [_P]),
+    "duo_release_rows": (_I32, [_P, _P, _I32]),
     "duo_append_kv": (_I32, [_P, _I32, _P, _P, _I32, _P]),
+    "duo_append_kv_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _I32, _P]),
     "duo_decode_attn": (_I32, [_P, _I32, _P, _P, _F, _P, _SZ, _P]),
+    "duo_decode_attn_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _F, _P, _SZ, _P]),
     "duo_decode_step": (_I32, [_P, _I32, _P, _P, _P, _P, _F, _P, _SZ, _P]),
+    "duo_decode_step_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "duo_decode_attn_static": (_I32, [_P, _I32, _P, _P, _F, _P]),
     "duo_prefill_attn": (_I32, [_P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
+    "duo_prefill_attn_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _F, _P]),
     "duo_seq_len": (_I32, [_P, _I32, ctypes.POINTER(_I64)]),
+    "duo_row_seq_len": (_I32, [_P, _I32, _I32, ctypes.POINTER(_I64)]),
+    "duo_row_blocks": (_I32, [_P, _I32, _P, _I32, ctypes.POINTER(_I32)]),
+    "duo_pool_free_blocks": (_I32, [_P, ctypes.POINTER(_I64)]),
     "duo_kv_bytes": (_I32, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
     "duo_layout_info": (_I32, [_P, _I32, ctypes.POINTER(duo_layout_view)]),
     "duo_set_decode_splits": (_I32, [_P, _I32]),
@@ -115,19 +130,96 @@ def duo_status_string(status):
     return lib().duo_status_string(status).decode()
 
 
-def duo_cache_create(layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype, capacity,
-                     head_mask, S, R, layout=DUO_LAYOUT_PACKED):
-    """head_mask: bytes-like / array of layers*n_kv_heads 0/1 values.  Returns a handle."""
+def _desc_and_mask(layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype, capacity, head_mask):
     desc = duo_cache_desc(layers, batch, n_q_heads, n_kv_heads, head_dim,
                           KV_DTYPES.get(kv_dtype, kv_dtype), capacity)
     vals = [int(x) for x in head_mask]
     if len(vals) != layers * n_kv_heads or any(not 0 <= x <= 255 for x in vals):
         raise ValueError("head_mask must hold layers * n_kv_heads byte values")
-    mask = (ctypes.c_uint8 * len(vals))(*vals)
+    return desc, (ctypes.c_uint8 * len(vals))(*vals)
+
+
+def duo_cache_create(layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype, capacity,
+                     head_mask, S, R, layout=DUO_LAYOUT_PACKED):
+    """head_mask: bytes-like / array of layers*n_kv_heads 0/1 values.  Returns a handle."""
+    desc, mask = _desc_and_mask(layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype,
+                                capacity, head_mask)
     out = _P()
     _check(lib().duo_cache_create(ctypes.byref(out), ctypes.byref(desc), mask, S, R, layout),
            "duo_cache_create")
     return out.value
+
+
+def duo_cache_create_paged(layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype, capacity,
+                           head_mask, S, R, pool_blocks):
+    desc, mask = _desc_and_mask(layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype,
+                                capacity, head_mask)
+    out = _P()
+    _check(lib().duo_cache_create_paged(ctypes.byref(out), ctypes.byref(desc), mask, S, R,
+                                        pool_blocks), "duo_cache_create_paged")
+    return out.value
+
+
+def _rows(rows):
+    """(pointer, count) of an int32 row list; (None, 0) for every row."""
+    if rows is None:
+        return None, 0
+    vals = [int(r) for r in rows]
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr, len(vals)
+
+
+def duo_release_rows(handle, rows=None):
+    arr, n = _rows(rows)
+    _check(lib().duo_release_rows(handle, arr, n), "duo_release_rows")
+
+
+def duo_append_kv_rows(handle, layer, rows, k_ptr, v_ptr, n_tokens, stream=0):
+    arr, n = _rows(rows)
+    _check(lib().duo_append_kv_rows(handle, layer, arr, n, k_ptr, v_ptr, n_tokens, stream),
+           "duo_append_kv_rows")
+
+
+def duo_decode_attn_rows(handle, layer, rows, q_ptr, out_ptr, softmax_scale, ws_ptr, ws_bytes,
+                         stream=0):
+    arr, n = _rows(rows)
+    _check(lib().duo_decode_attn_rows(handle, layer, arr, n, q_ptr, out_ptr, softmax_scale, ws_ptr,
+                                      ws_bytes, stream), "duo_decode_attn_rows")
+
+
+def duo_decode_step_rows(handle, layer, rows, q_ptr, k_new_ptr, v_new_ptr, out_ptr, softmax_scale,
+                         ws_ptr, ws_bytes, stream=0):
+    arr, n = _rows(rows)
+    _check(lib().duo_decode_step_rows(handle, layer, arr, n, q_ptr, k_new_ptr, v_new_ptr, out_ptr,
+                                      softmax_scale, ws_ptr, ws_bytes, stream),
+           "duo_decode_step_rows")
+
+
+def duo_prefill_attn_rows(handle, layer, rows, q_ptr, k_ptr, v_ptr, C, out_ptr, softmax_scale,
+                          stream=0):
+    arr, n = _rows(rows)
+    _check(lib().duo_prefill_attn_rows(handle, layer, arr, n, q_ptr, k_ptr, v_ptr, C, out_ptr,
+                                       softmax_scale, stream), "duo_prefill_attn_rows")
+
+
+def duo_row_seq_len(handle, layer, row):
+    n = _I64()
+    _check(lib().duo_row_seq_len(handle, layer, row, ctypes.byref(n)), "duo_row_seq_len")
+    return n.value
+
+
+def duo_row_blocks(handle, row):
+    n = _I32()
+    _check(lib().duo_row_blocks(handle, row, None, 0, ctypes.byref(n)), "duo_row_blocks")
+    arr = (ctypes.c_int32 * max(1, n.value))()
+    _check(lib().duo_row_blocks(handle, row, arr, n.value, ctypes.byref(n)), "duo_row_blocks")
+    return list(arr[:n.value])
+
+
+def duo_pool_free_blocks(handle):
+    n = _I64()
+    _check(lib().duo_pool_free_blocks(handle, ctypes.byref(n)), "duo_pool_free_blocks")
+    return n.value
 
 
 def duo_cache_destroy(handle):

@@ -30,13 +30,23 @@ class DuoCache:
 
     head_mask: [layers, n_kv_heads] of 0/1 (1 = retrieval head).
     kv_dtype: "f32", "bf16" or "int4" (K/V given in bf16 and quantised on append).
+    pool_blocks: None for the packed layout (``capacity`` tokens reserved per
+    batch row), or the block count of the paged layout's retrieval pool
+    (blocks of ``binding.PAGE_TOKENS`` tokens taken by rows as they grow;
+    ``capacity`` then bounds one row).  Each batch row is a sequence slot with
+    its own length; the ``*_rows`` methods act on a list of rows.
     """
 
     def __init__(self, layers, batch, n_q_heads, n_kv_heads, head_dim, kv_dtype, capacity,
-                 head_mask, S, R, device="cuda"):
+                 head_mask, S, R, device="cuda", pool_blocks=None):
         mask = torch.as_tensor(head_mask).reshape(-1).to(torch.uint8).tolist()
-        self.handle = B.duo_cache_create(layers, batch, n_q_heads, n_kv_heads, head_dim,
-                                         kv_dtype, capacity, mask, S, R)
+        if pool_blocks is None:
+            self.handle = B.duo_cache_create(layers, batch, n_q_heads, n_kv_heads, head_dim,
+                                             kv_dtype, capacity, mask, S, R)
+        else:
+            self.handle = B.duo_cache_create_paged(layers, batch, n_q_heads, n_kv_heads, head_dim,
+                                                   kv_dtype, capacity, mask, S, R, pool_blocks)
+        self.paged = pool_blocks is not None
         self.layers, self.batch = layers, batch
         self.n_q_heads, self.n_kv_heads, self.head_dim = n_q_heads, n_kv_heads, head_dim
         self.kv_dtype, self.capacity, self.S, self.R = kv_dtype, capacity, S, R
@@ -116,6 +126,77 @@ class DuoCache:
                            _stream_handle(stream, self.device))
         return out
 
+    # ------------------------------------------------------------ row calls
+    def _rows(self, rows):
+        rows = [int(r) for r in rows]
+        if not rows:
+            raise ValueError("empty row list")
+        return rows
+
+    def append_rows(self, layer, rows, k, v, stream=None):
+        """k, v: [len(rows), n_tokens, n_kv_heads, head_dim] for the listed rows."""
+        rows = self._rows(rows)
+        n = k.shape[1]
+        shape = (len(rows), n, self.n_kv_heads, self.head_dim)
+        self._check(k, shape, "k")
+        self._check(v, shape, "v")
+        B.duo_append_kv_rows(self.handle, layer, rows, k.data_ptr(), v.data_ptr(), n,
+                             _stream_handle(stream, self.device))
+
+    def decode_rows(self, layer, rows, q, out=None, scale=0.0, stream=None):
+        """q: [len(rows), n_q_heads, head_dim], each row's query at its last position."""
+        rows = self._rows(rows)
+        shape = (len(rows), self.n_q_heads, self.head_dim)
+        self._check(q, shape, "q")
+        if out is None:
+            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
+        self._check(out, shape, "out")
+        B.duo_decode_attn_rows(self.handle, layer, rows, q.data_ptr(), out.data_ptr(), float(scale),
+                               self.ws_ptr, self.ws_bytes, _stream_handle(stream, self.device))
+        return out
+
+    def step_rows(self, layer, rows, q, k_new, v_new, out=None, scale=0.0, stream=None):
+        """Append one token to each listed row and attend (see :meth:`step`)."""
+        rows = self._rows(rows)
+        kv_shape = (len(rows), self.n_kv_heads, self.head_dim)
+        shape = (len(rows), self.n_q_heads, self.head_dim)
+        self._check(q, shape, "q")
+        self._check(k_new, kv_shape, "k_new")
+        self._check(v_new, kv_shape, "v_new")
+        if out is None:
+            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
+        self._check(out, shape, "out")
+        B.duo_decode_step_rows(self.handle, layer, rows, q.data_ptr(), k_new.data_ptr(),
+                               v_new.data_ptr(), out.data_ptr(), float(scale), self.ws_ptr,
+                               self.ws_bytes, _stream_handle(stream, self.device))
+        return out
+
+    def prefill_rows(self, layer, rows, q, k, v, out=None, scale=0.0, stream=None):
+        """q: [len(rows), C, n_q_heads, d]; k, v: [len(rows), C, n_kv_heads, d]."""
+        rows = self._rows(rows)
+        C = q.shape[1]
+        self._check(q, (len(rows), C, self.n_q_heads, self.head_dim), "q")
+        self._check(k, (len(rows), C, self.n_kv_heads, self.head_dim), "k")
+        self._check(v, (len(rows), C, self.n_kv_heads, self.head_dim), "v")
+        if out is None:
+            out = torch.empty_like(q)
+        self._check(out, tuple(q.shape), "out")
+        B.duo_prefill_attn_rows(self.handle, layer, rows, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                C, out.data_ptr(), float(scale), _stream_handle(stream, self.device))
+        return out
+
+    def release_rows(self, rows=None):
+        B.duo_release_rows(self.handle, None if rows is None else self._rows(rows))
+
+    def row_seq_len(self, layer, row):
+        return B.duo_row_seq_len(self.handle, layer, row)
+
+    def row_blocks(self, row):
+        return B.duo_row_blocks(self.handle, row)
+
+    def pool_free_blocks(self):
+        return B.duo_pool_free_blocks(self.handle)
+
     # ------------------------------------------------------------ introspection
     def seq_len(self, layer):
         return B.duo_seq_len(self.handle, layer)
@@ -144,17 +225,33 @@ class DuoCache:
 
         name in ret_k, ret_v, str_k, str_v (rows of K/V elements or int4 codes) and,
         for int4, ret_k_sz, ret_v_sz, str_k_sz, str_v_sz (fp16 scale/zero pairs).
-        Returns a uint8 tensor [batch, heads, rows, row_bytes] (or [..., 4]).
+        Returns a uint8 tensor [batch, heads, rows, row_bytes] (or [..., 4]);
+        paged retrieval buffers are [pool_blocks, heads, page_tokens, ...].
         """
         lv = self.layout(layer)
         off = getattr(lv, name)
         if off < 0:
             return None
         heads = lv.n_retrieval if name.startswith("ret") else lv.n_streaming
-        rows = lv.capacity if name.startswith("ret") else lv.window_stride
+        outer, rows = self.batch, (lv.capacity if name.startswith("ret") else lv.window_stride)
+        if self.paged and name.startswith("ret"):
+            outer, rows = lv.pool_blocks, lv.page_tokens
         width = 4 if name.endswith("_sz") else lv.row_bytes
-        nbytes = self.batch * heads * rows * width
-        return self.storage[off:off + nbytes].view(self.batch, heads, rows, width)
+        nbytes = outer * heads * rows * width
+        return self.storage[off:off + nbytes].view(outer, heads, rows, width)
+
+    def gather_rows(self, layer, name, row, n):
+        """The first n retrieval rows of one batch row, in position order, as
+        [heads, n, width] (packed: a slice; paged: through the block table)."""
+        reg = self.region(layer, name)
+        if reg is None:
+            return None
+        if not self.paged:
+            return reg[row, :, :n]
+        P = self.layout(layer).page_tokens
+        blocks = self.row_blocks(row)
+        parts = [reg[blk] for blk in blocks[:(n + P - 1) // P]]
+        return torch.cat(parts, dim=1)[:, :n]
 
     def close(self):
         if getattr(self, "handle", None):

@@ -17,8 +17,7 @@ namespace duo {
 // One thread per 16-byte chunk of one (token, KV head) row of K and of V.
 __global__ void append_kernel(const __grid_constant__ AppendParams a, int row_bytes) {
   const int ch = row_bytes / 16;
-  const int64_t total = (int64_t)a.B * a.n_tok * a.Hkv * ch;
-  const int64_t end = a.n_cur + a.n_tok;
+  const int64_t total = (int64_t)a.rows.n * a.n_tok * a.Hkv * ch;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int c = (int)(i % ch);
@@ -26,23 +25,24 @@ __global__ void append_kernel(const __grid_constant__ AppendParams a, int row_by
     const int h = (int)(r % a.Hkv);
     r /= a.Hkv;
     const int64_t t = r % a.n_tok;
-    const int b = (int)(r / a.n_tok);
-    const int64_t p = a.n_cur + t;
+    const int lr = (int)(r / a.n_tok);  // launch row
+    const int b = a.rows.row[lr];
+    const int64_t p = a.rows.len[lr] + t;
+    const int64_t end = a.rows.len[lr] + a.n_tok;
     const int idx = a.h.index[h];
     int64_t off;
     uint8_t *dk, *dv;
     if (a.h.kind[h]) {
-      off = (((int64_t)b * a.n_ret + idx) * a.cap + p) * row_bytes;
+      off = ret_row(a.ret, b, idx, p) * row_bytes;
       dk = a.p.ret_k;
       dv = a.p.ret_v;
     } else {
       if (!(p < a.S || p >= end - a.R)) continue;
-      const int64_t slot = p < a.S ? p : a.S + (p - a.S) % a.R;
-      off = (((int64_t)b * a.n_str + idx) * a.Ws + slot) * row_bytes;
+      off = (((int64_t)b * a.n_str + idx) * a.Ws + ring_slot(p, a.S, a.R)) * row_bytes;
       dk = a.p.str_k;
       dv = a.p.str_v;
     }
-    // The input is [B][n_tok][Hkv][row], so chunk i of the input is chunk i.
+    // The input is [rows][n_tok][Hkv][row], so chunk i of the input is chunk i.
     const uint4 kk = __ldg(reinterpret_cast<const uint4 *>(a.k) + i);
     const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(a.v) + i);
     reinterpret_cast<uint4 *>(dk + off)[c] = kk;
@@ -60,8 +60,7 @@ __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
   constexpr int CPL = D / 32;
   static_assert(CPL == 2 || CPL == 4, "head_dim 64 or 128");
   const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)a.B * a.n_tok * a.Hkv * 2;
-  const int64_t end = a.n_cur + a.n_tok;
+  const int64_t warps = (int64_t)a.rows.n * a.n_tok * a.Hkv * 2;
   const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t w = gw; w < warps; w += nw) {
@@ -70,24 +69,25 @@ __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
     const int h = (int)(r % a.Hkv);
     r /= a.Hkv;
     const int64_t t = r % a.n_tok;
-    const int b = (int)(r / a.n_tok);
-    const int64_t p = a.n_cur + t;
+    const int lr = (int)(r / a.n_tok);  // launch row
+    const int b = a.rows.row[lr];
+    const int64_t p = a.rows.len[lr] + t;
+    const int64_t end = a.rows.len[lr] + a.n_tok;
     const int idx = a.h.index[h];
     int64_t row;
     uint8_t *codes, *sz;
     if (a.h.kind[h]) {
-      row = ((int64_t)b * a.n_ret + idx) * a.cap + p;
+      row = ret_row(a.ret, b, idx, p);
       codes = which ? a.p.ret_v : a.p.ret_k;
       sz = which ? a.p.ret_v_sz : a.p.ret_k_sz;
     } else {
       if (!(p < a.S || p >= end - a.R)) continue;
-      const int64_t slot = p < a.S ? p : a.S + (p - a.S) % a.R;
-      row = ((int64_t)b * a.n_str + idx) * a.Ws + slot;
+      row = ((int64_t)b * a.n_str + idx) * a.Ws + ring_slot(p, a.S, a.R);
       codes = which ? a.p.str_v : a.p.str_k;
       sz = which ? a.p.str_v_sz : a.p.str_k_sz;
     }
     const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(which ? a.v : a.k) +
-                               (((int64_t)b * a.n_tok + t) * a.Hkv + h) * D + lane * CPL;
+                               (((int64_t)lr * a.n_tok + t) * a.Hkv + h) * D + lane * CPL;
     float x[CPL];
     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
@@ -128,10 +128,22 @@ __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
   }
 }
 
+// Block-table writes of the paged layout: one thread per entry.
+__global__ void table_write_kernel(int32_t *table, const __grid_constant__ TableWrites w) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < w.n) table[w.index[i]] = w.block[i];
+}
+
+cudaError_t launch_table_writes(int32_t *table, const TableWrites &w, cudaStream_t s) {
+  if (w.n <= 0) return cudaSuccess;
+  table_write_kernel<<<1, kMaxTableWrites, 0, s>>>(table, w);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendParams &a, int kv_type, cudaStream_t s) {
-  if (a.n_tok <= 0) return cudaSuccess;
+  if (a.n_tok <= 0 || a.rows.n <= 0) return cudaSuccess;
   if (kv_type == kINT4) {
-    const int64_t warps = (int64_t)a.B * a.n_tok * a.Hkv * 2;
+    const int64_t warps = (int64_t)a.rows.n * a.n_tok * a.Hkv * 2;
     const int threads = 256;
     const int64_t blocks = (warps * 32 + threads - 1) / threads;
     const int grid = (int)(blocks < 148 * 64 ? blocks : 148 * 64);
@@ -142,7 +154,7 @@ cudaError_t launch_append(const AppendParams &a, int kv_type, cudaStream_t s) {
     return cudaGetLastError();
   }
   const int row_bytes = a.D * (kv_type == kF32 ? 4 : 2);
-  const int64_t total = (int64_t)a.B * a.n_tok * a.Hkv * (row_bytes / 16);
+  const int64_t total = (int64_t)a.rows.n * a.n_tok * a.Hkv * (row_bytes / 16);
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
   const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);

@@ -140,4 +140,18 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __fl
 __device__ __forceinline__ float load_in(const float *p) { return *p; }
 __device__ __forceinline__ float load_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 
+// Storage row of retrieval key `key` of (batch row b, retrieval head pidx);
+// see RetMap.
+__device__ __forceinline__ int64_t ret_row(const RetMap &m, int b, int pidx, int64_t key) {
+  if (!m.table) return ((int64_t)b * m.n_ret + pidx) * m.cap + key;
+  const int64_t blk = m.table[(int64_t)b * m.stride + (key >> kPageShift)];
+  return ((blk * m.n_ret + pidx) << kPageShift) + (key & (kPageTokens - 1));
+}
+
+// Ring slot of position p in a streaming head's buffer: sinks first, then
+// an R-slot ring.
+__device__ __forceinline__ int64_t ring_slot(int64_t p, int S, int R) {
+  return p < S ? p : S + (p - S) % R;
+}
+
 }  // namespace duo

@@ -12,21 +12,22 @@ namespace duo {
 // Second half of the epilogue: the per-warp states of the CTA are staged in
 // shared memory as red_m [NWARPS][G], red_l [NWARPS][G] (log2 units) and
 // red_o [NWARPS][G][D] (unnormalised), all starting at `smem`.  Combines them,
-// writes the output (single split) or this split's normalised partial and
-// log-sum-exp, and lets the last split of the head merge every partial.
+// writes the output `out` (the G rows of this KV head's query heads) when
+// `direct`, or else this split's normalised partial and log-sum-exp into
+// slot part0 + split, and lets the last of the nsplit splits of the head
+// (merge ticket `unit`) merge slots part0 .. part0 + nsplit - 1.
 template <typename T, int D, int G, int NWARPS>
 __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8_t *smem,
-                                                    int *s_last_p, bool retrieval, int b, int kvh,
-                                                    int pidx, int split) {
+                                                    int *s_last_p, bool direct, T *out,
+                                                    int64_t unit, int64_t part0, int nsplit,
+                                                    int split) {
   constexpr int NT = NWARPS * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int &s_last = *s_last_p;
   const float *red_m = reinterpret_cast<const float *>(smem);
   const float *red_l = red_m + NWARPS * G;
   const float *red_o = red_l + NWARPS * G;
-  const bool direct = !retrieval || P.nsplit == 1;
-  T *out = reinterpret_cast<T *>(P.out) + ((int64_t)b * P.Hq + (int64_t)kvh * G) * D;
-  const int64_t part = ((int64_t)b * P.n_ret + (retrieval ? pidx : 0)) * P.nsplit + split;
+  const int64_t part = part0 + split;
   // One output element per thread and step; D is a multiple of 32, so the
   // query head g is the same across a warp and lane w < NWARPS can hold warp
   // w's weight 2^(m_w - M) for all lanes to fetch.
@@ -61,24 +62,23 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   // the last ticket fences again before the barrier that lets its threads
   // read the other splits' partials.
   __syncthreads();
-  unsigned *cnt = P.ws_cnt + (int64_t)b * P.n_ret + pidx;
+  unsigned *cnt = P.ws_cnt + unit;
   if (tid == 0) {
     __threadfence();
-    s_last = (atomicAdd(cnt, 1u) == (unsigned)(P.nsplit - 1));
+    s_last = (atomicAdd(cnt, 1u) == (unsigned)(nsplit - 1));
     if (s_last) __threadfence();
   }
   __syncthreads();
   if (!s_last) return;
-  const int64_t part0 = ((int64_t)b * P.n_ret + pidx) * P.nsplit;
   // weights w_s = 2^(lse_s - max) per (split, query head), then the weighted
   // sum of the partials.  Warp w sums splits w, w+NWARPS, ... (U at a time,
   // their loads in flight together); lane l owns channels [4l, 4l+4) of every
   // query head (D/4 float4 per head row; for D = 64 the upper lanes idle).
   // The first batch of partials is loaded before the weights are reduced, so
   // that its latency overlaps that reduction.
-  float *s_w = reinterpret_cast<float *>(smem);        // [nsplit][G]
-  float *s_den = s_w + P.nsplit * G;                   // [G]
-  float *s_acc = s_w + ((P.nsplit * G + G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
+  float *s_w = reinterpret_cast<float *>(smem);      // [nsplit][G]
+  float *s_den = s_w + nsplit * G;                   // [G]
+  float *s_acc = s_w + ((nsplit * G + G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
   constexpr int L4 = D / 4;
   constexpr int U = G >= 8 ? 2 : 4;
   const bool owns = lane < L4;
@@ -90,13 +90,13 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int sp = warp + u * NWARPS;
-      v[u][g] = (owns && sp < P.nsplit) ? __ldcg(src + (sp * G + g) * L4) : zero4;
+      v[u][g] = (owns && sp < nsplit) ? __ldcg(src + (sp * G + g) * L4) : zero4;
     }
   // warp g (and g + NWARPS, ...) reduces query head g over the splits, one
   // split per lane at a time
   for (int g = warp; g < G; g += NWARPS) {
     float M = -INFINITY;
-    for (int sp = lane; sp < P.nsplit; sp += 32) {
+    for (int sp = lane; sp < nsplit; sp += 32) {
       const float x = __ldcg(P.ws_lse + (part0 + sp) * G + g);
       s_w[sp * G + g] = x;
       M = fmaxf(M, x);
@@ -104,7 +104,7 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float den = 0.f;
-    for (int sp = lane; sp < P.nsplit; sp += 32) {
+    for (int sp = lane; sp < nsplit; sp += 32) {
       const float x = s_w[sp * G + g];
       const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);  // a split that claimed no keys
       s_w[sp * G + g] = w;
@@ -131,16 +131,16 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int su = sp + u * NWARPS;
-        if (su < P.nsplit) fma4(acc[g], s_w[su * G + g], v[u][g]);
+        if (su < nsplit) fma4(acc[g], s_w[su * G + g], v[u][g]);
       }
     sp += U * NWARPS;
-    if (sp >= P.nsplit) break;
+    if (sp >= nsplit) break;
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int su = sp + u * NWARPS;
-        v[u][g] = (owns && su < P.nsplit) ? __ldcg(src + (su * G + g) * L4) : zero4;
+        v[u][g] = (owns && su < nsplit) ? __ldcg(src + (su * G + g) * L4) : zero4;
       }
   }
   if (owns) {
@@ -157,7 +157,7 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   }
   if (tid == 0) {  // leave the ticket (and chunk counter) ready for the next call
     *cnt = 0u;
-    if (P.ws_next) P.ws_next[((int64_t)b * P.n_ret + pidx) * kChunkCounterStride] = 0u;
+    if (P.ws_next) P.ws_next[unit * kChunkCounterStride] = 0u;
   }
 }
 
@@ -213,7 +213,13 @@ __device__ __forceinline__ void decode_finish(const DecodeParams &P, uint8_t *sm
   }
   __syncthreads();
 
-  decode_reduce_store<T, D, G, NWARPS>(P, smem, s_last_p, retrieval, b, kvh, pidx, split);
+  // CUDA-core decode: packed layout, every batch row at length P.n, the
+  // retrieval CTAs enumerated as ((b*n_ret + head)*nsplit + split).
+  const int64_t unit = (int64_t)b * P.n_ret + (retrieval ? pidx : 0);
+  decode_reduce_store<T, D, G, NWARPS>(
+      P, smem, s_last_p, !retrieval || P.nsplit == 1,
+      reinterpret_cast<T *>(P.out) + ((int64_t)b * P.Hq + (int64_t)kvh * G) * D, unit,
+      unit * P.nsplit, P.nsplit, split);
 }
 
 }  // namespace duo

@@ -99,87 +99,96 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
-  // ---- work item
-  const int n_ret_ctas = P.B * P.n_ret * P.nsplit;
-  int b, kvh, pidx, split;
+  // ---- work item: retrieval CTAs first (launch row r, head, split), then
+  // one CTA per (launch row, streaming head)
+  const int n_ret_ctas = P.cta0[P.rows.n];
+  int r, kvh, pidx, split, nsplit;
   bool retrieval;
-  int64_t row0, k0, k1;
-  const uint8_t *Kb, *Vb, *Ks = nullptr, *Vs = nullptr;
   if ((int)blockIdx.x < n_ret_ctas) {
-    split = blockIdx.x % P.nsplit;
-    const int r = blockIdx.x / P.nsplit;
-    pidx = r % P.n_ret;
-    b = r / P.n_ret;
+    int lo = 0, hi = P.rows.n;  // the last r with cta0[r] <= blockIdx.x
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (P.cta0[mid] <= (int)blockIdx.x) lo = mid; else hi = mid;
+    }
+    r = lo;
+    nsplit = P.nsplit_r[r];
+    const int local = (int)blockIdx.x - P.cta0[r];
+    pidx = local / nsplit;
+    split = local % nsplit;
     kvh = P.h.ret_heads[pidx];
     retrieval = true;
-    row0 = ((int64_t)b * P.n_ret + pidx) * P.cap;
-    Kb = P.p.ret_k;
-    Vb = P.p.ret_v;
-    if (Q4) {
-      Ks = P.p.ret_k_sz;
-      Vs = P.p.ret_v_sz;
-    }
-    k0 = (int64_t)split * P.split_len;
-    k1 = min(P.n, k0 + P.split_len);
   } else {
-    const int r = blockIdx.x - n_ret_ctas;
-    pidx = r % P.n_str;
-    b = r / P.n_str;
+    const int x = (int)blockIdx.x - n_ret_ctas;
+    r = x / P.n_str;
+    pidx = x % P.n_str;
     kvh = P.h.str_heads[pidx];
     retrieval = false;
     split = 0;
-    row0 = ((int64_t)b * P.n_str + pidx) * P.Ws;
-    Kb = P.p.str_k;
-    Vb = P.p.str_v;
-    if (Q4) {
-      Ks = P.p.str_k_sz;
-      Vs = P.p.str_v_sz;
-    }
-    k0 = 0;
-    k1 = min(P.n, (int64_t)P.W);
+    nsplit = 1;
   }
+  const int b = P.rows.row[r];
+  // Key indices and tile counts are 32-bit (a row holds fewer than 2^31
+  // tokens); byte offsets are formed in 64 bits.
+  const int n = P.rows.len[r];  // tokens incl. the new one; the query is at n-1
   constexpr int RB = Q4 ? D / 2 : D * 2;  // bytes per key row
-  Kb += row0 * RB;
-  Vb += row0 * RB;
-  if (Q4) {
-    Ks += row0 * 4;
-    Vs += row0 * 4;
-  }
+  // Streaming heads: one slot buffer, first storage row srow0.  Retrieval
+  // heads: key tiles are addressed block by block (a tile never crosses a
+  // block of the paged layout), with key indices local to the block.
+  auto srow0 = [&]() { return ((int64_t)b * P.n_str + pidx) * P.Ws; };
+  const int k0 = 0, k1 = retrieval ? n : min(n, P.W);
   constexpr int KG = Keys<Q4>::KG;
-  constexpr int64_t T = 16 * KG;  // keys per warp tile
+  constexpr int T = 16 * KG;  // keys per warp tile
+  constexpr int kBlockMask = ~(kPageTokens - 1);
   // A retrieval head with several splits is cut into tiles of T keys.  Each
   // split walks a fixed share of them; with P.pool the shares cover 7/8 of
   // the tiles and the rest is claimed one tile at a time by warps that have
   // finished (see below), so a CTA that gets less memory bandwidth takes
   // fewer tiles and the splits finish together.  Each CTA leaves one
   // partial.  Streaming heads and single-split heads walk [k0, k1).
-  const bool split_head = retrieval && P.nsplit > 1;
+  const bool split_head = retrieval && nsplit > 1;
   const bool pooled = split_head && P.pool;
-  const int64_t tiles = (P.n + T - 1) / T;
-  const int64_t ts = !split_head ? 0
-                     : pooled    ? (tiles - tiles / 8) / P.nsplit
-                                 : (tiles + P.nsplit - 1) / P.nsplit;  // tiles per split share
-  const int64_t t1 = min(tiles, (int64_t)(split + 1) * ts);           // end of this split's share
+  const int tiles = (n + T - 1) / T;
+  const int ts = !split_head ? 0
+                 : pooled    ? (tiles - tiles / 8) / nsplit
+                             : (tiles + nsplit - 1) / nsplit;  // tiles per split share
+  const int t1 = min(tiles, (split + 1) * ts);                 // end of this split's share
   // this warp's first two tiles, [first, first + T) and the one NWARPS tiles on
-  const int64_t first = split_head ? ((int64_t)split * ts + warp) * T : k0 + (int64_t)warp * T;
-  const int64_t last = split_head ? min(P.n, t1 * T) : k1;
+  const int first = split_head ? (split * ts + warp) * T : k0 + warp * T;
+  const int last = split_head ? min(n, t1 * T) : k1;
 
   // Launched with programmatic dependent launch, so this may run while the
   // previous kernel in the stream finishes.  Bring this warp's first two
   // tiles into L2 meanwhile: every global write lands in L2, so a line
   // fetched now cannot be stale when the loads below (after the wait) use it.
+  // A block-table entry read now may be stale; it only aims a prefetch, and
+  // is clamped to the pool so the address stays valid.
   if (lane == 0) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int64_t kb = first + (int64_t)i * NWARPS * T;
+      const int kb = first + i * NWARPS * T;
       if (kb < last) {
-        const int64_t rows = min(T, last - kb);
-        prefetch_l2(Kb + kb * RB, (uint32_t)(rows * RB));
-        prefetch_l2(Vb + kb * RB, (uint32_t)(rows * RB));
+        const int rows = min(T, last - kb);
+        int64_t row = srow0() + kb;
+        const uint8_t *pk = P.p.str_k, *pv = P.p.str_v, *psk = P.p.str_k_sz, *psv = P.p.str_v_sz;
+        if (retrieval) {
+          pk = P.p.ret_k;
+          pv = P.p.ret_v;
+          psk = P.p.ret_k_sz;
+          psv = P.p.ret_v_sz;
+          if (P.ret.table) {
+            int64_t blk = P.ret.table[(int64_t)b * P.ret.stride + (kb >> kPageShift)];
+            blk = blk < 0 ? 0 : (blk >= P.ret.blocks ? P.ret.blocks - 1 : blk);
+            row = ((blk * P.n_ret + pidx) << kPageShift) + (kb & (kPageTokens - 1));
+          } else {
+            row = ret_row(P.ret, b, pidx, kb);
+          }
+        }
+        prefetch_l2(pk + row * RB, (uint32_t)(rows * RB));
+        prefetch_l2(pv + row * RB, (uint32_t)(rows * RB));
         if (Q4) {  // 4-byte (scale, zero) rows; buffers hold a multiple of 4 rows
-          const uint32_t sz = (uint32_t)(((rows + 3) & ~3LL) * 4);
-          prefetch_l2(Ks + kb * 4, sz);
-          prefetch_l2(Vs + kb * 4, sz);
+          const uint32_t sz = (uint32_t)(((rows + 3) & ~3) * 4);
+          prefetch_l2(psk + row * 4, sz);
+          prefetch_l2(psv + row * 4, sz);
         }
       }
     }
@@ -188,16 +197,18 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // Fused append (bf16 cache): the token at position n-1 is not in the cache
-  // yet.  The CTA whose key range holds its row writes it there, skips that
-  // row in the main pass, and adds it in a one-key pass that reads the inputs.
+  // yet.  The warp whose tile holds its row writes it there, skips that row,
+  // and adds the key at the end from the inputs.
   const bool fused = !Q4 && P.knew != nullptr;
-  const int64_t newk = retrieval ? P.n - 1 : P.new_slot;  // its row in this head's buffer
+  const int newk = retrieval ? n - 1 : (int)ring_slot(n - 1, P.S, P.R);  // its key index in this head
   const bool owns_new = fused && !split_head && newk >= k0 && newk < k1;
   auto write_new = [&]() {  // one warp copies the new K and V rows into the cache
-    const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB;
+    const int64_t off = ((int64_t)r * P.Hkv + kvh) * (int64_t)RB;
     const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
     const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + off;
-    uint8_t *dst = const_cast<uint8_t *>(lane < 16 ? Kb : Vb) + newk * RB;
+    const int64_t row = retrieval ? ret_row(P.ret, b, pidx, newk) : srow0() + newk;
+    uint8_t *dst = const_cast<uint8_t *>(lane < 16 ? (retrieval ? P.p.ret_k : P.p.str_k)
+                                                   : (retrieval ? P.p.ret_v : P.p.str_v)) + row * RB;
     reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
   };
   if (owns_new && warp == 0) write_new();
@@ -208,7 +219,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const bool live = g < G;
   {
     const __nv_bfloat16 *qrow =
-        reinterpret_cast<const __nv_bfloat16 *>(P.q) + ((int64_t)b * P.Hq + (int64_t)kvh * G + g) * D;
+        reinterpret_cast<const __nv_bfloat16 *>(P.q) + ((int64_t)r * P.Hq + (int64_t)kvh * G + g) * D;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       int c0, c1, c2, c3;  // channels behind k-slots 2t, 2t+1, 2t+8, 2t+9
@@ -252,9 +263,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // 4-bit cache z = sum p*zp and cs = sum p*sc (as multiplied, see below)
   float m = -INFINITY, l = 0.f, z = 0.f, cs = 0.f;
 
-  // One warp, keys [kb0, kb0 + 16*KG) below hi of the buffers Kx/Vx (row
-  // index = key), except `skip_key`.
-  auto tile = [&](const uint8_t *Kx, const uint8_t *Vx, int64_t kb0, int64_t hi, int64_t skip_key) {
+  // One warp, keys [kb0, kb0 + 16*KG) below hi of the buffers Kx/Vx (and, for
+  // the 4-bit cache, the (scale, zero) rows Ksx/Vsx), row index = key, except
+  // `skip_key`.
+  auto tile = [&](const uint8_t *Kx, const uint8_t *Vx, const uint8_t *Ksx, const uint8_t *Vsx,
+                  int kb0, int hi, int skip_key) {
     // ------------------------------------------------------------ loads (all up front)
     // group kg covers keys kb = kb0 + 16*kg ..: K of key kb + 8*nt + g (this
     // thread's column of S); V of keys kb + {2t, 2t+1, 8+2t, 9+2t} (the k-slots
@@ -264,16 +277,16 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     uint4 vr[KG][4][Q4 ? 1 : 2];
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
-      const int64_t kb = kb0 + 16 * kg;
+      const int kb = kb0 + 16 * kg;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        const int64_t key = kb + 8 * nt + g;
+        const int key = kb + 8 * nt + g;
         const bool ok = key < hi && key != skip_key;
         if (Q4) {
-          kr[kg][nt][0] = ok ? ldg128(Kb + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
-          const int64_t key2 = kb + 8 * nt + 2 * t;
-          ksz[kg][nt] = key2 < hi ? ldg64(Ks + key2 * 4) : make_uint2(0, 0);
-          vsz[kg][nt] = key2 < hi ? ldg64(Vs + key2 * 4) : make_uint2(0, 0);
+          kr[kg][nt][0] = ok ? ldg128(Kx + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
+          const int key2 = kb + 8 * nt + 2 * t;
+          ksz[kg][nt] = key2 < hi ? ldg64(Ksx + key2 * 4) : make_uint2(0, 0);
+          vsz[kg][nt] = key2 < hi ? ldg64(Vsx + key2 * 4) : make_uint2(0, 0);
         } else {
 #pragma unroll
           for (int sp = 0; sp < 4; ++sp)
@@ -282,10 +295,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int64_t key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
+        const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
         const bool ok = key < hi && key != skip_key;
         if (Q4) {
-          const uint2 x = ok ? ldg64(Vb + key * RB + 8 * g) : make_uint2(0, 0);
+          const uint2 x = ok ? ldg64(Vx + key * RB + 8 * g) : make_uint2(0, 0);
           vr[kg][i][0] = make_uint4(x.x, x.y, 0, 0);
         } else {
 #pragma unroll
@@ -295,10 +308,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       }
     }
     // ------------------------------------------------------------ S = Q K^T
-    float sc[KG][2][2], vscale[KG][2][2], vzero[KG][2][2];
+    float sc[KG][2][2];
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
-      const int64_t kb = kb0 + 16 * kg;
+      const int kb = kb0 + 16 * kg;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         float s[4] = {0.f, 0.f, 0.f, 0.f};
@@ -317,20 +330,15 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
           }
         }
         // scores of query g at keys kb + 8*nt + 2t + e
-        const int64_t key = kb + 8 * nt + 2 * t;
+        const int key = kb + 8 * nt + 2 * t;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           float raw = s[e];
-          vscale[kg][nt][e] = 1.f;
-          vzero[kg][nt][e] = 0.f;
           if (Q4) {
             const __half2 kp = *reinterpret_cast<const __half2 *>(e ? &ksz[kg][nt].y : &ksz[kg][nt].x);
-            const __half2 vp = *reinterpret_cast<const __half2 *>(e ? &vsz[kg][nt].y : &vsz[kg][nt].x);
             // q.(128 + u) = q.u + 128*sum(q):  s = sc*q.u + zp*sum(q)
             const float ksc = __low2float(kp);
             raw = ksc * raw + (__high2float(kp) - 128.f * ksc) * qsum;
-            vscale[kg][nt][e] = __low2float(vp);
-            vzero[kg][nt][e] = __high2float(vp);
           }
           sc[kg][nt][e] = (live && key + e < hi && key + e != skip_key) ? raw * sl2 : -INFINITY;
         }
@@ -376,9 +384,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         for (int e = 0; e < 2; ++e) {
           p[nt][e] = (sc[kg][nt][e] == -INFINITY) ? 0.f : fast_exp2(sc[kg][nt][e] - m);
           l += p[nt][e];
-          if (Q4) {
-            z += p[nt][e] * vzero[kg][nt][e];
-            p[nt][e] *= vscale[kg][nt][e];
+          if (Q4) {  // the key's V (scale, zero), unpacked where used
+            const __half2 vp = *reinterpret_cast<const __half2 *>(e ? &vsz[kg][nt].y : &vsz[kg][nt].x);
+            z += p[nt][e] * __high2float(vp);
+            p[nt][e] *= __low2float(vp);
           }
         }
       // P^T fragment: b0 = keys 2t, 2t+1 (tile 0), b1 = keys 8+2t, 9+2t (tile 1)
@@ -435,44 +444,62 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       }
     }
   };
+  // A tile of keys [kb0, kb0 + T) below hi: retrieval keys through the block
+  // that holds them (indices local to the block), streaming keys in the slot
+  // buffer.
+  auto run_tile = [&](int kb0, int hi, int skip_key) {
+    int64_t row;
+    int base = 0;
+    const uint8_t *pk, *pv, *psk, *psv;
+    if (retrieval) {
+      base = kb0 & kBlockMask;
+      row = ret_row(P.ret, b, pidx, base);
+      pk = P.p.ret_k, pv = P.p.ret_v, psk = P.p.ret_k_sz, psv = P.p.ret_v_sz;
+    } else {
+      row = srow0();
+      pk = P.p.str_k, pv = P.p.str_v, psk = P.p.str_k_sz, psv = P.p.str_v_sz;
+    }
+    tile(pk + row * RB, pv + row * RB, Q4 ? psk + row * 4 : nullptr, Q4 ? psv + row * 4 : nullptr,
+         kb0 - base, hi - base, skip_key < 0 ? -1 : skip_key - base);
+  };
   bool new_here = owns_new && warp == 0;  // this warp adds the new token at the end
   if (split_head) {
     // The first pool claim is issued during the warp's last tile of its
     // share, so that its latency overlaps that tile.
-    const int64_t pool0 = pooled ? (int64_t)P.nsplit * ts : tiles;
-    unsigned *next = P.ws_next + ((int64_t)b * P.n_ret + pidx) * kChunkCounterStride;
-    auto visit = [&](int64_t tt) {
-      const int64_t kb0 = tt * T;
+    const int pool0 = pooled ? nsplit * ts : tiles;
+    unsigned *next = P.ws_next + ((int64_t)r * P.n_ret + pidx) * kChunkCounterStride;
+    auto visit = [&](int tt) {
+      const int kb0 = tt * T;
       const bool has_new = fused && newk >= kb0 && newk < kb0 + T;
       if (has_new) {
         write_new();
         new_here = true;
       }
-      tile(Kb, Vb, kb0, P.n, has_new ? newk : -1);
+      run_tile(kb0, n, has_new ? newk : -1);
     };
     unsigned c = 0;
-    int64_t tt = (int64_t)split * ts + warp;
+    int tt = split * ts + warp;
     if (pooled && tt >= t1 && lane == 0) c = atomicAdd(next, 1u);
     for (; tt < t1; tt += NWARPS) {
       if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
       visit(tt);
     }
     c = __shfl_sync(0xffffffffu, c, 0);
-    while (pool0 + (int64_t)c < tiles) {
+    while (pool0 + (int)c < tiles) {
       unsigned nx = 0;  // claim the following tile now; needed only after this one
       if (lane == 0) nx = atomicAdd(next, 1u);
-      visit(pool0 + c);
+      visit(pool0 + (int)c);
       c = __shfl_sync(0xffffffffu, nx, 0);
     }
   } else {
-    for (int64_t kb0 = k0 + (int64_t)warp * 16 * KG; kb0 < k1; kb0 += Keys<Q4>::STEP)
-      tile(Kb, Vb, kb0, k1, owns_new ? newk : -1);
+    for (int kb0 = k0 + warp * T; kb0 < k1; kb0 += Keys<Q4>::STEP)
+      run_tile(kb0, k1, owns_new ? newk : -1);
   }
   if (new_here) {
-    // the new token: buffers shifted so that row newk is the input row
-    const int64_t off = ((int64_t)b * P.Hkv + kvh) * (int64_t)RB - newk * RB;
+    // the new token, straight from the inputs (key 0 of a one-row buffer)
+    const int64_t off = ((int64_t)r * P.Hkv + kvh) * (int64_t)RB;
     tile(reinterpret_cast<const uint8_t *>(P.knew) + off, reinterpret_cast<const uint8_t *>(P.vnew) + off,
-         newk, newk + 1, -1);
+         nullptr, nullptr, 0, 1, -1);
   }
 
   // the next kernel in the stream may start its set-up now
@@ -512,7 +539,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     }
   }
   __syncthreads();
-  decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(P, smem, &s_last, retrieval, b, kvh, pidx, split);
+  decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(
+      P, smem, &s_last, nsplit == 1,
+      reinterpret_cast<__nv_bfloat16 *>(P.out) + ((int64_t)r * P.Hq + (int64_t)kvh * G) * D,
+      (int64_t)r * P.n_ret + pidx, (int64_t)(retrieval ? P.cta0[r] : 0) + (int64_t)pidx * nsplit,
+      nsplit, split);
 }
 
 template <bool Q4, int G>
@@ -537,7 +568,7 @@ cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
     cfg->num_sms = sms;
     return cudaSuccess;
   }
-  const int grid = d.B * d.n_ret * d.nsplit + d.B * d.n_str;
+  const int grid = d.cta0[d.rows.n] + d.rows.n * d.n_str;
   if (grid == 0) return cudaSuccess;
   if (!d.pdl) {
     kern<<<grid, NWARPS * 32, smem, s>>>(d);

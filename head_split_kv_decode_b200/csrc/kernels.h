@@ -14,6 +14,11 @@ constexpr int kMaxSplits = 512;
 // queue on one line)
 constexpr int kChunkCounterStride = 64;
 constexpr int kMaxDevices = 64;
+// Paged layout: retrieval tokens per block of the pool.
+constexpr int kPageShift = 8;
+constexpr int kPageTokens = 1 << kPageShift;
+// Batch rows one launch can take (row lists live in the kernel parameters).
+constexpr int kMaxLaunchRows = 128;
 
 enum KvType : int { kF32 = 0, kBF16 = 1, kINT4 = 2 };
 
@@ -39,37 +44,73 @@ struct HeadTables {
   int8_t str_heads[kMaxKvHeads]; // packed streaming index -> KV head
 };
 
+// The batch rows (sequence slots) a launch works on and each one's cache
+// length: before the new tokens (append), including the new token (decode),
+// or before the chunk (pre-fill).  A launch's inputs and outputs are indexed by
+// the position r in this list, the cache by row[r].
+struct LaunchRows {
+  int n;
+  int32_t row[kMaxLaunchRows];
+  int32_t len[kMaxLaunchRows];
+};
+
+// Where the retrieval rows of a layer live.  Packed: (b, head, key) is
+// storage row (b*n_ret + head)*cap + key.  Paged: key's block is
+// table[b*stride + key/kPageTokens] and the storage row is
+// (block*n_ret + head)*kPageTokens + key%kPageTokens.  Row r of a buffer is
+// at byte r*row_bytes; the int4 (scale, zero) arrays at byte r*4.
+struct RetMap {
+  const int32_t *table;  // device block table [B][stride]; null: packed layout
+  int stride;            // table entries per batch row
+  int n_ret;
+  int64_t cap;           // packed: rows per (b, head)
+  int64_t blocks;        // paged: blocks in the pool
+};
+
 struct AppendParams {
-  const void *k, *v;   // [B][n_tok][Hkv][D]
+  const void *k, *v;   // [rows.n][n_tok][Hkv][D]
   LayerPtrs p;
   HeadTables h;
-  int B, Hkv, D, n_ret, n_str, S, R, W;
+  RetMap ret;
+  LaunchRows rows;     // len = tokens in the cache before this append
+  int Hkv, D, n_ret, n_str, S, R, W;
   int Ws;              // rows per streaming head buffer (W, or W rounded up to 4 for int4)
-  int64_t cap, n_cur, n_tok;
+  int64_t n_tok;
 };
 
 struct DecodeParams {
-  const void *q;   // [B][Hq][D]
-  void *out;       // [B][Hq][D]
+  const void *q;   // [B][Hq][D] (tensor-core decode: [rows.n][Hq][D])
+  void *out;       // same shape as q
   LayerPtrs p;
   HeadTables h;
   int B, Hq, Hkv, G, D, n_ret, n_str, S, R, W;
   int Ws;              // rows per streaming head buffer
   int64_t cap;
+  // CUDA-core decode (packed layout, every row at length n): splits of
+  // split_len rows, nsplit per retrieval head.
   int64_t n;           // tokens in the cache, the query is at position n-1
   int nsplit;          // splits per retrieval head
   int64_t split_len;   // rows per split (multiple of the tile)
+  // Tensor-core decode: per launch row r (length rows.len[r], query at
+  // len-1), nsplit_r[r] splits per retrieval head; its retrieval CTAs are
+  // cta0[r] .. cta0[r+1]-1, head-major, and CTA c leaves its partial in
+  // slot c of ws_o / ws_lse.  Merge tickets and tile counters are indexed by
+  // r*n_ret + head.
+  LaunchRows rows;
+  int32_t cta0[kMaxLaunchRows + 1];
+  int16_t nsplit_r[kMaxLaunchRows];
+  RetMap ret;
   float scale_log2;    // softmax scale * log2(e)
-  float *ws_o;         // [B][n_ret][nsplit][G][D]
-  float *ws_lse;       // [B][n_ret][nsplit][G]
-  unsigned *ws_cnt;    // [B][n_ret] merge tickets
-  unsigned *ws_next;   // [B][n_ret][kChunkCounterStride] pool counter of each retrieval head (tensor-core decode)
+  float *ws_o;         // [partial slots][G][D]
+  float *ws_lse;       // [partial slots][G]
+  unsigned *ws_cnt;    // [units] merge tickets
+  unsigned *ws_next;   // [units][kChunkCounterStride] pool counter of each retrieval head (tensor-core decode)
   int *err;            // device error word
-  // Fused append (duo_decode_step): the K/V of the token at position n-1,
-  // [B][Hkv][D]; null when it is already in the cache.  The CTA that owns the
-  // token's row reads it from here and writes it to the cache.
+  // Fused append (duo_decode_step): the K/V of the token at position len-1 of
+  // each launch row, [rows.n][Hkv][D]; null when it is already in the cache.
+  // The warp whose key tile holds the token's row reads it from here and
+  // writes it to the cache.
   const void *knew, *vnew;
-  int64_t new_slot;    // streaming slot of position n-1
   int pdl;             // launched with programmatic dependent launch
   int pool;            // tensor-core decode: the last eighth of a split head's
                        // tiles is claimed at run time (0: every split gets an
@@ -77,14 +118,24 @@ struct DecodeParams {
 };
 
 struct PrefillParams {
-  const void *q, *k, *v;  // q [B][C][Hq][D], k/v [B][C][Hkv][D]
-  void *out;              // [B][C][Hq][D]
+  const void *q, *k, *v;  // q [rows.n][C][Hq][D], k/v [rows.n][C][Hkv][D]
+  void *out;              // [rows.n][C][Hq][D]
   LayerPtrs p;
   HeadTables h;
+  RetMap ret;
+  LaunchRows rows;        // len = tokens already in the cache (the chunk starts there)
   int B, Hq, Hkv, G, D, n_ret, n_str, S, R, W, C;
-  int64_t cap, c0;        // c0: tokens already in the cache
+  int64_t retrieval_rows; // storage rows of each retrieval buffer of the layer
   float scale_log2;
   int *err;
+};
+
+// Block-table writes of the paged layout, applied in stream order.
+constexpr int kMaxTableWrites = 256;
+struct TableWrites {
+  int n;
+  int32_t index[kMaxTableWrites];  // entry b*stride + i
+  int32_t block[kMaxTableWrites];
 };
 
 // Launch configuration facts the host needs to size splits and workspaces.
@@ -99,7 +150,12 @@ cudaError_t launch_append(const AppendParams &a, int kv_type, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &d, int kv_type, cudaStream_t s);
 // True when launch_decode can take the new token's K/V itself (fused append).
 bool decode_can_fuse_append(int kv_type, int D, int G);
+// True when the tensor-core decode serves this configuration: it alone reads
+// DecodeParams.rows (any launch rows, each at its own length) and the paged
+// layout; the CUDA-core decode takes every batch row at one length, packed.
+bool decode_mma_supported(int kv_type, int D, int G);
 cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s);
+cudaError_t launch_table_writes(int32_t *table, const TableWrites &w, cudaStream_t s);
 int *device_error_word();  // device address of the error word
 
 // Library-owned decode scratch for duo_decode_attn_static (decode_static.cu).

@@ -290,10 +290,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ret_q = P.n_ret * P.G, str_q = P.n_str * P.G;
   int blk = blockIdx.x;
   bool retrieval;
-  int b, hq, kvh, pidx, pair;
-  if (blk < P.B * ret_q * n_pairs) {
+  int b, hq, kvh, pidx, pair;  // b: launch row (indexes the inputs and outputs)
+  if (blk < P.rows.n * ret_q * n_pairs) {
     retrieval = true;
-    const int per = P.B * ret_q;
+    const int per = P.rows.n * ret_q;
     pair = n_pairs - 1 - blk / per;
     const int r = blk % per;
     b = r / ret_q;
@@ -303,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     hq = kvh * P.G + rr % P.G;
   } else {
     retrieval = false;
-    blk -= P.B * ret_q * n_pairs;
-    const int per = P.B * str_q;
+    blk -= P.rows.n * ret_q * n_pairs;
+    const int per = P.rows.n * str_q;
     pair = n_pairs - 1 - blk / per;
     const int r = blk % per;
     b = r / str_q;
@@ -313,9 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     kvh = P.h.str_heads[pidx];
     hq = kvh * P.G + rr % P.G;
   }
+  const int brow = P.rows.row[b];       // its batch row in the cache
+  const int64_t c0 = P.rows.len[b];     // tokens of that row already in the cache
   const int q0 = pair * 2 * BM;
   Sched sc;
-  sc.init(retrieval, P.c0, P.C, P.S, P.R, P.W, q0);
+  sc.init(retrieval, c0, P.C, P.S, P.R, P.W, q0);
   const int n_tiles = sc.count();
 
   // ---- set-up: barriers, tensor memory
@@ -352,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load3(base + kQB + BOX, &M.q, 64, hq, qz + BM, bar(Q_FULL));
       const CUtensorMap *pk = retrieval ? &M.kr : &M.ks;
       const CUtensorMap *pv = retrieval ? &M.vr : &M.vs;
-      const int pz = b * (retrieval ? P.n_ret : P.n_str) + pidx;
+      const int pz = brow * P.n_str + pidx;  // streaming slot buffer
       int issued_k = 0, issued_v = 0;
       auto issue = [&](int j, bool is_v) -> bool {
         const int st = j & 1;
@@ -365,9 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar((is_v ? V_FULL0 : K_FULL0) + st);
         mbar_arrive_expect_tx(fb, TILE);
         if (seg == 0) {
+          // retrieval: the storage row of the tile's first key (a tile of BN
+          // keys never crosses a block of the paged layout); streaming: slot
           const CUtensorMap *m = is_v ? pv : pk;
-          tma_load3(dst, m, 0, idx * BN, pz, fb);
-          tma_load3(dst + BOX, m, 64, idx * BN, pz, fb);
+          const int y = retrieval ? (int)ret_row(P.ret, brow, pidx, (int64_t)idx * BN) : idx * BN;
+          const int z = retrieval ? 0 : pz;
+          tma_load3(dst, m, 0, y, z, fb);
+          tma_load3(dst + BOX, m, 64, y, z, fb);
         } else {
           const CUtensorMap *m = is_v ? &M.vc : &M.kc;
           const int z = b * P.C + idx * BN;
@@ -470,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;                 // row of the query tile = TMEM lane
     const int crow = q0 + x * BM + row;             // chunk row
-    const int64_t ipos = P.c0 + crow;               // absolute query position
+    const int64_t ipos = c0 + crow;                 // absolute query position
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + (x ? 128u : 0u) + lane_off;
     const uint32_t tO = tmem + (x ? 384u : 256u) + lane_off;
@@ -503,19 +509,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (retrieval) {
             vis[ch] = range_bits(0, hi, first, ch);
           } else {
-            vis[ch] = range_bits(0, min(hi, (int64_t)P.S - P.c0), first, ch) |
+            vis[ch] = range_bits(0, min(hi, (int64_t)P.S - c0), first, ch) |
                       range_bits((int64_t)crow - P.R + 1, hi, first, ch);
           }
         }
       } else if (retrieval) {
         // page rows are positions; all below c0 are visible
 #pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) vis[ch] = range_bits(0, P.c0, first, ch);
+        for (int ch = 0; ch < BN / 32; ++ch) vis[ch] = range_bits(0, c0, first, ch);
       } else {
         // slot buffer: sinks, plus the ring slots of positions in
         // [max(S, ipos-R+1), c0) (a cyclic slot range)
         const int64_t filled = sc.filled;
-        const int64_t p_lo = max((int64_t)P.S, ipos - P.R + 1), p_hi = P.c0;  // [p_lo, p_hi)
+        const int64_t p_lo = max((int64_t)P.S, ipos - P.R + 1), p_hi = c0;  // [p_lo, p_hi)
         int64_t r1lo = 0, r1hi = 0, r2lo = 0, r2hi = 0;
         if (p_lo < p_hi) {
           const int64_t cnt = p_hi - p_lo;
@@ -687,14 +693,20 @@ cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s) {
   Maps maps;
   std::memset(&maps, 0, sizeof(maps));
   const uint64_t row = HD * 2;
-  const uint64_t BC = (uint64_t)p.B * p.C;
+  if (p.rows.n <= 0) return cudaSuccess;
+  const uint64_t BC = (uint64_t)p.rows.n * p.C;  // inputs and outputs: the launch rows
   bool ok = make_map(&maps.q, p.q, p.Hq, BC, row, row * p.Hq, 1, BM) &&
             make_map(&maps.kc, p.k, p.Hkv, BC, row, row * p.Hkv, 1, BN) &&
             make_map(&maps.vc, p.v, p.Hkv, BC, row, row * p.Hkv, 1, BN);
   // A kind with no heads in this layer keeps zeroed maps: no CTA reads them.
-  if (ok && p.n_ret > 0)
-    ok = make_map(&maps.kr, p.p.ret_k, p.cap, (uint64_t)p.B * p.n_ret, row, row * p.cap, BN, 1) &&
-         make_map(&maps.vr, p.p.ret_v, p.cap, (uint64_t)p.B * p.n_ret, row, row * p.cap, BN, 1);
+  // Retrieval buffers are addressed by storage row (packed or paged), so
+  // their maps are flat; TMA coordinates are 32-bit.
+  if (ok && p.n_ret > 0) {
+    if (p.retrieval_rows >= (1LL << 31)) return cudaErrorInvalidValue;
+    const uint64_t rr = (uint64_t)p.retrieval_rows;
+    ok = make_map(&maps.kr, p.p.ret_k, rr, 1, row, row * rr, BN, 1) &&
+         make_map(&maps.vr, p.p.ret_v, rr, 1, row, row * rr, BN, 1);
+  }
   if (ok && p.n_str > 0)
     ok = make_map(&maps.ks, p.p.str_k, p.W, (uint64_t)p.B * p.n_str, row, row * p.W, BN, 1) &&
          make_map(&maps.vs, p.p.str_v, p.W, (uint64_t)p.B * p.n_str, row, row * p.W, BN, 1);
@@ -712,7 +724,7 @@ cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s) {
     attr = true;
   }
   const int n_pairs = (p.C + 2 * BM - 1) / (2 * BM);
-  const int grid = p.B * (p.n_ret + p.n_str) * p.G * n_pairs;
+  const int grid = p.rows.n * (p.n_ret + p.n_str) * p.G * n_pairs;
   prefill_kernel<<<grid, kThreads, kSmemBytes, s>>>(p, maps);
   return cudaGetLastError();
 }

@@ -155,10 +155,19 @@ class Workload:
     outlier_frac: float = 0.0
     outlier_mult: float = 1.0
     batches: tuple = field(default=())
+    row_lengths: tuple = field(default=())  # per-row contexts of a mixed-length batch
 
     @property
     def group(self):
         return self.n_q_heads // self.n_kv_heads
+
+
+def mixed_lengths(seed, n, lo, hi):
+    """n seeded context lengths, log-uniform in [lo, hi]: the length mix of a
+    serving batch whose sequences arrived at different times."""
+    g = torch.Generator().manual_seed(seed)
+    u = torch.rand(n, generator=g, dtype=torch.float64)
+    return tuple(int(round(lo * (hi / lo) ** x)) for x in u.tolist())
 
 
 WORKLOADS = {
@@ -176,6 +185,10 @@ WORKLOADS = {
     "llama3_8b_gqa_prefill_32k": Workload(
         4, "Llama-3-8B-shaped GQA chunked pre-fill bf16: 32/8 heads, d128, 32768-token prompt in 4096-token chunks, 50% retrieval, S64+R256",
         "bf16", 32, 1, 32, 8, 128, 32768, 64, 256, 0.5, chunk=4096),
+    "llama3_8b_gqa_paged_mixed": Workload(
+        6, "Llama-3-8B-shaped GQA decode bf16, paged KV: 32 layers, 32/8 heads, d128, 8 sequences of 2K-64K tokens (log-uniform), 50% retrieval, S64+R256",
+        "bf16", 32, 8, 32, 8, 128, 65536, 64, 256, 0.5, steps=64,
+        row_lengths=mixed_lengths(6001, 8, 2048, 65536)),
     "llama3_8b_gqa_int4_1m": Workload(
         5, "Llama-3-8B-shaped GQA decode with INT4 KV: 32 layers, 32/8 heads, d128, ctx 1048576, 25% retrieval, S64+R256",
         "int4", 32, 1, 32, 8, 128, 1048576, 64, 256, 0.25, steps=64,

@@ -44,6 +44,11 @@
  *    duo_decode_attn; the new token sees itself).  Pre-fill is
  *    attend-then-append (duo_prefill_attn reads the cache as it stood before
  *    the chunk plus the chunk's own K/V; the caller then appends the chunk).
+ *  - Rows: each batch row is a sequence slot with its own length per layer.
+ *    The plain calls act on every row, each at its own length; the *_rows
+ *    calls act on a list of distinct rows, and their tensors hold only the
+ *    listed rows, in list order (the leading "batch" dimension becomes the
+ *    list length).
  */
 #ifndef DUO_H
 #define DUO_H
@@ -57,13 +62,15 @@ extern "C" {
 
 #define DUO_MAX_KV_HEADS 64
 #define DUO_MAX_SPLITS 512
+#define DUO_PAGE_TOKENS 256     /* tokens per retrieval block of the paged layout */
+#define DUO_MAX_LAUNCH_ROWS 128 /* rows per kernel launch; longer row lists take several */
 
 typedef struct CUstream_st *duo_stream; /* a cudaStream_t; NULL = legacy stream */
 
 typedef enum duo_status {
   DUO_OK = 0,
   DUO_ERR_ARG = 1,         /* null pointer, bad size, bad layer, misaligned pointer */
-  DUO_ERR_CAPACITY = 2,    /* an append would overflow a retrieval page */
+  DUO_ERR_CAPACITY = 2,    /* an append would pass capacity, or the block pool is exhausted */
   DUO_ERR_LAYOUT = 3,      /* head mask / head counts inconsistent */
   DUO_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
   DUO_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
@@ -77,7 +84,11 @@ typedef enum duo_kv_dtype { DUO_F32 = 0, DUO_BF16 = 1, DUO_INT4 = 2 } duo_kv_dty
 typedef enum duo_layout {
   /* Retrieval KV heads: one contiguous [capacity, d] page each for K and V.
    * Streaming KV heads: one [S + R, d] slot buffer each for K and V. */
-  DUO_LAYOUT_PACKED = 0
+  DUO_LAYOUT_PACKED = 0,
+  /* Retrieval KV heads: blocks of DUO_PAGE_TOKENS tokens from a pool shared
+   * by all rows, found through a per-row block table (duo_cache_create_paged).
+   * Streaming KV heads as in the packed layout. */
+  DUO_LAYOUT_PAGED = 1
 } duo_layout;
 
 typedef struct duo_cache_desc {
@@ -87,7 +98,7 @@ typedef struct duo_cache_desc {
   int32_t n_kv_heads;  /* <= DUO_MAX_KV_HEADS, divides n_q_heads */
   int32_t head_dim;    /* 64 or 128 */
   int32_t kv_dtype;    /* duo_kv_dtype */
-  int64_t capacity;    /* max tokens a retrieval page holds (INT4: rounded up to 4) */
+  int64_t capacity;    /* max tokens of one row (INT4: rounded up to 4) */
 } duo_cache_desc;
 
 typedef struct duo_cache duo_cache;
@@ -101,21 +112,43 @@ typedef struct duo_layout_view {
   int32_t window_stride; /* rows per streaming head buffer: window, rounded up to 4 for INT4 */
   int32_t row_bytes;     /* bytes of one token of one head: d*4 (f32), d*2 (bf16), d/2 (int4 codes) */
   int64_t capacity;
-  int64_t seq_len;       /* tokens appended so far */
-  int64_t ret_k, ret_v;  /* [batch][n_retrieval][capacity][row] */
+  int64_t seq_len;       /* the longest row's length */
+  int64_t ret_k, ret_v;  /* packed [batch][n_retrieval][capacity][row];
+                            paged  [pool_blocks][n_retrieval][DUO_PAGE_TOKENS][row] */
   int64_t str_k, str_v;  /* [batch][n_streaming][window_stride][row] */
   int64_t ret_k_sz, ret_v_sz, str_k_sz, str_v_sz; /* int4 only: fp16 (scale, zero) per token, same indexing */
   int32_t kind[DUO_MAX_KV_HEADS];         /* 1 retrieval, 0 streaming, per KV head */
   int32_t packed_index[DUO_MAX_KV_HEADS]; /* index among heads of the same kind */
+  int32_t layout;        /* duo_layout */
+  int32_t page_tokens;   /* paged: DUO_PAGE_TOKENS; packed: 0 */
+  int32_t table_stride;  /* paged: block-table entries per row */
+  int64_t pool_blocks;   /* paged: blocks in the pool */
+  int64_t block_table;   /* paged: int32 [batch][table_stride] (shared by all layers); else -1 */
 } duo_layout_view;
 
 /* Create a cache description.  head_mask: host array [layers][n_kv_heads] of
  * 0/1 (1 = retrieval).  S >= 0 sinks, R >= 1 recent slots.  layout must be
- * DUO_LAYOUT_PACKED.  No device memory is touched.
+ * DUO_LAYOUT_PACKED (use duo_cache_create_paged for the paged layout).  No
+ * device memory is touched.
  * Errors: DUO_ERR_ARG (null/out-of-range), DUO_ERR_LAYOUT (heads inconsistent). */
 duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc,
                             const uint8_t *head_mask, int32_t S, int32_t R,
                             int32_t layout);
+
+/* Create a cache with the paged layout, for serving many sequences of
+ * different lengths: retrieval K/V live in a pool of pool_blocks blocks of
+ * DUO_PAGE_TOKENS tokens (every layer holds its own pool of the same block
+ * count), which rows take as they grow and give back on duo_release_rows or
+ * duo_cache_reset; block ids are shared by all layers of a row.
+ * desc.capacity bounds one row's length.  The allocator runs on the host;
+ * new block-table entries are written on the stream before the kernels that
+ * need them.  Requires a configuration the tensor-core decode serves (bf16 or
+ * 4-bit KV, head_dim 128); pre-fill needs bf16.
+ * Errors: as duo_cache_create; DUO_ERR_ARG for pool_blocks <= 0;
+ * DUO_ERR_UNSUPPORTED for other configurations. */
+duo_status duo_cache_create_paged(duo_cache **out, const duo_cache_desc *desc,
+                                  const uint8_t *head_mask, int32_t S, int32_t R,
+                                  int64_t pool_blocks);
 
 void duo_cache_destroy(duo_cache *cache);
 
@@ -125,47 +158,84 @@ duo_status duo_cache_required_bytes(const duo_cache *cache, size_t *cache_bytes,
                                     size_t *workspace_bytes);
 
 /* Bind caller-owned device memory (256-byte aligned, >= cache_bytes).  The
- * memory is zero-filled synchronously and every layer's length reset to 0. */
+ * memory is zero-filled synchronously and every length reset to 0 (paged:
+ * every block returned to the pool). */
 duo_status duo_cache_bind(duo_cache *cache, void *device_mem, size_t bytes);
 
-/* Reset every layer's length to 0 without touching device memory. */
+/* Reset every row of every layer to length 0 (paged: return every block to
+ * the pool) without touching device memory. */
 duo_status duo_cache_reset(duo_cache *cache);
 
-/* Append n_tokens tokens (positions seq_len .. seq_len+n_tokens-1) of K and V
- * to one layer: retrieval heads write page rows, streaming heads write only the
- * positions that survive the chunk (sinks and the last R positions) into their
- * slots, evicting what was there.  INT4 caches quantise each (token, head) row
- * of head_dim channels (asymmetric min/max, fp16 scale and zero, 4-bit codes,
- * low nibble = even channel).  Advances the layer length by n_tokens.
- * Errors: DUO_ERR_CAPACITY if seq_len + n_tokens > capacity. */
+/* Rows n_rows listed in rows (distinct, in range) go back to length 0 in every
+ * layer; paged: their blocks return to the pool.  rows == NULL: every row.
+ * Host only. */
+duo_status duo_release_rows(duo_cache *cache, const int32_t *rows, int32_t n_rows);
+
+/* Append n_tokens tokens to one layer of every row (each row at its own
+ * positions len .. len+n_tokens-1): retrieval heads write page (or block)
+ * rows, streaming heads write only the positions that survive the chunk
+ * (sinks and the last R positions) into their slots, evicting what was
+ * there.  INT4 caches quantise each (token, head) row of head_dim channels
+ * (asymmetric min/max, fp16 scale and zero, 4-bit codes, low nibble = even
+ * channel).  Paged: rows take the blocks they need from the pool first.
+ * Advances each row's length by n_tokens.
+ * Errors: DUO_ERR_CAPACITY if a row would pass capacity or the pool cannot
+ * cover every row (nothing is changed then). */
 duo_status duo_append_kv(duo_cache *cache, int32_t layer, const void *k,
                          const void *v, int32_t n_tokens, duo_stream stream);
 
-/* Single-token decode attention for one layer: the query at position
- * seq_len-1 of every query head attends to its KV head's visible set.
- * Retrieval heads run split-K flash decoding (per-split log-sum-exp partials
- * in the workspace, merged by the last split of each head); streaming heads
- * run one pass over their slot buffer.  softmax_scale <= 0 means 1/sqrt(d).
- * The workspace must be zero-filled before its first use with any cache; each
- * call leaves its counters at zero again.  Workspace size: from
- * duo_cache_required_bytes.  Errors: DUO_ERR_STATE if the layer is empty. */
+/* duo_append_kv for the n_rows rows listed (k, v: [n_rows, n_tokens,
+ * n_kv_heads, head_dim]).  rows == NULL: every row.  Errors also DUO_ERR_ARG
+ * for a repeated or out-of-range row. */
+duo_status duo_append_kv_rows(duo_cache *cache, int32_t layer, const int32_t *rows,
+                              int32_t n_rows, const void *k, const void *v,
+                              int32_t n_tokens, duo_stream stream);
+
+/* Single-token decode attention for one layer: in every row, the query at
+ * position len-1 (len = that row's length) of every query head attends to its
+ * KV head's visible set.  Retrieval heads run split-K flash decoding
+ * (per-split log-sum-exp partials in the workspace, merged by the last split
+ * of each head; the tensor-core decode gives each row a split count in
+ * proportion to its length); streaming heads run one pass over their slot
+ * buffer.  softmax_scale <= 0 means 1/sqrt(d).  The workspace must be
+ * zero-filled before its first use with any cache; each call leaves its
+ * counters at zero again.  Workspace size: from duo_cache_required_bytes.
+ * Errors: DUO_ERR_STATE if a row is empty; DUO_ERR_UNSUPPORTED for rows of
+ * different lengths on a configuration without the tensor-core decode (fp32
+ * caches, head_dim 64). */
 duo_status duo_decode_attn(duo_cache *cache, int32_t layer, const void *q,
                            void *out, float softmax_scale, void *workspace,
                            size_t workspace_bytes, duo_stream stream);
 
+/* duo_decode_attn for the n_rows rows listed (q, out: [n_rows, n_q_heads,
+ * head_dim]).  Tensor-core decode configurations only (other configurations
+ * accept only rows == NULL). */
+duo_status duo_decode_attn_rows(duo_cache *cache, int32_t layer, const int32_t *rows,
+                                int32_t n_rows, const void *q, void *out,
+                                float softmax_scale, void *workspace,
+                                size_t workspace_bytes, duo_stream stream);
+
 /* One decode step for one layer in a single launch where the kernels allow
- * it: append the new token (k_new, v_new: [batch, n_kv_heads, head_dim]) at
- * position seq_len and attend with q at that position, exactly as
- * duo_append_kv(.., 1, ..) followed by duo_decode_attn.  The CTA that owns the
- * new token's row takes its K/V from the inputs and writes them to the cache.
- * Configurations without a fused kernel (fp32 caches, head_dim 64, 4-bit
- * caches) run the two calls.  Advances the layer length by one.  The launch
- * uses programmatic dependent launch, so its set-up overlaps the previous
- * kernel in the stream.  Errors as for the two calls. */
+ * it: append each row's new token (k_new, v_new: [batch, n_kv_heads,
+ * head_dim]) at position len and attend with q at that position, exactly as
+ * duo_append_kv(.., 1, ..) followed by duo_decode_attn.  The warp whose key
+ * tile holds the new token's row takes its K/V from the inputs and writes
+ * them to the cache.  Configurations without a fused kernel (fp32 caches,
+ * head_dim 64, 4-bit caches) run the two calls.  Advances each row's length
+ * by one.  The launch uses programmatic dependent launch, so its set-up
+ * overlaps the previous kernel in the stream.  Errors as for the two calls. */
 duo_status duo_decode_step(duo_cache *cache, int32_t layer, const void *q,
                            const void *k_new, const void *v_new, void *out,
                            float softmax_scale, void *workspace,
                            size_t workspace_bytes, duo_stream stream);
+
+/* duo_decode_step for the n_rows rows listed (q, out: [n_rows, n_q_heads,
+ * head_dim]; k_new, v_new: [n_rows, n_kv_heads, head_dim]). */
+duo_status duo_decode_step_rows(duo_cache *cache, int32_t layer, const int32_t *rows,
+                                int32_t n_rows, const void *q, const void *k_new,
+                                const void *v_new, void *out, float softmax_scale,
+                                void *workspace, size_t workspace_bytes,
+                                duo_stream stream);
 
 /* Decode attention like duo_decode_attn, but with no workspace argument and
  * no allocation of any kind: the split-K scratch (partial outputs, log-sum-exp
@@ -183,33 +253,58 @@ duo_status duo_decode_step(duo_cache *cache, int32_t layer, const void *q,
  *  - Every call shares the one array: calls that may overlap on the GPU (other
  *    streams, other threads, other caches) race and must be serialised by the
  *    caller.  The merge tickets are cleared on the stream before each launch.
- *  - If the scratch this layer needs (batch x retrieval heads x splits x
- *    group x (head_dim + 1) x 4 bytes, plus tickets) exceeds the array, the
- *    call returns DUO_ERR_WORKSPACE before enqueuing anything.
- * Results equal duo_decode_attn's for the same cache state. */
+ *  - If the scratch this layer needs (the retrieval splits of all rows x
+ *    group x (head_dim + 1) x 4 bytes, plus tickets and counters) exceeds the
+ *    array, the call returns DUO_ERR_WORKSPACE before enqueuing anything.
+ * Results equal duo_decode_attn's for the same cache state (bit for bit with
+ * duo_set_decode_reproducible, else up to rounding). */
 #define DUO_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
 duo_status duo_decode_attn_static(duo_cache *cache, int32_t layer, const void *q,
                                   void *out, float softmax_scale, duo_stream stream);
 
-/* Chunked pre-fill attention for one layer: C queries at positions
- * seq_len .. seq_len+C-1 attend to the cache as it stands (positions below
- * seq_len) plus the chunk's own k/v: causal for retrieval heads, Lambda mask
+/* Chunked pre-fill attention for one layer: in every row, C queries at
+ * positions len .. len+C-1 attend to the cache as it stands (positions below
+ * len) plus the chunk's own k/v: causal for retrieval heads, Lambda mask
  * (sinks plus the R most recent positions) for streaming heads, with key tiles
  * outside the Lambda band skipped.  Runs on the sm_100a tensor cores
  * (tcgen05.mma, accumulators in tensor memory, operands loaded by TMA).  Does
  * not append; call duo_append_kv with the same k/v afterwards.  Requires a
  * DUO_BF16 cache with head_dim 128 (other cases: DUO_ERR_UNSUPPORTED).  The
- * workspace argument is unused (pass NULL, 0). */
+ * workspace argument is unused (pass NULL, 0).
+ * Errors: DUO_ERR_CAPACITY if len + C would pass capacity in a row. */
 duo_status duo_prefill_attn(duo_cache *cache, int32_t layer, const void *q,
                             const void *k, const void *v, int32_t C, void *out,
                             float softmax_scale, void *workspace,
                             size_t workspace_bytes, duo_stream stream);
 
+/* duo_prefill_attn for the n_rows rows listed (q, out: [n_rows, C, n_q_heads,
+ * head_dim]; k, v: [n_rows, C, n_kv_heads, head_dim]), each at its own length. */
+duo_status duo_prefill_attn_rows(duo_cache *cache, int32_t layer, const int32_t *rows,
+                                 int32_t n_rows, const void *q, const void *k,
+                                 const void *v, int32_t C, void *out,
+                                 float softmax_scale, duo_stream stream);
+
+/* The longest row's length in one layer (every row's, when all rows advance
+ * together). */
 duo_status duo_seq_len(const duo_cache *cache, int32_t layer, int64_t *n);
 
+/* One row's length in one layer. */
+duo_status duo_row_seq_len(const duo_cache *cache, int32_t layer, int32_t row, int64_t *n);
+
+/* Paged layout: the blocks row holds, in logical order (block i holds
+ * positions [DUO_PAGE_TOKENS i, DUO_PAGE_TOKENS (i+1)) of the row in every
+ * layer).  *n_blocks receives the count; blocks (may be NULL) receives the
+ * ids if max_blocks is large enough (else DUO_ERR_ARG).  Packed: 0 blocks. */
+duo_status duo_row_blocks(const duo_cache *cache, int32_t row, int32_t *blocks,
+                          int32_t max_blocks, int32_t *n_blocks);
+
+/* Paged layout: blocks in the pool that no row holds.  Packed: 0. */
+duo_status duo_pool_free_blocks(const duo_cache *cache, int64_t *free_blocks);
+
 /* KV bytes held now (kept) and what a full cache of every head would hold
- * (full_equivalent): kept = sum over layers, batch, KV heads of
- * (retrieval ? n : min(n, S+R)) * bytes_per_token_per_head. */
+ * (full_equivalent): kept = sum over layers, rows, KV heads of
+ * (retrieval ? n : min(n, S+R)) * bytes_per_token_per_head, n = the row's
+ * length in that layer. */
 duo_status duo_kv_bytes(const duo_cache *cache, int64_t *kept,
                         int64_t *full_equivalent);
 
@@ -234,7 +329,8 @@ duo_status duo_set_decode_splits(duo_cache *cache, int32_t splits);
  * cache or on outside {0, 1}. */
 duo_status duo_set_decode_reproducible(duo_cache *cache, int32_t on);
 
-/* Split count the next decode of this layer will use. */
+/* Split count the next decode of this layer will use (tensor-core decode: the
+ * largest any row gets at the current lengths). */
 duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
                              int32_t *splits);
 
