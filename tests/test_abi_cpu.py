@@ -133,3 +133,74 @@ def test_status_strings(lib):
     for s in range(9):
         assert B.duo_status_string(s)
     assert "unknown" in B.duo_status_string(99)
+
+
+def _create_paged(pool_blocks=10, **kw):
+    args = dict(layers=2, batch=3, n_q_heads=8, n_kv_heads=4, head_dim=128, kv_dtype="bf16",
+                capacity=1000, head_mask=[1, 0, 0, 1, 0, 1, 0, 0], S=4, R=60,
+                pool_blocks=pool_blocks)
+    args.update(kw)
+    return B.duo_cache_create_paged(**args)
+
+
+def test_paged_layout_plan(lib):
+    """Pool buffers [blocks][n_ret][256][row] per layer, then one block table
+    [batch][ceil(capacity/256)] of int32; every byte accounted for."""
+    h = _create_paged()
+    try:
+        cb, _ = B.duo_cache_required_bytes(h)
+        v0, v1 = B.duo_layout_info(h, 0), B.duo_layout_info(h, 1)
+        assert v0.layout == B.DUO_LAYOUT_PAGED and v0.page_tokens == B.PAGE_TOKENS == 256
+        assert v0.pool_blocks == 10 and v0.table_stride == 4  # ceil(1000 / 256)
+        assert (v0.n_retrieval, v1.n_retrieval) == (2, 1)
+        pool0 = 10 * 2 * 256 * 256
+        assert v0.ret_k == 0 and v0.ret_v == pool0
+        assert v0.str_k == 2 * pool0 and v0.str_v == v0.str_k + 3 * 2 * 64 * 256
+        pool1 = 10 * 1 * 256 * 256
+        assert v1.ret_v - v1.ret_k == pool1
+        assert v0.block_table == v1.str_v + 3 * 3 * 64 * 256
+        assert cb == v0.block_table + 3 * 4 * 4 + (-(3 * 4 * 4) % 256)
+        assert B.duo_pool_free_blocks(h) == 10
+        assert B.duo_row_blocks(h, 0) == []
+        assert B.duo_row_seq_len(h, 1, 2) == 0
+        B.duo_release_rows(h, [2, 0])
+        B.duo_release_rows(h)
+        for rows in ([3], [1, 1], [-1]):
+            with pytest.raises(B.DuoError) as e:
+                B.duo_release_rows(h, rows)
+            assert e.value.name == "DUO_ERR_ARG"
+        # row calls before bind fail before touching anything
+        with pytest.raises(B.DuoError) as e:
+            B.duo_append_kv_rows(h, 0, [1], 16, 16, 1)
+        assert e.value.name == "DUO_ERR_STATE"
+        packed = _create()
+        try:
+            vp = B.duo_layout_info(packed, 0)
+            assert vp.layout == B.DUO_LAYOUT_PACKED and vp.page_tokens == 0
+            assert vp.block_table == -1 and B.duo_pool_free_blocks(packed) == 0
+        finally:
+            B.duo_cache_destroy(packed)
+    finally:
+        B.duo_cache_destroy(h)
+
+
+def test_paged_create_rejects(lib):
+    with pytest.raises(B.DuoError) as e:
+        _create_paged(pool_blocks=0)
+    assert e.value.name == "DUO_ERR_ARG"
+    for kw in (dict(kv_dtype="f32"), dict(head_dim=64)):
+        with pytest.raises(B.DuoError) as e:  # no tensor-core decode for these
+            _create_paged(**kw)
+        assert e.value.name == "DUO_ERR_UNSUPPORTED"
+    with pytest.raises(B.DuoError) as e:  # the paged layout has its own create call
+        _create(layout=B.DUO_LAYOUT_PAGED)
+    assert e.value.name == "DUO_ERR_ARG"
+    h = _create_paged(kv_dtype="int4")
+    try:
+        v = B.duo_layout_info(h, 0)
+        pool = 10 * 2 * 256  # rows of each retrieval buffer
+        assert v.ret_v == pool * 64 and v.str_k == 2 * pool * 64
+        assert v.ret_k_sz == v.str_v + 3 * 2 * 64 * 64  # after the streaming codes
+        assert v.ret_v_sz - v.ret_k_sz == pool * 4
+    finally:
+        B.duo_cache_destroy(h)
