@@ -485,13 +485,18 @@ def prefill_exact_flops(w, C, c0, retrieval):
     return 4 * w.head_dim * total
 
 
-def run_prefill(args, w, rank, world, peaks):
+def run_prefill(args, w, rank, world, peaks, kv_dtype="bf16"):
+    """One layer's prompt in chunks: attend, then append.  kv_dtype "int4"
+    keeps the history in a 4-bit cache; each timed call then also expands the
+    history it reads to bf16 (the launch before the tensor-core pass)."""
     from head_split_kv_decode_b200.cache import DuoCache
 
     mask = synth.workload_mask(w)[:1]
     C = w.chunk
     n_chunks = w.context // C
-    cache = DuoCache(1, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, "bf16", w.context, mask, w.S, w.R)
+    cache = DuoCache(1, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, kv_dtype, w.context, mask, w.S,
+                     w.R)
+    pws, pwsb = cache._prefill_ws()
     dt = torch.bfloat16
     b_ids = [rank]
     pos = range(w.context)
@@ -511,7 +516,7 @@ def run_prefill(args, w, rank, world, peaks):
             if events is not None:
                 events[c][0].record(stream)
             st = lib.duo_prefill_attn(cache.handle, 0, q.data_ptr(), k.data_ptr(), v.data_ptr(), C,
-                                      out.data_ptr(), 0.0, None, 0, sh)
+                                      out.data_ptr(), 0.0, pws, pwsb, sh)
             if st:
                 raise B.DuoError(st, "duo_prefill_attn")
             if events is not None:
@@ -545,8 +550,11 @@ def run_prefill(args, w, rank, world, peaks):
             exact_fl += G * prefill_exact_flops(w, C, c * C, ret)
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     tflops = tile_fl / (attn_ms * 1e-3) / 1e12
+    del cache
+    torch.cuda.empty_cache()
     return {
         "metric": "prefill attn TFLOP/s (tile-counted, 128x128 tiles)",
+        "kv_dtype": kv_dtype,
         "value": tflops,
         "unit": "TFLOP/s",
         "exact_tflops": exact_fl / (attn_ms * 1e-3) / 1e12,
@@ -558,7 +566,7 @@ def run_prefill(args, w, rank, world, peaks):
         "exact_flops_per_layer": exact_fl,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "traffic": None},
-        "gpu_launches": reps * n_chunks * 2,
+        "gpu_launches": reps * n_chunks * (3 if kv_dtype == "int4" else 2),
     }
 
 
@@ -708,6 +716,11 @@ def main(argv=None):
                           "decode_splits": rx["splits"], "gpu_launches": rx["gpu_launches"]}
         extra["llama3_8b_gqa_paged_mixed"] = run_paged_mixed(
             args, synth.WORKLOADS["llama3_8b_gqa_paged_mixed"], rank, world, peaks)
+        pq = run_prefill(args, synth.WORKLOADS["llama3_8b_gqa_prefill_32k"], rank, world, peaks,
+                         kv_dtype="int4")
+        extra["prefill_int4_cache"] = {k: pq[k] for k in ("value", "unit", "exact_tflops",
+                                                            "ms_per_layer", "kv_dtype")}
+        extra["prefill_int4_cache"]["frac"] = pq["roofline"]["frac"]
     prefill = None
     if not args.no_prefill:
         try:

@@ -87,7 +87,8 @@ SIGNATURES = {
     "duo_decode_step_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _P, _P, _F, _P, _SZ, _P]),
     "duo_decode_attn_static": (_I32, [_P, _I32, _P, _P, _F, _P]),
     "duo_prefill_attn": (_I32, [_P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
-    "duo_prefill_attn_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _F, _P]),
+    "duo_prefill_attn_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
+    "duo_prefill_workspace_bytes": (_I32, [_P, ctypes.POINTER(_SZ)]),
     "duo_seq_len": (_I32, [_P, _I32, ctypes.POINTER(_I64)]),
     "duo_row_seq_len": (_I32, [_P, _I32, _I32, ctypes.POINTER(_I64)]),
     "duo_row_blocks": (_I32, [_P, _I32, _P, _I32, ctypes.POINTER(_I32)]),
@@ -196,10 +197,17 @@ def duo_decode_step_rows(handle, layer, rows, q_ptr, k_new_ptr, v_new_ptr, out_p
 
 
 def duo_prefill_attn_rows(handle, layer, rows, q_ptr, k_ptr, v_ptr, C, out_ptr, softmax_scale,
-                          stream=0):
+                          ws_ptr=None, ws_bytes=0, stream=0):
     arr, n = _rows(rows)
     _check(lib().duo_prefill_attn_rows(handle, layer, arr, n, q_ptr, k_ptr, v_ptr, C, out_ptr,
-                                       softmax_scale, stream), "duo_prefill_attn_rows")
+                                       softmax_scale, ws_ptr, ws_bytes, stream),
+           "duo_prefill_attn_rows")
+
+
+def duo_prefill_workspace_bytes(handle):
+    n = _SZ()
+    _check(lib().duo_prefill_workspace_bytes(handle, ctypes.byref(n)), "duo_prefill_workspace_bytes")
+    return n.value
 
 
 def duo_row_seq_len(handle, layer, row):

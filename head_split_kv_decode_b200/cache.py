@@ -61,6 +61,17 @@ class DuoCache:
         B.duo_cache_bind(self.handle, self.base_ptr, self.cache_bytes)
         self._ws, woff = _aligned_buffer(self.ws_bytes, self.device, zero=True)
         self.ws_ptr = self._ws.data_ptr() + woff
+        self.prefill_ws_bytes = B.duo_prefill_workspace_bytes(self.handle)
+        self._pf_ws, self.pf_ws_ptr = None, None
+
+    def _prefill_ws(self):
+        """Pre-fill scratch (4-bit caches only), allocated on first use."""
+        if self.prefill_ws_bytes == 0:
+            return None, 0
+        if self._pf_ws is None:
+            self._pf_ws, off = _aligned_buffer(self.prefill_ws_bytes, self.device, zero=True)
+            self.pf_ws_ptr = self._pf_ws.data_ptr() + off
+        return self.pf_ws_ptr, self.prefill_ws_bytes
 
     # ------------------------------------------------------------ checks
     def _check(self, t, shape, name, dtype=None):
@@ -121,8 +132,9 @@ class DuoCache:
         if out is None:
             out = torch.empty_like(q)
         self._check(out, tuple(q.shape), "out")
+        ws, wsb = self._prefill_ws()
         B.duo_prefill_attn(self.handle, layer, q.data_ptr(), k.data_ptr(), v.data_ptr(), C,
-                           out.data_ptr(), float(scale), None, 0,
+                           out.data_ptr(), float(scale), ws, wsb,
                            _stream_handle(stream, self.device))
         return out
 
@@ -181,8 +193,10 @@ class DuoCache:
         if out is None:
             out = torch.empty_like(q)
         self._check(out, tuple(q.shape), "out")
+        ws, wsb = self._prefill_ws()
         B.duo_prefill_attn_rows(self.handle, layer, rows, q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                C, out.data_ptr(), float(scale), _stream_handle(stream, self.device))
+                                C, out.data_ptr(), float(scale), ws, wsb,
+                                _stream_handle(stream, self.device))
         return out
 
     def release_rows(self, rows=None):

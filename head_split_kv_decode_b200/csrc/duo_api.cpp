@@ -623,19 +623,81 @@ duo_status step_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &ro
 
 // ---------------------------------------------------------------- pre-fill
 
+// Pre-fill scratch of a 4-bit cache: the bf16 expansion of one layer's
+// history, [retrieval K][retrieval V] at the layer's storage rows and
+// [streaming K][streaming V] as [batch][n_str][S+R][d]; the largest layer.
+struct PrefillScratch {
+  int64_t ret_v, str_k, str_v, total;
+};
+
+PrefillScratch prefill_scratch(const duo_cache *c, int layer) {
+  const int64_t row = (int64_t)c->desc.head_dim * 2;
+  const auto &L = c->layers[layer];
+  PrefillScratch ps;
+  const int64_t ret = round_up(L.ret_rows * row, kAlign);
+  const int64_t str = round_up((int64_t)c->desc.batch * L.n_str * c->W * row, kAlign);
+  ps.ret_v = ret;
+  ps.str_k = 2 * ret;
+  ps.str_v = 2 * ret + str;
+  ps.total = 2 * ret + 2 * str;
+  return ps;
+}
+
+size_t prefill_ws_bytes(const duo_cache *c) {
+  if (c->desc.kv_dtype != DUO_INT4) return 0;
+  int64_t m = 0;
+  for (int l = 0; l < c->desc.layers; ++l) m = std::max(m, prefill_scratch(c, l).total);
+  return (size_t)m;
+}
+
 duo_status prefill_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &rows,
                         const void *q, const void *k, const void *v, int32_t C, void *out,
-                        float scale, cudaStream_t s) {
+                        float scale, void *ws, size_t ws_bytes, cudaStream_t s) {
   if (!q || !k || !v || !out || C <= 0) return DUO_ERR_ARG;
   if (!std::isfinite(scale)) return DUO_ERR_ARG;
   const duo_cache_desc &d = c->desc;
-  if (d.kv_dtype != DUO_BF16 || d.head_dim != 128) return DUO_ERR_UNSUPPORTED;
+  if ((d.kv_dtype != DUO_BF16 && d.kv_dtype != DUO_INT4) || d.head_dim != 128)
+    return DUO_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DUO_ERR_ARG;
   const auto &L = c->layers[layer];
   duo_status st = check_room(c, layer, rows, C);
   if (st != DUO_OK) return st;
+  const bool q4 = d.kv_dtype == DUO_INT4;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  if (q4) {
+    if (!ws || ws_bytes < prefill_ws_bytes(c)) return DUO_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return DUO_ERR_ARG;
+  }
   duo::PrefillParams p{};
   p.p = layer_ptrs(c, layer);
+  duo::DequantParams dq{};
+  if (q4) {
+    // the kernel reads the bf16 expansion of the history instead of the codes
+    const PrefillScratch ps = prefill_scratch(c, layer);
+    dq.p = p.p;
+    dq.h = L.h;
+    dq.ret = ret_map(c, layer);
+    dq.n_ret = L.n_ret;
+    dq.n_str = L.n_str;
+    dq.S = c->S;
+    dq.R = c->R;
+    dq.W = c->W;
+    dq.Ws = c->Ws;
+    dq.D = d.head_dim;
+    dq.ret_k = reinterpret_cast<__nv_bfloat16 *>(wsb);
+    dq.ret_v = reinterpret_cast<__nv_bfloat16 *>(wsb + ps.ret_v);
+    dq.str_k = reinterpret_cast<__nv_bfloat16 *>(wsb + ps.str_k);
+    dq.str_v = reinterpret_cast<__nv_bfloat16 *>(wsb + ps.str_v);
+    p.p = duo::LayerPtrs{};
+    if (L.n_ret) {
+      p.p.ret_k = wsb;
+      p.p.ret_v = wsb + ps.ret_v;
+    }
+    if (L.n_str) {
+      p.p.str_k = wsb + ps.str_k;
+      p.p.str_v = wsb + ps.str_v;
+    }
+  }
   p.h = L.h;
   p.ret = ret_map(c, layer);
   p.B = d.batch;
@@ -666,6 +728,10 @@ duo_status prefill_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> 
     p.k = static_cast<const uint8_t *>(k) + (int64_t)g0 * kv_row;
     p.v = static_cast<const uint8_t *>(v) + (int64_t)g0 * kv_row;
     p.out = static_cast<uint8_t *>(out) + (int64_t)g0 * q_row;
+    if (q4) {
+      dq.rows = p.rows;
+      if ((st = cuda_status(duo::launch_dequant_history(dq, s))) != DUO_OK) return st;
+    }
     if ((st = launch_status(duo::launch_prefill(p, s))) != DUO_OK) return st;
   }
   return DUO_OK;
@@ -793,19 +859,23 @@ duo_status duo_decode_attn_static(duo_cache *c, int32_t layer, const void *q, vo
 duo_status duo_prefill_attn(duo_cache *c, int32_t layer, const void *q, const void *k,
                             const void *v, int32_t C, void *out, float scale, void *ws,
                             size_t ws_bytes, duo_stream stream) {
-  (void)ws;
-  (void)ws_bytes;
-  return duo_prefill_attn_rows(c, layer, nullptr, 0, q, k, v, C, out, scale, stream);
+  return duo_prefill_attn_rows(c, layer, nullptr, 0, q, k, v, C, out, scale, ws, ws_bytes, stream);
 }
 
 duo_status duo_prefill_attn_rows(duo_cache *c, int32_t layer, const int32_t *rows, int32_t n_rows,
                                  const void *q, const void *k, const void *v, int32_t C, void *out,
-                                 float scale, duo_stream stream) {
+                                 float scale, void *ws, size_t ws_bytes, duo_stream stream) {
   duo_status st = check_layer(c, layer);
   if (st != DUO_OK) return st;
   std::vector<int32_t> list;
   if ((st = make_rows(c, rows, n_rows, &list)) != DUO_OK) return st;
-  return prefill_rows(c, layer, list, q, k, v, C, out, scale, (cudaStream_t)stream);
+  return prefill_rows(c, layer, list, q, k, v, C, out, scale, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+duo_status duo_prefill_workspace_bytes(const duo_cache *c, size_t *bytes) {
+  if (!c || !bytes) return DUO_ERR_ARG;
+  *bytes = prefill_ws_bytes(c);
+  return DUO_OK;
 }
 
 duo_status duo_release_rows(duo_cache *c, const int32_t *rows, int32_t n_rows) {

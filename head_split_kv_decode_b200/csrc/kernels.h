@@ -2,6 +2,7 @@
 // kernels.  Not part of the public ABI.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -130,6 +131,17 @@ struct PrefillParams {
   int *err;
 };
 
+// 4-bit history expanded to bf16 for the pre-fill: retrieval rows keep their
+// storage row; streaming rows go to [B][n_str][W][D] (slot order).
+struct DequantParams {
+  LayerPtrs p;         // the 4-bit cache buffers of the layer
+  HeadTables h;
+  RetMap ret;
+  LaunchRows rows;     // len = tokens of each row to expand (its history)
+  int n_ret, n_str, S, R, W, Ws, D;
+  __nv_bfloat16 *ret_k, *ret_v, *str_k, *str_v;  // bf16 scratch
+};
+
 // Block-table writes of the paged layout, applied in stream order.
 constexpr int kMaxTableWrites = 256;
 struct TableWrites {
@@ -156,6 +168,7 @@ bool decode_can_fuse_append(int kv_type, int D, int G);
 bool decode_mma_supported(int kv_type, int D, int G);
 cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s);
 cudaError_t launch_table_writes(int32_t *table, const TableWrites &w, cudaStream_t s);
+cudaError_t launch_dequant_history(const DequantParams &d, cudaStream_t s);
 int *device_error_word();  // device address of the error word
 
 // Library-owned decode scratch for duo_decode_attn_static (decode_static.cu).

@@ -268,10 +268,19 @@ duo_status duo_decode_attn_static(duo_cache *cache, int32_t layer, const void *q
  * (sinks plus the R most recent positions) for streaming heads, with key tiles
  * outside the Lambda band skipped.  Runs on the sm_100a tensor cores
  * (tcgen05.mma, accumulators in tensor memory, operands loaded by TMA).  Does
- * not append; call duo_append_kv with the same k/v afterwards.  Requires a
- * DUO_BF16 cache with head_dim 128 (other cases: DUO_ERR_UNSUPPORTED).  The
- * workspace argument is unused (pass NULL, 0).
- * Errors: DUO_ERR_CAPACITY if len + C would pass capacity in a row. */
+ * not append; call duo_append_kv with the same k/v afterwards.  Requires
+ * head_dim 128 and a DUO_BF16 or DUO_INT4 cache (other cases:
+ * DUO_ERR_UNSUPPORTED).  DUO_BF16: the workspace is unused (pass NULL, 0).
+ * DUO_INT4: the part of the cache the chunk reads (retrieval keys below each
+ * row's length, filled streaming slots) is first expanded to bf16, x = sc*u+zp
+ * rounded to bf16, in the workspace (duo_prefill_workspace_bytes, 256-byte
+ * aligned), which the tensor-core pass then reads; the chunk's own k/v enter
+ * exactly as given.  The workspace must be zero-filled before its first use:
+ * key tiles are 128 rows, so a tile can cover rows past a row's length whose
+ * probabilities are 0, and those rows must hold finite values (zeros or an
+ * earlier call's expansion) for 0 * value to stay 0.
+ * Errors: DUO_ERR_CAPACITY if len + C would pass capacity in a row;
+ * DUO_ERR_WORKSPACE if an INT4 cache gets a missing or small workspace. */
 duo_status duo_prefill_attn(duo_cache *cache, int32_t layer, const void *q,
                             const void *k, const void *v, int32_t C, void *out,
                             float softmax_scale, void *workspace,
@@ -282,7 +291,13 @@ duo_status duo_prefill_attn(duo_cache *cache, int32_t layer, const void *q,
 duo_status duo_prefill_attn_rows(duo_cache *cache, int32_t layer, const int32_t *rows,
                                  int32_t n_rows, const void *q, const void *k,
                                  const void *v, int32_t C, void *out,
-                                 float softmax_scale, duo_stream stream);
+                                 float softmax_scale, void *workspace,
+                                 size_t workspace_bytes, duo_stream stream);
+
+/* Workspace bytes duo_prefill_attn needs: 0 for a DUO_BF16 cache; for a
+ * DUO_INT4 cache the bf16 size of one layer's retrieval storage rows plus its
+ * streaming buffers (K and V), for the largest layer. */
+duo_status duo_prefill_workspace_bytes(const duo_cache *cache, size_t *bytes);
 
 /* The longest row's length in one layer (every row's, when all rows advance
  * together). */

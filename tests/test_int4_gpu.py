@@ -103,8 +103,9 @@ def test_int4_split_counts_agree():
         assert_parity(cache.decode(0, q), ref, "int4", "splits=%d" % splits)
 
 
-def test_int4_constant_rows_and_prefill_unsupported():
-    """A (token, head) row of identical values has scale 0: codes 0, x_hat = zp."""
+def test_int4_constant_rows_and_prefill_limits():
+    """A (token, head) row of identical values has scale 0: codes 0, x_hat = zp.
+    Pre-fill on a 4-bit cache needs room for the chunk and head_dim 128."""
     from head_split_kv_decode_b200.binding import DuoError
     B, Hq, Hkv, D, n = 1, 2, 2, 128, 40
     K = torch.full((B, n, Hkv, D), 0.75, dtype=BF, device="cuda")
@@ -118,8 +119,14 @@ def test_int4_constant_rows_and_prefill_unsupported():
     assert (Kh == 0.75).all()
     ref = OA.decode_reference(f64(q), Kh, _dequant_history(V)[0], mask.numpy(), 2, 8)
     assert_parity(out, ref, "int4", "constant rows")
-    with pytest.raises(DuoError) as e:
+    with pytest.raises(DuoError) as e:  # the cache is full
         cache.prefill(0, torch.zeros(B, 8, Hq, D, dtype=BF, device="cuda"),
                       torch.zeros(B, 8, Hkv, D, dtype=BF, device="cuda"),
                       torch.zeros(B, 8, Hkv, D, dtype=BF, device="cuda"))
+    assert e.value.name == "DUO_ERR_CAPACITY"
+    c64 = DuoCache(1, B, Hq, Hkv, 64, "int4", 64, mask[None], 2, 8)
+    with pytest.raises(DuoError) as e:
+        c64.prefill(0, torch.zeros(B, 8, Hq, 64, dtype=BF, device="cuda"),
+                    torch.zeros(B, 8, Hkv, 64, dtype=BF, device="cuda"),
+                    torch.zeros(B, 8, Hkv, 64, dtype=BF, device="cuda"))
     assert e.value.name == "DUO_ERR_UNSUPPORTED"

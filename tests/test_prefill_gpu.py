@@ -101,3 +101,44 @@ def test_prefill_rejects_unsupported_and_capacity():
     with pytest.raises(DuoError) as e:
         cb.prefill(0, qb, qb, qb)
     assert e.value.name == "DUO_ERR_CAPACITY"
+
+
+def _int4_view(x):
+    """What a 4-bit cache holds for bf16 rows x [B, n, H, D]: the exact
+    dequantisation of each (token, head) group, float64."""
+    from oracle import int4 as OQ
+    return OQ.dequantize_int4(*OQ.quantize_int4(x.float().cpu().numpy()))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,S,R", [(1, 8, 2, 4, 64), (2, 8, 4, 64, 256)])
+@pytest.mark.parametrize("paged", [False, True])
+def test_prefill_int4_cache(B, Hq, Hkv, S, R, paged):
+    """Chunks attend to a 4-bit cache (expanded to bf16 for the tensor cores)
+    plus their own bf16 k/v; the oracle reads the dequantised history exactly."""
+    bounds = [(0, 300), (300, 812), (812, 1500)]
+    n = bounds[-1][1]
+    seed = 41 + Hkv + S
+    Q, K, V = _prompt(seed, B, n, Hq, Hkv)
+    mask = seeded_mask(seed, Hkv, max(1, Hkv // 2))
+    kw = dict(pool_blocks=B * 8) if paged else {}
+    cache = DuoCache(1, B, Hq, Hkv, 128, "int4", n, mask[None], S, R, **kw)
+    assert cache.prefill_ws_bytes > 0
+    outs = _run_chunks(cache, Q, K, V, bounds)
+    Kq, Vq = _int4_view(K), _int4_view(V)
+    for (c0, o), (_, c1) in zip(outs, bounds):
+        k_view = np.concatenate([Kq[:, :c0], f64(K[:, c0:c1])], axis=1)
+        v_view = np.concatenate([Vq[:, :c0], f64(V[:, c0:c1])], axis=1)
+        ref = OA.prefill_reference(f64(Q[:, c0:c1]), k_view, v_view, c0, mask.numpy(), S, R)
+        assert_parity(o, ref, "bf16", "int4 prefill chunk at %d" % c0)
+
+
+def test_prefill_int4_needs_workspace():
+    from head_split_kv_decode_b200 import binding as Bd
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    c4 = DuoCache(1, 1, 8, 2, 128, "int4", 512, mask[None], 4, 64)
+    qb = torch.zeros(1, 128, 8, 128, device="cuda", dtype=BF)
+    kb = torch.zeros(1, 128, 2, 128, device="cuda", dtype=BF)
+    with pytest.raises(Bd.DuoError) as e:
+        Bd.duo_prefill_attn(c4.handle, 0, qb.data_ptr(), kb.data_ptr(), kb.data_ptr(), 128,
+                            qb.data_ptr(), 0.0, None, 0)
+    assert e.value.name == "DUO_ERR_WORKSPACE"
