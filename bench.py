@@ -147,15 +147,15 @@ class ClockSampler:
 
 # DRAM traffic of one fused decode launch (dram__bytes_read.sum +
 # dram__bytes_write.sum) from an ncu capture of one layer of the 128K batch-1
-# GQA workload (4 retrieval + 4 streaming KV heads, context 131075), and that
+# GQA workload (4 retrieval + 4 streaming KV heads, context 131076), and that
 # launch's algorithmic bytes.  The ratio scales to the benchmark's launches; it
 # is reported only while the kernel's sources hash as they did when the
 # counters were taken (otherwise traffic is null).
 DECODE_TRAFFIC = {
     "sources": ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h"),
-    "sha256": "249c97faa4c8fbeb90a80da2820e9932755cd0926ccfa1d8cfb9c0120d98a5a4",
-    "dram_bytes": 269760768 + 4478720,
-    "algorithmic_bytes": 269117440,
+    "sha256": "8bfbbe46ac82eafbe9d4c1ef9e95dee617a8cf4005a3d7d1e3b0567c7e1479f7",
+    "dram_bytes": 269782272 + 5693952,
+    "algorithmic_bytes": 269120512,
 }
 
 
