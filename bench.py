@@ -454,6 +454,70 @@ def run_paged_mixed(args, w, rank, world, peaks):
     return res
 
 
+def run_shard_rank(args, w, world_emulated, rank, peaks):
+    """One rank's share of a sequence-sharded decode: the sequence of
+    w.context * world_emulated tokens is split into world_emulated shards; this
+    measures rank 0 (the first w.context positions, and the streaming heads) —
+    per layer one partial decode and the merge of world_emulated partials.  The
+    exchange of the partials between GPUs is not part of it."""
+    from head_split_kv_decode_b200.cache import DuoCache, merge_partials
+    from head_split_kv_decode_b200 import shard
+
+    K_, Wm = min(args.steps, 16), args.warmup
+    total = w.context * world_emulated
+    lo, hi = shard.shard_ranges(total, world_emulated)[0]
+    mask = synth.workload_mask(w)
+    dt = torch.bfloat16
+    cache = DuoCache(w.layers, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, "bf16", hi - lo, mask,
+                     w.S, w.R)
+    cache.set_retrieval_shard(lo, hi)
+    zeros = torch.zeros(1, 65536, w.n_kv_heads, w.head_dim, dtype=dt, device="cuda")
+    b_ids = [rank]
+    for layer in range(w.layers):
+        for p0 in range(0, hi, 16384):  # this shard's positions: real values
+            pos = range(p0, p0 + 16384)
+            k = synth.history(w, layer, "k", b_ids, pos, device="cuda", mask_row=mask[layer])
+            v = synth.history(w, layer, "v", b_ids, pos, device="cuda", mask_row=mask[layer])
+            cache.append(layer, k.to(dt).contiguous(), v.to(dt).contiguous())
+        for p0 in range(hi, total, 65536):  # the other shards' positions only pass through
+            cache.append(layer, zeros, zeros)  # the streaming window
+        torch.cuda.synchronize()
+    q = [synth.queries(w, layer, b_ids, [total - 1], device="cuda")[:, 0].to(dt).contiguous()
+         for layer in range(w.layers)]
+    o_all = torch.full((world_emulated, 1, w.n_q_heads, w.head_dim), 0.0, device="cuda")
+    lse_all = torch.full((world_emulated, 1, w.n_q_heads), -float("inf"), device="cuda")
+    out = torch.empty(1, w.n_q_heads, w.head_dim, dtype=dt, device="cuda")
+
+    def step():
+        for layer in range(w.layers):
+            cache.decode_partial(layer, q[layer], o_all[0], lse_all[0], owns_streaming=True)
+            merge_partials(o_all, lse_all, out)
+
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K_):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K_
+    n_ret = [int(mask[layer].sum()) for layer in range(w.layers)]
+    step_bytes = sum(decode_bytes_per_layer(w, 1, hi - lo, n_ret[l], 0) +
+                     (w.n_kv_heads - n_ret[l]) * min(total, w.S + w.R) * 4 * w.head_dim * 2
+                     for l in range(w.layers))
+    res = {"workload": "%s: rank 0 of %d shards of a %d-token sequence (partial decode + merge of "
+                       "%d partials per layer; the exchange between GPUs not included)"
+                       % (w.name, world_emulated, total, world_emulated),
+           "value": step_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+           "ms_per_layer": ms / w.layers, "gpu_launches": 2 * w.layers,
+           "frac": step_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del cache
+    torch.cuda.empty_cache()
+    return res
+
+
 # --------------------------------------------------------------------------- prefill
 
 
@@ -716,6 +780,7 @@ def main(argv=None):
                           "decode_splits": rx["splits"], "gpu_launches": rx["gpu_launches"]}
         extra["llama3_8b_gqa_paged_mixed"] = run_paged_mixed(
             args, synth.WORKLOADS["llama3_8b_gqa_paged_mixed"], rank, world, peaks)
+        extra["sequence_sharded_1m_rank0_of_8"] = run_shard_rank(args, w, 8, rank, peaks)
         pq = run_prefill(args, synth.WORKLOADS["llama3_8b_gqa_prefill_32k"], rank, world, peaks,
                          kv_dtype="int4")
         extra["prefill_int4_cache"] = {k: pq[k] for k in ("value", "unit", "exact_tflops",

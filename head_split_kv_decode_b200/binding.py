@@ -89,6 +89,9 @@ SIGNATURES = {
     "duo_prefill_attn": (_I32, [_P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
     "duo_prefill_attn_rows": (_I32, [_P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _F, _P, _SZ, _P]),
     "duo_prefill_workspace_bytes": (_I32, [_P, ctypes.POINTER(_SZ)]),
+    "duo_set_retrieval_shard": (_I32, [_P, _I64, _I64]),
+    "duo_decode_attn_partial": (_I32, [_P, _I32, _P, _P, _P, _I32, _F, _P, _SZ, _P]),
+    "duo_merge_partials": (_I32, [_I32, _I64, _I32, _P, _P, _P, _I32, _P]),
     "duo_seq_len": (_I32, [_P, _I32, ctypes.POINTER(_I64)]),
     "duo_row_seq_len": (_I32, [_P, _I32, _I32, ctypes.POINTER(_I64)]),
     "duo_row_blocks": (_I32, [_P, _I32, _P, _I32, ctypes.POINTER(_I32)]),
@@ -316,3 +319,20 @@ def duo_poll_device_error():
     if st not in (DUO_OK, 6):
         raise DuoError(st, "duo_poll_device_error")
     return code.value
+
+
+def duo_set_retrieval_shard(handle, lo, hi):
+    _check(lib().duo_set_retrieval_shard(handle, lo, hi), "duo_set_retrieval_shard")
+
+
+def duo_decode_attn_partial(handle, layer, q_ptr, o_ptr, lse_ptr, owns_streaming, softmax_scale,
+                            ws_ptr, ws_bytes, stream=0):
+    _check(lib().duo_decode_attn_partial(handle, layer, q_ptr, o_ptr, lse_ptr,
+                                         1 if owns_streaming else 0, softmax_scale, ws_ptr,
+                                         ws_bytes, stream), "duo_decode_attn_partial")
+
+
+def duo_merge_partials(n_parts, rows, head_dim, o_ptr, lse_ptr, out_ptr, out_dtype, stream=0):
+    _check(lib().duo_merge_partials(n_parts, rows, head_dim, o_ptr, lse_ptr, out_ptr,
+                                    KV_DTYPES.get(out_dtype, out_dtype), stream),
+           "duo_merge_partials")

@@ -199,6 +199,28 @@ class DuoCache:
                                 _stream_handle(stream, self.device))
         return out
 
+    # ------------------------------------------------------------ sequence shards
+    def set_retrieval_shard(self, lo, hi):
+        """Keep only retrieval positions [lo, hi) (call before any append)."""
+        B.duo_set_retrieval_shard(self.handle, int(lo), int(hi))
+
+    def decode_partial(self, layer, q, o_part=None, lse_part=None, owns_streaming=True, scale=0.0,
+                       stream=None):
+        """This cache's share of the decode: returns (o_part f32 [batch, Hq, d],
+        lse_part f32 [batch, Hq]) to merge with :func:`merge_partials`."""
+        shape = (self.batch, self.n_q_heads, self.head_dim)
+        self._check(q, shape, "q")
+        if o_part is None:
+            o_part = torch.empty(shape, dtype=torch.float32, device=q.device)
+        if lse_part is None:
+            lse_part = torch.empty(shape[:2], dtype=torch.float32, device=q.device)
+        self._check(o_part, shape, "o_part", torch.float32)
+        self._check(lse_part, shape[:2], "lse_part", torch.float32)
+        B.duo_decode_attn_partial(self.handle, layer, q.data_ptr(), o_part.data_ptr(),
+                                  lse_part.data_ptr(), owns_streaming, float(scale), self.ws_ptr,
+                                  self.ws_bytes, _stream_handle(stream, self.device))
+        return o_part, lse_part
+
     def release_rows(self, rows=None):
         B.duo_release_rows(self.handle, None if rows is None else self._rows(rows))
 
@@ -277,3 +299,24 @@ class DuoCache:
             self.close()
         except Exception:
             pass
+
+
+def merge_partials(o_parts, lse_parts, out, stream=None):
+    """o_parts f32 [n, batch, Hq, d], lse_parts f32 [n, batch, Hq] (device,
+    contiguous) -> out [batch, Hq, d] (bf16 or f32): the attention over the
+    union of the shards' keys."""
+    n, rows, d = o_parts.shape[0], o_parts[0].numel() // o_parts.shape[-1], o_parts.shape[-1]
+    if tuple(lse_parts.shape) != tuple(o_parts.shape[:-1]) or tuple(out.shape) != tuple(o_parts.shape[1:]):
+        raise ValueError("partials and output shapes disagree")
+    for t in (o_parts, lse_parts, out):
+        if not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError("partials and output must be contiguous device tensors")
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise ValueError("partials must be float32")
+    kind = {torch.bfloat16: "bf16", torch.float32: "f32"}.get(out.dtype)
+    if kind is None:
+        raise ValueError("out must be bfloat16 or float32")
+    s = stream if stream is not None else torch.cuda.current_stream(out.device)
+    B.duo_merge_partials(n, rows, d, o_parts.data_ptr(), lse_parts.data_ptr(), out.data_ptr(), kind,
+                         s.cuda_stream)
+    return out

@@ -33,7 +33,8 @@ __global__ void append_kernel(const __grid_constant__ AppendParams a, int row_by
     int64_t off;
     uint8_t *dk, *dv;
     if (a.h.kind[h]) {
-      off = ret_row(a.ret, b, idx, p) * row_bytes;
+      if (p < a.shard_lo || p >= a.shard_hi) continue;  // another shard's position
+      off = ret_row(a.ret, b, idx, p - a.shard_lo) * row_bytes;
       dk = a.p.ret_k;
       dv = a.p.ret_v;
     } else {
@@ -77,7 +78,8 @@ __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
     int64_t row;
     uint8_t *codes, *sz;
     if (a.h.kind[h]) {
-      row = ret_row(a.ret, b, idx, p);
+      if (p < a.shard_lo || p >= a.shard_hi) continue;  // another shard's position
+      row = ret_row(a.ret, b, idx, p - a.shard_lo);
       codes = which ? a.p.ret_v : a.p.ret_k;
       sz = which ? a.p.ret_v_sz : a.p.ret_k_sz;
     } else {

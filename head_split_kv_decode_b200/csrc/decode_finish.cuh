@@ -12,15 +12,18 @@ namespace duo {
 // Second half of the epilogue: the per-warp states of the CTA are staged in
 // shared memory as red_m [NWARPS][G], red_l [NWARPS][G] (log2 units) and
 // red_o [NWARPS][G][D] (unnormalised), all starting at `smem`.  Combines them,
-// writes the output `out` (the G rows of this KV head's query heads) when
-// `direct`, or else this split's normalised partial and log-sum-exp into
-// slot part0 + split, and lets the last of the nsplit splits of the head
+// writes the result of this KV head's G query heads (rows out_row ..
+// out_row + G - 1 of the output, or of P.part_o / P.part_lse in partial mode)
+// when `direct`, or else this split's normalised partial and log-sum-exp
+// into slot part0 + split, and lets the last of the nsplit splits of the head
 // (merge ticket `unit`) merge slots part0 .. part0 + nsplit - 1.
 template <typename T, int D, int G, int NWARPS>
 __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8_t *smem,
-                                                    int *s_last_p, bool direct, T *out,
+                                                    int *s_last_p, bool direct, int64_t out_row,
                                                     int64_t unit, int64_t part0, int nsplit,
                                                     int split) {
+  constexpr float kLn2 = 0.6931471805599453f;  // log-sum-exps leave in natural log
+  T *out = reinterpret_cast<T *>(P.out) + out_row * D;
   constexpr int NT = NWARPS * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int &s_last = *s_last_p;
@@ -45,7 +48,11 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
     float O = 0.f;
 #pragma unroll
     for (int w = 0; w < NWARPS; ++w) O += red_o[(w * G + g) * D + c] * __shfl_sync(0xffffffffu, sw, w);
-    if (direct) {
+    if (direct && P.part_o) {
+      const bool empty = L == 0.f;  // this shard holds no key of the head
+      P.part_o[(out_row + g) * D + c] = empty ? 0.f : O / L;
+      if (c == 0) P.part_lse[out_row + g] = empty ? -INFINITY : (M + fast_log2(L)) * kLn2;
+    } else if (direct) {
       store_out(out + g * D + c, O / L);
     } else {
       // a split whose CTA claimed no keys leaves weight zero (lse -inf)
@@ -76,9 +83,10 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   // query head (D/4 float4 per head row; for D = 64 the upper lanes idle).
   // The first batch of partials is loaded before the weights are reduced, so
   // that its latency overlaps that reduction.
-  float *s_w = reinterpret_cast<float *>(smem);      // [nsplit][G]
-  float *s_den = s_w + nsplit * G;                   // [G]
-  float *s_acc = s_w + ((nsplit * G + G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
+  float *s_w = reinterpret_cast<float *>(smem);          // [nsplit][G]
+  float *s_den = s_w + nsplit * G;                       // [G]
+  float *s_mx = s_den + G;                               // [G]
+  float *s_acc = s_w + ((nsplit * G + 2 * G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
   constexpr int L4 = D / 4;
   constexpr int U = G >= 8 ? 2 : 4;
   const bool owns = lane < L4;
@@ -112,7 +120,10 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-    if (lane == 0) s_den[g] = den;
+    if (lane == 0) {
+      s_den[g] = den;
+      s_mx[g] = M;
+    }
   }
   __syncthreads();
   float4 acc[G];
@@ -153,7 +164,12 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
     float num = 0.f;
 #pragma unroll
     for (int w = 0; w < NWARPS; ++w) num += s_acc[(w * G + g) * D + c];
-    store_out(out + g * D + c, num / s_den[g]);
+    if (P.part_o) {
+      P.part_o[(out_row + g) * D + c] = num / s_den[g];
+      if (c == 0) P.part_lse[out_row + g] = (s_mx[g] + fast_log2(s_den[g])) * kLn2;
+    } else {
+      store_out(out + g * D + c, num / s_den[g]);
+    }
   }
   if (tid == 0) {  // leave the ticket (and chunk counter) ready for the next call
     *cnt = 0u;
@@ -216,10 +232,9 @@ __device__ __forceinline__ void decode_finish(const DecodeParams &P, uint8_t *sm
   // CUDA-core decode: packed layout, every batch row at length P.n, the
   // retrieval CTAs enumerated as ((b*n_ret + head)*nsplit + split).
   const int64_t unit = (int64_t)b * P.n_ret + (retrieval ? pidx : 0);
-  decode_reduce_store<T, D, G, NWARPS>(
-      P, smem, s_last_p, !retrieval || P.nsplit == 1,
-      reinterpret_cast<T *>(P.out) + ((int64_t)b * P.Hq + (int64_t)kvh * G) * D, unit,
-      unit * P.nsplit, P.nsplit, split);
+  decode_reduce_store<T, D, G, NWARPS>(P, smem, s_last_p, !retrieval || P.nsplit == 1,
+                                       (int64_t)b * P.Hq + (int64_t)kvh * G, unit,
+                                       unit * P.nsplit, P.nsplit, split);
 }
 
 }  // namespace duo

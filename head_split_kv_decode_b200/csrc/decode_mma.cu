@@ -130,12 +130,18 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // Key indices and tile counts are 32-bit (a row holds fewer than 2^31
   // tokens); byte offsets are formed in 64 bits.
   const int n = P.rows.len[r];  // tokens incl. the new one; the query is at n-1
+  // A sequence shard's retrieval heads hold positions [shard_lo, shard_hi)
+  // at page rows from 0; `keys` of them are below n.  Streaming heads hold
+  // the whole window.
+  const int keys = retrieval ? (int)max((int64_t)0, min((int64_t)n, P.shard_hi) - P.shard_lo)
+                             : min(n, P.W);
+  const bool new_here_shard = !retrieval || (n - 1 >= P.shard_lo && n - 1 < P.shard_hi);
   constexpr int RB = Q4 ? D / 2 : D * 2;  // bytes per key row
   // Streaming heads: one slot buffer, first storage row srow0.  Retrieval
   // heads: key tiles are addressed block by block (a tile never crosses a
   // block of the paged layout), with key indices local to the block.
   auto srow0 = [&]() { return ((int64_t)b * P.n_str + pidx) * P.Ws; };
-  const int k0 = 0, k1 = retrieval ? n : min(n, P.W);
+  const int k0 = 0, k1 = keys;
   constexpr int KG = Keys<Q4>::KG;
   constexpr int T = 16 * KG;  // keys per warp tile
   constexpr int kBlockMask = ~(kPageTokens - 1);
@@ -147,14 +153,14 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // partial.  Streaming heads and single-split heads walk [k0, k1).
   const bool split_head = retrieval && nsplit > 1;
   const bool pooled = split_head && P.pool;
-  const int tiles = (n + T - 1) / T;
+  const int tiles = (keys + T - 1) / T;
   const int ts = !split_head ? 0
                  : pooled    ? (tiles - tiles / 8) / nsplit
                              : (tiles + nsplit - 1) / nsplit;  // tiles per split share
   const int t1 = min(tiles, (split + 1) * ts);                 // end of this split's share
   // this warp's first two tiles, [first, first + T) and the one NWARPS tiles on
   const int first = split_head ? (split * ts + warp) * T : k0 + warp * T;
-  const int last = split_head ? min(n, t1 * T) : k1;
+  const int last = split_head ? min(keys, t1 * T) : k1;
 
   // Launched with programmatic dependent launch, so this may run while the
   // previous kernel in the stream finishes.  Bring this warp's first two
@@ -199,8 +205,16 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // Fused append (bf16 cache): the token at position n-1 is not in the cache
   // yet.  The warp whose tile holds its row writes it there, skips that row,
   // and adds the key at the end from the inputs.
-  const bool fused = !Q4 && P.knew != nullptr;
-  const int newk = retrieval ? n - 1 : (int)ring_slot(n - 1, P.S, P.R);  // its key index in this head
+  // In partial mode a rank that does not own the streaming heads leaves
+  // their rows empty (another shard contributes them).
+  if (P.part_o && !retrieval && !P.own_str) {
+    const int64_t row0 = (int64_t)r * P.Hq + (int64_t)kvh * G;
+    for (int i = tid; i < G * D; i += NWARPS * 32) P.part_o[row0 * D + i] = 0.f;
+    if (tid < G) P.part_lse[row0 + tid] = -INFINITY;
+    return;
+  }
+  const bool fused = !Q4 && P.knew != nullptr && new_here_shard;
+  const int newk = retrieval ? n - 1 - (int)P.shard_lo : (int)ring_slot(n - 1, P.S, P.R);  // its row
   const bool owns_new = fused && !split_head && newk >= k0 && newk < k1;
   auto write_new = [&]() {  // one warp copies the new K and V rows into the cache
     const int64_t off = ((int64_t)r * P.Hkv + kvh) * (int64_t)RB;
@@ -475,7 +489,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         write_new();
         new_here = true;
       }
-      run_tile(kb0, n, has_new ? newk : -1);
+      run_tile(kb0, keys, has_new ? newk : -1);
     };
     unsigned c = 0;
     int tt = split * ts + warp;
@@ -540,8 +554,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   }
   __syncthreads();
   decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(
-      P, smem, &s_last, nsplit == 1,
-      reinterpret_cast<__nv_bfloat16 *>(P.out) + ((int64_t)r * P.Hq + (int64_t)kvh * G) * D,
+      P, smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
       (int64_t)r * P.n_ret + pidx, (int64_t)(retrieval ? P.cta0[r] : 0) + (int64_t)pidx * nsplit,
       nsplit, split);
 }

@@ -62,6 +62,7 @@ struct duo_cache {
   int row_bytes;
   uint8_t *base;
   int forced_splits;
+  int64_t shard_lo, shard_hi;  // retrieval heads keep positions [lo, hi) (sequence shard)
   bool reproducible;       // decode splits take fixed key shares only
   bool have_cfg;           // decode launch facts, queried once per cache
   duo::DecodeConfig cfg;
@@ -82,6 +83,15 @@ int64_t &len_of(duo_cache *c, int layer, int row) {
 }
 int64_t len_of(const duo_cache *c, int layer, int row) {
   return c->seq_len[(size_t)layer * c->desc.batch + row];
+}
+
+constexpr int64_t kNoShardEnd = 1LL << 62;
+
+bool sharded(const duo_cache *c) { return c->shard_lo != 0 || c->shard_hi != kNoShardEnd; }
+
+// Retrieval rows a row holds in this cache's shard when its length is n.
+int64_t ret_len(const duo_cache *c, int64_t n) {
+  return std::max<int64_t>(0, std::min(n, c->shard_hi) - c->shard_lo);
 }
 
 bool mma_path(const duo_cache *c) {
@@ -249,7 +259,7 @@ duo_status check_room(const duo_cache *c, int layer, const std::vector<int32_t> 
                       int64_t n_tokens) {
   if (c->layers[layer].n_ret == 0 && c->layout == DUO_LAYOUT_PACKED) return DUO_OK;
   for (int b : rows)
-    if (len_of(c, layer, b) + n_tokens > c->desc.capacity) return DUO_ERR_CAPACITY;
+    if (ret_len(c, len_of(c, layer, b) + n_tokens) > c->desc.capacity) return DUO_ERR_CAPACITY;
   return DUO_OK;
 }
 
@@ -263,7 +273,7 @@ duo_status reserve_blocks(duo_cache *c, int layer, const std::vector<int32_t> &r
   std::vector<int32_t> need(rows.size());
   int64_t total = 0;
   for (size_t i = 0; i < rows.size(); ++i) {
-    const int64_t end = len_of(c, layer, rows[i]) + n_tokens;
+    const int64_t end = ret_len(c, len_of(c, layer, rows[i]) + n_tokens);
     const int64_t blocks = (end + duo::kPageTokens - 1) / duo::kPageTokens;
     need[i] = (int32_t)std::max<int64_t>(0, blocks - c->held[rows[i]]);
     total += need[i];
@@ -345,6 +355,8 @@ duo_status create(duo_cache **out, const duo_cache_desc *desc, const uint8_t *he
   c->seq_len.assign((size_t)d.layers * d.batch, 0);
   c->base = nullptr;
   c->forced_splits = 0;
+  c->shard_lo = 0;
+  c->shard_hi = kNoShardEnd;
   c->reproducible = false;
   c->have_cfg = false;
   c->row_bytes = d.kv_dtype == DUO_INT4 ? d.head_dim / 2 : d.head_dim * elem_bytes(d.kv_dtype);
@@ -425,6 +437,8 @@ duo_status append_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &
   a.W = c->W;
   a.Ws = c->Ws;
   a.n_tok = n_tokens;
+  a.shard_lo = c->shard_lo;
+  a.shard_hi = c->shard_hi;
   // inputs [rows][n_tokens][Hkv][D] in f32 (f32 caches) or bf16
   const int64_t in_row = (int64_t)n_tokens * d.n_kv_heads * d.head_dim * elem_bytes(d.kv_dtype);
   for (size_t g0 = 0; g0 < rows.size(); g0 += duo::kMaxLaunchRows) {
@@ -471,7 +485,15 @@ void fill_decode_common(const duo_cache *c, int32_t layer, const void *q, void *
   p->scale_log2 = sc * 1.4426950408889634f;
   p->err = duo::device_error_word();
   p->pool = c->reproducible ? 0 : 1;
+  p->shard_lo = c->shard_lo;
+  p->shard_hi = c->shard_hi;
 }
+
+// Partial-mode outputs of a decode (sequence shards), or none.
+struct Partial {
+  float *o, *lse;
+  int own_str;
+};
 
 // Where a decode launch keeps its split partials: the caller's workspace, or
 // the library's static array (cleared on the stream before the launch).
@@ -525,9 +547,14 @@ duo_status attach_scratch(const duo_cache *c, int64_t units, int64_t slots, cons
 // each row's new token is appended in the same launch (fused step).
 duo_status decode_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &rows,
                        const void *q, const void *k_new, const void *v_new, void *out, float scale,
-                       const Scratch &scratch, cudaStream_t s) {
-  if (!q || !out || !std::isfinite(scale)) return DUO_ERR_ARG;
+                       const Scratch &scratch, cudaStream_t s, const Partial *part = nullptr) {
+  if (!q || !std::isfinite(scale)) return DUO_ERR_ARG;
+  if (part ? (!part->o || !part->lse) : !out) return DUO_ERR_ARG;
   const bool fused = k_new != nullptr;
+  // A shard's decode is only meaningful as a partial to be merged; partials
+  // come from the tensor-core decode and do not append.
+  if (sharded(c) && !part) return DUO_ERR_UNSUPPORTED;
+  if (part && (fused || !mma_path(c))) return DUO_ERR_UNSUPPORTED;
   const duo_cache_desc &d = c->desc;
   const auto &L = c->layers[layer];
   const int G = d.n_q_heads / d.n_kv_heads;
@@ -571,13 +598,20 @@ duo_status decode_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &
     const int nr = (int)std::min<size_t>(duo::kMaxLaunchRows, rows.size() - g0);
     duo::DecodeParams &p = plans[i];
     fill_decode_common(c, layer, static_cast<const uint8_t *>(q) + (int64_t)g0 * q_row,
-                       static_cast<uint8_t *>(out) + (int64_t)g0 * q_row, scale, &p);
+                       out ? static_cast<uint8_t *>(out) + (int64_t)g0 * q_row : nullptr, scale, &p);
     p.rows.n = nr;
+    int32_t rlen[duo::kMaxLaunchRows];  // retrieval keys of each row in this shard
     for (int r = 0; r < nr; ++r) {
       p.rows.row[r] = rows[g0 + r];
       p.rows.len[r] = (int32_t)(len_of(c, layer, rows[g0 + r]) + (fused ? 1 : 0));
+      rlen[r] = (int32_t)ret_len(c, p.rows.len[r]);
     }
-    choose_row_splits(c, layer, p.rows.len, nr, cfg, p.nsplit_r);
+    choose_row_splits(c, layer, rlen, nr, cfg, p.nsplit_r);
+    if (part) {
+      p.part_o = part->o + (int64_t)g0 * d.n_q_heads * d.head_dim;
+      p.part_lse = part->lse + (int64_t)g0 * d.n_q_heads;
+      p.own_str = part->own_str;
+    }
     p.cta0[0] = 0;
     for (int r = 0; r < nr; ++r) {
       p.cta0[r + 1] = p.cta0[r] + L.n_ret * p.nsplit_r[r];
@@ -662,6 +696,7 @@ duo_status prefill_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> 
   const auto &L = c->layers[layer];
   duo_status st = check_room(c, layer, rows, C);
   if (st != DUO_OK) return st;
+  if (sharded(c)) return DUO_ERR_UNSUPPORTED;
   const bool q4 = d.kv_dtype == DUO_INT4;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   if (q4) {
@@ -890,6 +925,41 @@ duo_status duo_release_rows(duo_cache *c, const int32_t *rows, int32_t n_rows) {
   return DUO_OK;
 }
 
+duo_status duo_set_retrieval_shard(duo_cache *c, int64_t lo, int64_t hi) {
+  if (!c || lo < 0 || hi <= lo) return DUO_ERR_ARG;
+  if (!mma_path(c)) return DUO_ERR_UNSUPPORTED;
+  for (int64_t n : c->seq_len)
+    if (n != 0) return DUO_ERR_STATE;
+  c->shard_lo = lo;
+  c->shard_hi = std::min(hi, kNoShardEnd);
+  return DUO_OK;
+}
+
+duo_status duo_decode_attn_partial(duo_cache *c, int32_t layer, const void *q, float *o_part,
+                                   float *lse_part, int32_t owns_streaming, float scale, void *ws,
+                                   size_t ws_bytes, duo_stream stream) {
+  duo_status st = check_layer(c, layer);
+  if (st != DUO_OK) return st;
+  if (owns_streaming != 0 && owns_streaming != 1) return DUO_ERR_ARG;
+  std::vector<int32_t> list;
+  if ((st = make_rows(c, nullptr, 0, &list)) != DUO_OK) return st;
+  const Partial part{o_part, lse_part, owns_streaming};
+  return decode_rows(c, layer, list, q, nullptr, nullptr, nullptr, scale,
+                     Scratch{ws, ws_bytes, false}, (cudaStream_t)stream, &part);
+}
+
+duo_status duo_merge_partials(int32_t n_parts, int64_t rows, int32_t head_dim, const float *o_parts,
+                              const float *lse_parts, void *out, int32_t out_dtype,
+                              duo_stream stream) {
+  if (n_parts <= 0 || rows <= 0 || !o_parts || !lse_parts || !out) return DUO_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return DUO_ERR_ARG;
+  if (out_dtype != DUO_F32 && out_dtype != DUO_BF16) return DUO_ERR_ARG;
+  if (!aligned16(o_parts)) return DUO_ERR_ARG;
+  return launch_status(duo::launch_merge_partials(n_parts, rows, head_dim, o_parts, lse_parts, out,
+                                                  out_dtype == DUO_F32 ? duo::kF32 : duo::kBF16,
+                                                  (cudaStream_t)stream));
+}
+
 duo_status duo_seq_len(const duo_cache *c, int32_t layer, int64_t *n) {
   if (!c || !n || layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
   int64_t m = 0;
@@ -937,7 +1007,7 @@ duo_status duo_kv_bytes(const duo_cache *c, int64_t *kept, int64_t *full) {
     for (int b = 0; b < d.batch; ++b) {
       const int64_t n = len_of(c, l, b);
       const int64_t win = n < c->W ? n : c->W;
-      k += (c->layers[l].n_ret * n + c->layers[l].n_str * win) * per;
+      k += (c->layers[l].n_ret * ret_len(c, n) + c->layers[l].n_str * win) * per;
       f += (int64_t)d.n_kv_heads * n * per;
     }
   if (kept) *kept = k;

@@ -74,6 +74,7 @@ struct AppendParams {
   HeadTables h;
   RetMap ret;
   LaunchRows rows;     // len = tokens in the cache before this append
+  int64_t shard_lo, shard_hi;  // retrieval heads keep positions [lo, hi) at row p - lo
   int Hkv, D, n_ret, n_str, S, R, W;
   int Ws;              // rows per streaming head buffer (W, or W rounded up to 4 for int4)
   int64_t n_tok;
@@ -101,6 +102,15 @@ struct DecodeParams {
   int32_t cta0[kMaxLaunchRows + 1];
   int16_t nsplit_r[kMaxLaunchRows];
   RetMap ret;
+  // Sequence shard: retrieval heads hold positions [shard_lo, shard_hi) at
+  // page row position - shard_lo (default [0, 2^62)).
+  int64_t shard_lo, shard_hi;
+  // Partial mode (part_o non-null): instead of out, every query head leaves
+  // its normalised output [rows.n][Hq][D] f32 in part_o and its natural-log
+  // log-sum-exp [rows.n][Hq] in part_lse (-inf and zeros where it saw no
+  // key); streaming heads contribute only when own_str.
+  float *part_o, *part_lse;
+  int own_str;
   float scale_log2;    // softmax scale * log2(e)
   float *ws_o;         // [partial slots][G][D]
   float *ws_lse;       // [partial slots][G]
@@ -169,6 +179,11 @@ bool decode_mma_supported(int kv_type, int D, int G);
 cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s);
 cudaError_t launch_table_writes(int32_t *table, const TableWrites &w, cudaStream_t s);
 cudaError_t launch_dequant_history(const DequantParams &d, cudaStream_t s);
+// out[rows][D] = sum_i exp(lse_i - L) o_i, L = log sum_i exp(lse_i), over
+// n_parts partials o [n_parts][rows][D] f32, lse [n_parts][rows] (natural log);
+// out_type kBF16 or kF32.
+cudaError_t launch_merge_partials(int n_parts, int64_t rows, int D, const float *o,
+                                  const float *lse, void *out, int out_type, cudaStream_t s);
 int *device_error_word();  // device address of the error word
 
 // Library-owned decode scratch for duo_decode_attn_static (decode_static.cu).

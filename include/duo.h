@@ -299,6 +299,44 @@ duo_status duo_prefill_attn_rows(duo_cache *cache, int32_t layer, const int32_t 
  * streaming buffers (K and V), for the largest layer. */
 duo_status duo_prefill_workspace_bytes(const duo_cache *cache, size_t *bytes);
 
+/* Sequence sharding, for a sequence too long for one GPU's retrieval caches:
+ * several caches (normally one per GPU) each keep a contiguous range of the
+ * retrieval heads' positions, and every one keeps the whole, tiny, streaming
+ * state.  After this call the cache's retrieval heads store only positions
+ * [lo, hi) of each row, at page (or block) rows position - lo; appends still
+ * pass every token (positions outside [lo, hi) touch only the streaming
+ * heads), and capacity counts the rows this shard stores.  Such a cache
+ * decodes only through duo_decode_attn_partial, and pre-fill is not offered.
+ * Call while every length is 0 (fresh, bound or reset cache).  Tensor-core
+ * decode configurations only (bf16 or 4-bit KV, head_dim 128).
+ * Errors: DUO_ERR_ARG (lo < 0 or hi <= lo), DUO_ERR_STATE (tokens present),
+ * DUO_ERR_UNSUPPORTED (other configurations). */
+duo_status duo_set_retrieval_shard(duo_cache *cache, int64_t lo, int64_t hi);
+
+/* Decode attention of every row over this cache's share of the keys, as a
+ * partial to merge with the other shards': per (row, query head) the output
+ * normalised over this share, o_part [batch, n_q_heads, head_dim] float32, and
+ * the natural-log log-sum-exp of the scaled scores over it, lse_part [batch,
+ * n_q_heads] float32 (-inf with o_part 0 where the share holds no visible
+ * key).  Streaming heads are included only when owns_streaming is 1 (exactly
+ * one shard should own them; every shard holds the same streaming state).
+ * Does not append.  Workspace as for duo_decode_attn.  Works on unsharded
+ * caches too (the whole sequence as one share). */
+duo_status duo_decode_attn_partial(duo_cache *cache, int32_t layer, const void *q,
+                                   float *o_part, float *lse_part, int32_t owns_streaming,
+                                   float softmax_scale, void *workspace,
+                                   size_t workspace_bytes, duo_stream stream);
+
+/* Merge n_parts partials (the shards' o_part / lse_part, gathered in device
+ * memory as o_parts [n_parts, rows, head_dim] and lse_parts [n_parts, rows]
+ * float32, rows = batch * n_q_heads) into out [rows, head_dim] of out_dtype
+ * (DUO_BF16 or DUO_F32): out = sum_i exp(lse_i - L) o_i, L = log sum_i
+ * exp(lse_i); rows no shard saw a key of are 0.  The exchange of the partials
+ * between GPUs (an all-gather over NVLink) is the caller's. */
+duo_status duo_merge_partials(int32_t n_parts, int64_t rows, int32_t head_dim,
+                              const float *o_parts, const float *lse_parts, void *out,
+                              int32_t out_dtype, duo_stream stream);
+
 /* The longest row's length in one layer (every row's, when all rows advance
  * together). */
 duo_status duo_seq_len(const duo_cache *cache, int32_t layer, int64_t *n);
