@@ -153,8 +153,8 @@ class ClockSampler:
 # counters were taken (otherwise traffic is null).
 DECODE_TRAFFIC = {
     "sources": ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h"),
-    "sha256": "8bfbbe46ac82eafbe9d4c1ef9e95dee617a8cf4005a3d7d1e3b0567c7e1479f7",
-    "dram_bytes": 269782272 + 5693952,
+    "sha256": "6fd07545dbe932c3018517ffdb397ebf446b12761c44dabc6006db5acedf031f",
+    "dram_bytes": 269783296 + 5163008,
     "algorithmic_bytes": 269120512,
 }
 
