@@ -52,6 +52,11 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
+template <bool B>
+struct BoolC {
+  static constexpr bool value = B;
+};
+
 __device__ __forceinline__ uint4 ldg128(const void *p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -280,8 +285,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // One warp, keys [kb0, kb0 + 16*KG) below hi of the buffers Kx/Vx (and, for
   // the 4-bit cache, the (scale, zero) rows Ksx/Vsx), row index = key, except
   // `skip_key`.
-  auto tile = [&](const uint8_t *Kx, const uint8_t *Vx, const uint8_t *Ksx, const uint8_t *Vsx,
-                  int kb0, int hi, int skip_key) {
+  // `full` (a compile-time flag) promises that all keys of the tile lie below
+  // hi and none is skip_key, so no load or score needs a bounds test.
+  auto tile = [&](auto full, const uint8_t *Kx, const uint8_t *Vx, const uint8_t *Ksx,
+                  const uint8_t *Vsx, int kb0, int hi, int skip_key) {
+    constexpr bool FULL = decltype(full)::value;
     // ------------------------------------------------------------ loads (all up front)
     // group kg covers keys kb = kb0 + 16*kg ..: K of key kb + 8*nt + g (this
     // thread's column of S); V of keys kb + {2t, 2t+1, 8+2t, 9+2t} (the k-slots
@@ -295,12 +303,12 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int key = kb + 8 * nt + g;
-        const bool ok = key < hi && key != skip_key;
+        const bool ok = FULL || (key < hi && key != skip_key);
         if (Q4) {
           kr[kg][nt][0] = ok ? ldg128(Kx + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
           const int key2 = kb + 8 * nt + 2 * t;
-          ksz[kg][nt] = key2 < hi ? ldg64(Ksx + key2 * 4) : make_uint2(0, 0);
-          vsz[kg][nt] = key2 < hi ? ldg64(Vsx + key2 * 4) : make_uint2(0, 0);
+          ksz[kg][nt] = (FULL || key2 < hi) ? ldg64(Ksx + key2 * 4) : make_uint2(0, 0);
+          vsz[kg][nt] = (FULL || key2 < hi) ? ldg64(Vsx + key2 * 4) : make_uint2(0, 0);
         } else {
 #pragma unroll
           for (int sp = 0; sp < 4; ++sp)
@@ -310,7 +318,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
-        const bool ok = key < hi && key != skip_key;
+        const bool ok = FULL || (key < hi && key != skip_key);
         if (Q4) {
           const uint2 x = ok ? ldg64(Vx + key * RB + 8 * g) : make_uint2(0, 0);
           vr[kg][i][0] = make_uint4(x.x, x.y, 0, 0);
@@ -354,7 +362,8 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
             const float ksc = __low2float(kp);
             raw = ksc * raw + (__high2float(kp) - 128.f * ksc) * qsum;
           }
-          sc[kg][nt][e] = (live && key + e < hi && key + e != skip_key) ? raw * sl2 : -INFINITY;
+          sc[kg][nt][e] =
+              (live && (FULL || (key + e < hi && key + e != skip_key))) ? raw * sl2 : -INFINITY;
         }
       }
     }
@@ -473,8 +482,17 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       row = srow0();
       pk = P.p.str_k, pv = P.p.str_v, psk = P.p.str_k_sz, psv = P.p.str_v_sz;
     }
-    tile(pk + row * RB, pv + row * RB, Q4 ? psk + row * 4 : nullptr, Q4 ? psv + row * 4 : nullptr,
-         kb0 - base, hi - base, skip_key < 0 ? -1 : skip_key - base);
+    // 4-bit only: on the bf16 path a second copy of the tile costs more in
+    // registers than the bounds tests it saves
+    if constexpr (Q4) {
+      const int lo_k = kb0 - base, hi_k = hi - base, sk = skip_key < 0 ? -1 : skip_key - base;
+      if (lo_k + T <= hi_k && (sk < lo_k || sk >= lo_k + T)) {
+        tile(BoolC<true>{}, pk + row * RB, pv + row * RB, psk + row * 4, psv + row * 4, lo_k, hi_k, sk);
+        return;
+      }
+    }
+    tile(BoolC<false>{}, pk + row * RB, pv + row * RB, Q4 ? psk + row * 4 : nullptr,
+         Q4 ? psv + row * 4 : nullptr, kb0 - base, hi - base, skip_key < 0 ? -1 : skip_key - base);
   };
   bool new_here = owns_new && warp == 0;  // this warp adds the new token at the end
   if (split_head) {
@@ -512,7 +530,8 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   if (new_here) {
     // the new token, straight from the inputs (key 0 of a one-row buffer)
     const int64_t off = ((int64_t)r * P.Hkv + kvh) * (int64_t)RB;
-    tile(reinterpret_cast<const uint8_t *>(P.knew) + off, reinterpret_cast<const uint8_t *>(P.vnew) + off,
+    tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + off,
+         reinterpret_cast<const uint8_t *>(P.vnew) + off,
          nullptr, nullptr, 0, 1, -1);
   }
 
