@@ -416,11 +416,11 @@ duo_status create(duo_cache **out, const duo_cache_desc *desc, const uint8_t *he
 
 duo_status append_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &rows,
                        const void *k, const void *v, int32_t n_tokens, cudaStream_t s) {
-  if (!k || !v || n_tokens < 0) return DUO_ERR_ARG;
-  if (!aligned16(k) || !aligned16(v)) return DUO_ERR_ARG;
+  if (n_tokens < 0) return DUO_ERR_ARG;
+  if (n_tokens > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return DUO_ERR_ARG;
   duo_status st = check_room(c, layer, rows, n_tokens);
   if (st != DUO_OK) return st;
-  if (n_tokens == 0) return DUO_OK;
+  if (n_tokens == 0) return DUO_OK;  // k and v are not read (may be NULL)
   if ((st = reserve_blocks(c, layer, rows, n_tokens, s)) != DUO_OK) return st;
   const auto &L = c->layers[layer];
   const duo_cache_desc &d = c->desc;

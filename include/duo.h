@@ -178,7 +178,8 @@ duo_status duo_release_rows(duo_cache *cache, const int32_t *rows, int32_t n_row
  * there.  INT4 caches quantise each (token, head) row of head_dim channels
  * (asymmetric min/max, fp16 scale and zero, 4-bit codes, low nibble = even
  * channel).  Paged: rows take the blocks they need from the pool first.
- * Advances each row's length by n_tokens.
+ * Advances each row's length by n_tokens.  n_tokens == 0 changes nothing
+ * and reads neither k nor v (either may be NULL then).
  * Errors: DUO_ERR_CAPACITY if a row would pass capacity or the pool cannot
  * cover every row (nothing is changed then). */
 duo_status duo_append_kv(duo_cache *cache, int32_t layer, const void *k,

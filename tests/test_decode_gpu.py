@@ -162,6 +162,23 @@ def test_capacity_error_and_no_partial_state():
     assert cache.seq_len(0) == 10
 
 
+def test_empty_inputs():
+    """A zero-token append is a no-op (length, bytes and the next decode are
+    unchanged); decoding a layer that holds no token is a state error."""
+    from head_split_kv_decode_b200.binding import DuoError
+    cache, K, V, q, mask = _build(2, 8, 2, 128, "bf16", 300, 4, 64, n_ret=1, seed=9)
+    before = cache.decode(0, q).clone()
+    nb = cache.kv_bytes()
+    empty = torch.empty(2, 0, 2, 128, dtype=torch.bfloat16, device="cuda")
+    cache.append(0, empty, empty)
+    assert cache.seq_len(0) == 300 and cache.kv_bytes() == nb
+    assert torch.equal(cache.decode(0, q), before)
+    fresh = DuoCache(1, 2, 8, 2, 128, "bf16", 64, mask[None], 4, 64)
+    with pytest.raises(DuoError) as e:
+        fresh.decode(0, q)
+    assert e.value.name == "DUO_ERR_STATE"
+
+
 def test_workspace_too_small_is_rejected():
     from head_split_kv_decode_b200 import binding as B
     cache, K, V, q, mask = _build(1, 4, 2, 128, "bf16", 5000, 4, 64, n_ret=1, seed=3)
