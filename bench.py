@@ -153,8 +153,8 @@ class ClockSampler:
 # counters were taken (otherwise traffic is null).
 DECODE_TRAFFIC = {
     "sources": ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h"),
-    "sha256": "6fd07545dbe932c3018517ffdb397ebf446b12761c44dabc6006db5acedf031f",
-    "dram_bytes": 269783296 + 5163008,
+    "sha256": "abeb3a94fbd790f3cb6f27832eef02e415b99b53ec0fbd1e65e439171fe58b1c",
+    "dram_bytes": 269781760 + 4422400,
     "algorithmic_bytes": 269120512,
 }
 
