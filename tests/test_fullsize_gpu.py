@@ -4,7 +4,8 @@ the oracle computes one by one:
 
 * Llama-2-7B-shaped MHA decode at 32K context (needle keys planted in the
   retrieval heads), every query head of one layer;
-* Llama-3-8B-shaped GQA decode at 128K context, batch 1 and batch 4;
+* Llama-3-8B-shaped GQA decode at 128K context, batch 1 and batch 4, and 128
+  fused decode steps (append + attend) with the streaming rings checked after;
 * the 32K-token GQA pre-fill in 4K chunks (sampled rows of every chunk and head);
 * the 1M-token INT4 GQA decode (one retrieval and one streaming KV head).
 
@@ -19,6 +20,7 @@ import pytest
 import torch
 
 from oracle import attention as OA
+from oracle import cache as OC
 from oracle import int4 as OQ
 from head_split_kv_decode_b200 import synth
 from head_split_kv_decode_b200.cache import DuoCache
@@ -50,9 +52,10 @@ def _fill_decode(w, B, layer=0, chunk=16384):
     return cache, q, out, row
 
 
-def _oracle_head(w, layer, b, h, row, q, quantised=False):
-    """fp64 oracle for the G query heads of KV head h, batch row b, at t = context."""
-    t = w.context
+def _oracle_head(w, layer, b, h, row, q, quantised=False, t=None):
+    """fp64 oracle for the G query heads of KV head h, batch row b, at position
+    t (default: the context length)."""
+    t = w.context if t is None else t
     retrieval = bool(row[h])
     if retrieval:
         keys = np.arange(t + 1)
@@ -92,6 +95,48 @@ def test_llama3_gqa_128k_decode(B, rows):
         got = out[b].float().cpu()
         ref = np.concatenate([_oracle_head(w, 0, b, h, row, q) for h in range(w.n_kv_heads)])
         assert_parity(got, ref, "bf16", "128K GQA decode B=%d b=%d" % (B, b))
+
+
+def test_llama3_gqa_128k_128_fused_decode_steps():
+    """128 decode steps with ring-buffer append/evict at 128K, batch 1: each
+    step appends its token and attends in one fused launch.  Sampled steps
+    match the oracle (one retrieval and one streaming KV head), and after the
+    last step a streaming head's slot buffers hold the sinks and the last R
+    tokens bit for bit (the ring has advanced 128 slots)."""
+    w = synth.WORKLOADS["llama3_8b_gqa_128k"]
+    steps, n0, G = 128, w.context, w.group
+    row = synth.workload_mask(w)[0]
+    dt = synth.io_dtype(w)
+    cache = DuoCache(1, 1, w.n_q_heads, w.n_kv_heads, w.head_dim, w.kv_dtype, n0 + steps,
+                     row[None], w.S, w.R)
+    for p0 in range(0, n0, 16384):
+        pos = range(p0, min(n0, p0 + 16384))
+        k = synth.history(w, 0, "k", [0], pos, device="cuda", mask_row=row).to(dt)
+        v = synth.history(w, 0, "v", [0], pos, device="cuda", mask_row=row).to(dt)
+        cache.append(0, k.contiguous(), v.contiguous())
+    ret = [h for h in range(w.n_kv_heads) if row[h]][0]
+    strm = [h for h in range(w.n_kv_heads) if not row[h]][0]
+    for s_ in range(steps):
+        t = n0 + s_
+        k = synth.history(w, 0, "k", [0], [t], device="cuda", mask_row=row)[:, 0].to(dt).contiguous()
+        v = synth.history(w, 0, "v", [0], [t], device="cuda", mask_row=row)[:, 0].to(dt).contiguous()
+        q = synth.queries(w, 0, [0], [t], device="cuda")[:, 0].to(dt).contiguous()
+        out = cache.step(0, q, k, v)
+        if s_ in (0, 1, 77, steps - 1):
+            got = out[0].float().cpu()
+            for h in (ret, strm):
+                ref = _oracle_head(w, 0, 0, h, row, q, t=t)
+                assert_parity(got[h * G:(h + 1) * G], ref, "bf16", "step %d head %d" % (s_, h))
+    assert cache.seq_len(0) == n0 + steps
+    torch.cuda.synchronize()
+    idx = cache.layout(0).packed_index[strm]
+    for which, name in (("k", "str_k"), ("v", "str_v")):
+        hist = synth.history(w, 0, which, [0], range(n0 + steps), heads=[strm], mask_row=row)
+        hist = hist.to(dt)[0, :, 0].contiguous().view(torch.uint8).numpy()
+        exp, filled = OC.expected_streaming_buffer(hist, w.S, w.R)
+        got = cache.region(0, name)[0, idx].cpu().numpy()
+        assert filled.all()
+        np.testing.assert_array_equal(got[:w.S + w.R], exp)
 
 
 def test_llama3_gqa_prefill_32k_sampled_rows():
