@@ -58,28 +58,39 @@ constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                               ((uint32_t)(HD >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-// Shared-memory matrix descriptor, 128-byte swizzle.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+// Shared-memory matrix descriptor, 128-byte swizzle, split in two words.  The
+// high word (stride between 8-row groups 1024 B, version 1, swizzle mode 128 B)
+// is the same for every operand here; the low word holds the start address
+// (>> 4, 14 bits) and the leading-byte offset.  Operands are passed as low
+// words (advancing a k-step adds to the address field, which stays below 2^14
+// since shared memory is < 256 KB) and joined to the high word in the MMA, so
+// the issuing thread does 32-bit instead of 64-bit arithmetic per product.
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t addr, uint32_t lbo_bytes) {
+  return ((addr & 0x3FFFFu) >> 4) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
 
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+// D (TMEM) (+)= A (smem) * B (smem)
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t idesc,
                                        uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+      "mov.b64 da, {%1, %5};\n\t"
+      "mov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, {%6, %7, %8, %9}, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+// D (TMEM) (+)= A (TMEM) * B (smem)
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t idesc,
                                        uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+      "mov.b64 db, {%2, %5};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, {%6, %7, %8, %9}, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(acc), "n"(kDescHi), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -405,23 +416,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
       const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
-      // Descriptors are built once; the start-address field (address >> 4,
-      // 14 bits) is advanced by adding offsets (shared memory < 256 KB, so the
-      // field never carries out).
-      const uint64_t dq[2] = {sdesc(base + kQA, 16, 1024), sdesc(base + kQB, 16, 1024)};
-      const uint64_t dk[2] = {sdesc(base + kK0, 16, 1024), sdesc(base + kK1, 16, 1024)};
-      const uint64_t dv[2] = {sdesc(base + kV0, BOX, 1024), sdesc(base + kV1, BOX, 1024)};
+      // Descriptor low words are built once.  K-major Q and K: step k of 16
+      // columns is 32 bytes into a 64-column box, the second box 16 KB on; V
+      // is MN-major: 16 keys are 16 rows of 128 bytes.
+      const uint32_t dq[2] = {sdesc_lo(base + kQA, 16), sdesc_lo(base + kQB, 16)};
+      const uint32_t dk[2] = {sdesc_lo(base + kK0, 16), sdesc_lo(base + kK1, 16)};
+      const uint32_t dv[2] = {sdesc_lo(base + kV0, BOX), sdesc_lo(base + kV1, BOX)};
       auto issue_s = [&](int x, int st) {
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
-          const uint64_t off = (uint64_t)(((k >> 2) * BOX + (k & 3) * 32) >> 4);
+          const uint32_t off = (uint32_t)(((k >> 2) * BOX + (k & 3) * 32) >> 4);
           mma_ss(tS[x], dq[x] + off, dk[st] + off, kIdescS, k > 0);
         }
       };
       auto issue_pv = [&](int x, int st, int j) {
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k)
-          mma_ts(tO[x], tS[x] + 8u * k, dv[st] + (uint64_t)((k * 2048) >> 4), kIdescPV, (j > 0 || k > 0));
+          mma_ts(tO[x], tS[x] + 8u * k, dv[st] + (uint32_t)((k * 2048) >> 4), kIdescPV, (j > 0 || k > 0));
       };
       bool ok = mbar_wait(bar(Q_FULL), 0, P.err, kErrWaitMma) &&
                 mbar_wait(bar(K_FULL0), 0, P.err, kErrWaitMma);
