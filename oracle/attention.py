@@ -18,7 +18,7 @@ What the method computes, from the pages:
 
 The method therefore reaches *exactly* masked softmax attention, so the oracle
 is that definition written out, evaluated in float64 on the exact stored input
-values.  Readings where the pages are silent (each listed in the design doc):
+values.  Readings taken where the pages are silent:
 
 * scale: 1/sqrt(d) unless the caller overrides it;
 * window: sinks are the absolute positions 0..S-1; "recent R" counts the

@@ -6,8 +6,8 @@ Pages: "DuoAttention: Efficient Long-Context LLM Inference with Retrieval and
 Streaming Heads" (hotpaper.ai), abstract (combined with quantisation, 3.3M-token
 Llama-3-8B decoding on one A100) and section "기술적 접근법" (compatible with
 8-bit weights plus a 4-bit KV cache).  The pages give no scheme; the reading
-used (listed in the design doc) is per (token, KV head) group of d channels, K and V
-separately:
+used here is one group per (token, KV head) of d channels, K and V separately,
+asymmetric, with fp16 scale and zero:
 
     mn = min x,  mx = max x                      (exact)
     sc = fp16_rn( fp32(mx - mn) / 15 )           (two fp32 roundings, then fp16)
