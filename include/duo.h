@@ -40,6 +40,11 @@
  *    anything is enqueued; a failed launch returns DUO_ERR_CUDA.  Nothing
  *    throws across this boundary.  Calls on one cache must be ordered by the
  *    caller (one stream, or events).
+ *  - Host threads: a handle's metadata (lengths, block tables, the block
+ *    pool) is updated by the calls without locking, so calls on one cache
+ *    from several host threads must be serialised by the caller.  Different
+ *    caches share nothing on the host (duo_decode_attn_static's device
+ *    scratch is shared; see there).
  *  - Ordering: decode is append-then-attend (duo_append_kv with one token, then
  *    duo_decode_attn; the new token sees itself).  Pre-fill is
  *    attend-then-append (duo_prefill_attn reads the cache as it stood before
