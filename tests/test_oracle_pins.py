@@ -179,6 +179,67 @@ def test_rows_are_probability_vectors():
         np.testing.assert_allclose(ones, 1.0, rtol=0, atol=1e-12)
 
 
+# ---------------------------------------------------------------- invariances
+
+
+def test_streaming_decode_depends_only_on_its_window():
+    """Changing K/V at a position that is neither a sink nor recent leaves a
+    streaming head's output unchanged; changing one inside the window does
+    not (the mask definition, checked without the ring)."""
+    r = _rng(31)
+    n, d, S, R = 40, 8, 3, 5
+    q = r.standard_normal((1, 2, d))
+    k = r.standard_normal((1, n, 2, d))
+    v = r.standard_normal((1, n, 2, d))
+    mask = np.array([0, 1])
+    base = A.decode_reference(q, k, v, mask, S, R)
+    for p in range(n):
+        k2, v2 = k.copy(), v.copy()
+        k2[0, p, 0] += 3.0
+        v2[0, p, 0] -= 2.0
+        got = A.decode_reference(q, k2, v2, mask, S, R)
+        inside = p < S or n - 1 - p < R
+        np.testing.assert_array_equal(got[0, 1], base[0, 1])  # retrieval head untouched
+        if inside:
+            assert np.abs(got[0, 0] - base[0, 0]).max() > 1e-6, p
+        else:
+            np.testing.assert_array_equal(got[0, 0], base[0, 0])
+
+
+def test_value_affine_equivariance():
+    """Softmax weights sum to one: O(q, K, a V + b) = a O(q, K, V) + b, for
+    both kinds of head, at decode and in pre-fill."""
+    r = _rng(32)
+    n, d, S, R, a, b = 23, 8, 2, 4, -1.75, 0.625
+    q = r.standard_normal((1, n, 4, d))
+    k = r.standard_normal((1, n, 2, d))
+    v = r.standard_normal((1, n, 2, d))
+    mask = np.array([1, 0])
+    o = A.prefill_reference(q, k, v, 0, mask, S, R)
+    o2 = A.prefill_reference(q, k, a * v + b, 0, mask, S, R)
+    np.testing.assert_allclose(o2, a * o + b, rtol=0, atol=1e-12)
+    od = A.decode_reference(q[:, -1], k, v, mask, S, R)
+    od2 = A.decode_reference(q[:, -1], k, a * v + b, mask, S, R)
+    np.testing.assert_allclose(od2, a * od + b, rtol=0, atol=1e-12)
+
+
+def test_retrieval_decode_ignores_history_order():
+    """At decode every earlier key is visible to a retrieval head, so
+    reordering the history (K and V together) leaves its output unchanged,
+    while a streaming head, which sees positions, changes."""
+    r = _rng(33)
+    n, d, S, R = 30, 8, 2, 4
+    q = r.standard_normal((1, 4, d))
+    k = r.standard_normal((1, n, 2, d))
+    v = r.standard_normal((1, n, 2, d))
+    mask = np.array([1, 0])
+    perm = np.concatenate([r.permutation(n - 1), [n - 1]])
+    base = A.decode_reference(q, k, v, mask, S, R)
+    got = A.decode_reference(q, k[:, perm], v[:, perm], mask, S, R)
+    np.testing.assert_allclose(got[0, :2], base[0, :2], rtol=0, atol=1e-12)
+    assert np.abs(got[0, 2:] - base[0, 2:]).max() > 1e-6
+
+
 # ---------------------------------------------------------------- golden
 
 
@@ -369,6 +430,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
             test_streaming_bruteforce_tiny(2, 3)
         with pytest.raises(AssertionError):
             test_golden_equal_logits_prefill()
+        with pytest.raises(AssertionError):
+            test_streaming_decode_depends_only_on_its_window()
         monkeypatch.setattr(A, "visible_mask", good_mask)
 
     good_attn = A.masked_attention
@@ -382,6 +445,14 @@ def test_planted_mistakes_are_caught(monkeypatch):
             vv = vv.T
         return good_attn(q, k, vv, mask, scale)
 
+    def unnormalised(q, k, v, mask, scale):
+        # weights exp(s - max) without dividing by their sum
+        s_ = np.where(mask, (np.asarray(q) @ np.asarray(k).T) * scale, -np.inf)
+        return np.exp(s_ - s_.max(axis=1, keepdims=True)) @ np.asarray(v)
+
+    monkeypatch.setattr(A, "masked_attention", unnormalised)
+    with pytest.raises(AssertionError):
+        test_value_affine_equivariance()
     monkeypatch.setattr(A, "masked_attention", no_scale)
     with pytest.raises(AssertionError):
         test_all_retrieval_prefill_equals_causal_sdpa(4, 4, 37, 16)
