@@ -215,6 +215,32 @@ def test_decode_step_fused_append(kind, D, Hq, Hkv):
 
 
 @pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("S,R", [(0, 1), (0, 16), (5, 1), (600, 700)])
+def test_decode_degenerate_windows(kind, D, S, R):
+    """The method's degenerate windows at decode: no sinks, a window of only the
+    current token, sinks only plus the current token, and a window longer than
+    the context (streaming = full attention).  Plain append + decode after a
+    chunked fill, then fused steps that evict from the ring every step."""
+    B, Hq, Hkv, n0, steps = 2, 8, 4, 333, 12
+    total = n0 + steps
+    mask = torch.tensor([1, 0, 0, 1], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, D, kind, total, mask[None], S, R)
+    K = synth.kv_field(91 + S, range(B), range(total), Hkv, D, device="cuda").to(DT[kind])
+    V = synth.kv_field(92 + R, range(B), range(total), Hkv, D, device="cuda").to(DT[kind])
+    Q = synth.kv_field(93, range(B), range(total), Hq, D, device="cuda").to(DT[kind])
+    for p0, p1 in ((0, 100), (100, 101), (101, n0)):
+        cache.append(0, K[:, p0:p1].contiguous(), V[:, p0:p1].contiguous())
+    out = cache.decode(0, Q[:, n0 - 1].contiguous())
+    ref = _oracle(K[:, :n0], V[:, :n0], Q[:, n0 - 1], mask, S, R)
+    assert_parity(out, ref, kind, "S=%d R=%d decode" % (S, R))
+    for t in range(n0, total):
+        out = cache.step(0, Q[:, t].contiguous(), K[:, t].contiguous(), V[:, t].contiguous())
+        ref = _oracle(K[:, :t + 1], V[:, :t + 1], Q[:, t], mask, S, R)
+        assert_parity(out, ref, kind, "S=%d R=%d step t=%d" % (S, R, t))
+    _check_cache_bytes(cache, K, V, mask, S, R)
+
+
+@pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
 def test_reproducible_mode(kind, D):
     """Fixed split shares: repeated decodes of one cache state are bit-identical;
     the default (pooled) mode agrees with them within rounding; both match the
