@@ -50,8 +50,7 @@ def _fill(cache, K, V, chunks):
 
 @pytest.mark.parametrize("B,Hq,Hkv,D", [(1, 8, 2, 128), (2, 4, 4, 64), (1, 8, 8, 128)])
 @pytest.mark.parametrize("n", [1, 3, 70, 333, 2049])
-def test_int4_append_bit_exact_and_decode(B, Hq, Hkv, D, n):
-    S, R = 4, 64
+def test_int4_append_bit_exact_and_decode(B, Hq, Hkv, D, n, S=4, R=64):
     seed = n + D + Hkv
     K, V, q = _inputs(seed, B, n, Hq, Hkv, D)
     mask = seeded_mask(seed, Hkv, max(1, Hkv // 2))
@@ -87,6 +86,14 @@ def test_int4_append_bit_exact_and_decode(B, Hq, Hkv, D, n):
                     np.testing.assert_array_equal(st_sz[b, idx, :S + R].cpu().numpy()[filled], exp[filled])
     kept, full = cache.kv_bytes()
     assert (kept, full) == OC.kv_bytes(mask[None].numpy(), B, n, S, R, D, "int4")
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("S,R", [(0, 1), (5, 1), (0, 7), (600, 700)])
+def test_int4_degenerate_windows(D, S, R):
+    """4-bit cache with the degenerate windows (slot buffers padded to a
+    multiple of 4 rows when S + R is not): codes, scale/zero and decode."""
+    test_int4_append_bit_exact_and_decode(2, 8, 4, D, 333, S=S, R=R)
 
 
 def test_int4_split_counts_agree():
