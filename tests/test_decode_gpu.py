@@ -241,6 +241,30 @@ def test_decode_degenerate_windows(kind, D, S, R):
 
 
 @pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
+def test_batch_beyond_one_launch(kind, D):
+    """130 batch rows: appends, decodes (automatic and forced split counts) and
+    the fused step are issued as launches of at most 128 rows."""
+    B, Hq, Hkv, n, S, R = 130, 4, 2, 45, 3, 8
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, D, kind, n + 4, mask[None], S, R)
+    K = synth.kv_field(71, range(B), range(n + 1), Hkv, D, device="cuda").to(DT[kind])
+    V = synth.kv_field(72, range(B), range(n + 1), Hkv, D, device="cuda").to(DT[kind])
+    Q = synth.kv_field(73, range(B), range(n + 1), Hq, D, device="cuda").to(DT[kind])
+    cache.append(0, K[:, :n - 1].contiguous(), V[:, :n - 1].contiguous())
+    cache.append(0, K[:, n - 1:n].contiguous(), V[:, n - 1:n].contiguous())
+    ref = _oracle(K[:, :n], V[:, :n], Q[:, n - 1], mask, S, R)
+    for splits in (0, 3):
+        cache.set_decode_splits(splits)
+        out = cache.decode(0, Q[:, n - 1].contiguous())
+        assert_parity(out, ref, kind, "130 rows, splits=%d" % splits)
+    cache.set_decode_splits(0)
+    out = cache.step(0, Q[:, n].contiguous(), K[:, n].contiguous(), V[:, n].contiguous())
+    ref = _oracle(K, V, Q[:, n], mask, S, R)
+    assert_parity(out, ref, kind, "130 rows, fused step")
+    _check_cache_bytes(cache, K, V, mask, S, R)
+
+
+@pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
 def test_reproducible_mode(kind, D):
     """Fixed split shares: repeated decodes of one cache state are bit-identical;
     the default (pooled) mode agrees with them within rounding; both match the

@@ -61,6 +61,21 @@ def test_prefill_parity_small(B, Hq, Hkv, S, R, bounds):
         assert_parity(o, ref, "bf16", "chunk [%d,%d) S=%d R=%d" % (c0, c1, S, R))
 
 
+def test_prefill_batch_beyond_one_launch():
+    """130 batch rows: the pre-fill (and the appends between chunks) is issued
+    as launches of at most 128 rows; every row matches the oracle."""
+    B, Hq, Hkv, n, S, R = 130, 4, 2, 300, 4, 64
+    Q, K, V = _prompt(55, B, n, Hq, Hkv)
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, 128, "bf16", n, mask[None], S, R)
+    bounds = [(0, 100), (100, 300)]
+    outs = _run_chunks(cache, Q, K, V, bounds)
+    Kd, Vd = f64(K), f64(V)
+    for (c0, o), (_, c1) in zip(outs, bounds):
+        ref = OA.prefill_reference(f64(Q[:, c0:c1]), Kd, Vd, c0, mask.numpy(), S, R)
+        assert_parity(o, ref, "bf16", "130 rows chunk [%d,%d)" % (c0, c1))
+
+
 def test_prefill_all_heads_one_kind():
     B, Hq, Hkv, n = 1, 4, 2, 600
     for bits in ([1, 1], [0, 0]):
