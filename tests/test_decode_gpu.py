@@ -240,13 +240,15 @@ def test_decode_degenerate_windows(kind, D, S, R):
     _check_cache_bytes(cache, K, V, mask, S, R)
 
 
-@pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
-def test_batch_beyond_one_launch(kind, D):
+@pytest.mark.parametrize("kind,D,paged", [("bf16", 128, False), ("f32", 64, False), ("bf16", 128, True)])
+def test_batch_beyond_one_launch(kind, D, paged):
     """130 batch rows: appends, decodes (automatic and forced split counts) and
-    the fused step are issued as launches of at most 128 rows."""
+    the fused step are issued as launches of at most 128 rows (paged: with
+    each launch's rows reading through their own block tables)."""
     B, Hq, Hkv, n, S, R = 130, 4, 2, 45, 3, 8
     mask = torch.tensor([1, 0], dtype=torch.uint8)
-    cache = DuoCache(1, B, Hq, Hkv, D, kind, n + 4, mask[None], S, R)
+    kw = dict(pool_blocks=B + 3) if paged else {}
+    cache = DuoCache(1, B, Hq, Hkv, D, kind, n + 4, mask[None], S, R, **kw)
     K = synth.kv_field(71, range(B), range(n + 1), Hkv, D, device="cuda").to(DT[kind])
     V = synth.kv_field(72, range(B), range(n + 1), Hkv, D, device="cuda").to(DT[kind])
     Q = synth.kv_field(73, range(B), range(n + 1), Hq, D, device="cuda").to(DT[kind])
@@ -261,7 +263,13 @@ def test_batch_beyond_one_launch(kind, D):
     out = cache.step(0, Q[:, n].contiguous(), K[:, n].contiguous(), V[:, n].contiguous())
     ref = _oracle(K, V, Q[:, n], mask, S, R)
     assert_parity(out, ref, kind, "130 rows, fused step")
-    _check_cache_bytes(cache, K, V, mask, S, R)
+    if paged:
+        for r in (0, 127, 128, 129):  # retrieval rows through the block table
+            got = cache.gather_rows(0, "ret_k", r, n + 1)[0].cpu()
+            want = K[r, :, 0].cpu().contiguous().view(torch.uint8)
+            assert torch.equal(got, want), r
+    else:
+        _check_cache_bytes(cache, K, V, mask, S, R)
 
 
 @pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
