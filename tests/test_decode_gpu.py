@@ -272,6 +272,53 @@ def test_batch_beyond_one_launch(kind, D, paged):
         _check_cache_bytes(cache, K, V, mask, S, R)
 
 
+@pytest.mark.parametrize("kind,D,paged", [("bf16", 128, False), ("f32", 64, False), ("bf16", 128, True)])
+def test_layers_with_different_masks(kind, D, paged):
+    """Three layers with different head masks (mixed, all streaming, all
+    retrieval), filled to different lengths: each layer decodes against the
+    oracle with its own mask and holds its own bytes (paged: the layers'
+    retrieval rows share block ids but not storage)."""
+    B, Hq, Hkv, S, R = 2, 8, 4, 4, 16
+    masks = torch.tensor([[1, 0, 0, 1], [0, 0, 0, 0], [1, 1, 1, 1]], dtype=torch.uint8)
+    lens = [300, 120, 517]
+    kw = dict(pool_blocks=B * 3 + 2) if paged else {}
+    cache = DuoCache(3, B, Hq, Hkv, D, kind, 600, masks, S, R, **kw)
+    data = []
+    for layer, n in enumerate(lens):
+        K = synth.kv_field(100 + layer, range(B), range(n), Hkv, D, device="cuda").to(DT[kind])
+        V = synth.kv_field(110 + layer, range(B), range(n), Hkv, D, device="cuda").to(DT[kind])
+        q = synth.kv_field(120 + layer, range(B), [n - 1], Hq, D, device="cuda")[:, 0].to(DT[kind])
+        data.append((K, V, q))
+    for layer in (2, 0, 1):  # layers are filled in any order
+        K, V, _ = data[layer]
+        half = lens[layer] // 2
+        cache.append(layer, K[:, :half].contiguous(), V[:, :half].contiguous())
+        cache.append(layer, K[:, half:].contiguous(), V[:, half:].contiguous())
+    for layer, n in enumerate(lens):
+        K, V, q = data[layer]
+        assert cache.seq_len(layer) == n
+        out = cache.decode(layer, q)
+        ref = _oracle(K, V, q, masks[layer], S, R)
+        assert_parity(out, ref, kind, "layer %d" % layer)
+        if not paged:
+            torch.cuda.synchronize()
+            lv = cache.layout(layer)
+            rows = {nm: cache.region(layer, nm) for nm in ("ret_k", "str_k")}
+            for h in range(Hkv):
+                idx = lv.packed_index[h]
+                want = K[1, :, h].cpu().contiguous().view(torch.uint8)
+                if masks[layer][h]:
+                    assert torch.equal(rows["ret_k"][1, idx, :n].cpu(), want)
+                else:
+                    exp, filled = OC.expected_streaming_buffer(want.numpy(), S, R)
+                    got = rows["str_k"][1, idx].cpu().numpy()
+                    np.testing.assert_array_equal(got[filled], exp[filled])
+        elif masks[layer].any():
+            got = cache.gather_rows(layer, "ret_k", 1, n)[0].cpu()
+            h0 = int(torch.nonzero(masks[layer])[0])
+            assert torch.equal(got, K[1, :, h0].cpu().contiguous().view(torch.uint8))
+
+
 @pytest.mark.parametrize("kind,D", [("bf16", 128), ("f32", 64)])
 def test_reproducible_mode(kind, D):
     """Fixed split shares: repeated decodes of one cache state are bit-identical;
