@@ -3,11 +3,14 @@
 
 Default workload: Llama-3-8B-shaped GQA decode at 128K context (32 layers,
 32 query / 8 KV heads, head_dim 128, bf16, 50% retrieval KV heads, S=64 sinks +
-R=256 recent), batch 1.  One step = one decode token through all 32 layers:
-append the token's K/V (append/evict kernel) then attend (split-K retrieval +
-streaming + log-sum-exp merge, one launch per layer).  The chunked pre-fill
+R=256 recent), batch 1.  One step = one decode token through all 32 layers,
+one fused launch per layer (``duo_decode_step``): the token's K/V is appended
+(page row / ring slot) and the query attends (split-K retrieval heads,
+streaming heads, log-sum-exp merge by the last split).  The chunked pre-fill
 (32K prompt, 4K chunks, tcgen05 tensor cores) is measured in the same run and
-reported under "prefill".
+reported under "prefill"; ``--extra`` adds the other workloads (batch 4, MHA
+32K, 4-bit 1M, paged mixed lengths, one rank of a sharded sequence, pre-fill on
+a 4-bit cache).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl duo|reference]
 
