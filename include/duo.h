@@ -148,7 +148,8 @@ duo_status duo_cache_create(duo_cache **out, const duo_cache_desc *desc,
  * desc.capacity bounds one row's length.  The allocator runs on the host;
  * new block-table entries are written on the stream before the kernels that
  * need them.  Requires a configuration the tensor-core decode serves (bf16 or
- * 4-bit KV, head_dim 128); pre-fill needs bf16.
+ * 4-bit KV, head_dim 128); pre-fill works on both (a 4-bit cache through the
+ * workspace of duo_prefill_workspace_bytes).
  * Errors: as duo_cache_create; DUO_ERR_ARG for pool_blocks <= 0;
  * DUO_ERR_UNSUPPORTED for other configurations. */
 duo_status duo_cache_create_paged(duo_cache **out, const duo_cache_desc *desc,
