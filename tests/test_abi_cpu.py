@@ -204,3 +204,47 @@ def test_paged_create_rejects(lib):
         assert v.ret_v_sz - v.ret_k_sz == pool * 4
     finally:
         B.duo_cache_destroy(h)
+
+
+def test_binding_signatures_match_the_header():
+    """Every prototype in include/duo.h and the ctypes signature the binding
+    declares for it agree on arity and on each argument's kind (pointer,
+    32-bit or 64-bit integer, float), so the two cannot drift apart."""
+    import ctypes
+    import re
+    from head_split_kv_decode_b200 import binding as Bd
+
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "duo.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b(duo_status|void|const char \*)\s*(duo_\w+)\s*\(([^)]*)\)\s*;", hdr):
+        args = [a.strip() for a in m.group(3).split(",") if a.strip() and a.strip() != "void"]
+        protos[m.group(2)] = args
+
+    def kind_c(decl):
+        if "*" in decl or decl.startswith("duo_stream"):
+            return "ptr"
+        if decl.startswith(("int64_t", "size_t")):
+            return "i64"
+        if decl.startswith("float"):
+            return "f32"
+        if decl.startswith(("int32_t", "int ", "duo_status")):
+            return "i32"
+        raise AssertionError("unknown C type: " + decl)
+
+    def kind_py(t):
+        if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and not isinstance(t._type_, str):
+            return "ptr"
+        if t in (ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint64):
+            return "i64"
+        if t is ctypes.c_float:
+            return "f32"
+        if t in (ctypes.c_int32, ctypes.c_uint32):
+            return "i32"
+        raise AssertionError("unknown ctypes type: %r" % (t,))
+
+    assert set(protos) == set(Bd.SIGNATURES), set(protos) ^ set(Bd.SIGNATURES)
+    for name, (_, argtypes) in Bd.SIGNATURES.items():
+        c_kinds = [kind_c(a) for a in protos[name]]
+        py_kinds = [kind_py(t) for t in argtypes]
+        assert c_kinds == py_kinds, (name, c_kinds, py_kinds)
