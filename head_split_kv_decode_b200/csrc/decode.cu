@@ -227,13 +227,23 @@ __global__ void __launch_bounds__(128) decode_kernel(const __grid_constant__ Dec
     if (tid == 0 && t + STAGES < ntiles) issue(t + STAGES);
   }
   if (failed) {
-    // Let the copies already in flight land before the CTA's shared memory
-    // can be handed to another CTA, then give up without writing outputs.
+    // Let the copies already in flight land before shared memory is reused
+    // below (and before the CTA's shared memory can go to another CTA).
     if (tid == 0)
       for (int tt = t; tt < min(ntiles, t + STAGES); ++tt)
         mbar_wait(smem_u32(&bars[tt % STAGES]), (uint32_t)((tt / STAGES) & 1), P.err,
                   kErrWaitTileLoad);
-    return;
+    __syncthreads();  // every thread saw the failure (the barrier above)
+    // Leave this split empty (weight zero) but still take its merge ticket
+    // below, so that the workspace counters return to zero; the error word
+    // tells the caller the output is not valid.
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) of[g][j] = make_float2(0.f, 0.f);
+    }
   }
 
   decode_finish<T, D, G, NWARPS, NP>(

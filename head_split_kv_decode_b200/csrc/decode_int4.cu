@@ -271,7 +271,18 @@ __global__ void __launch_bounds__(128) decode_int4_kernel(const __grid_constant_
       for (int tt = t; tt < min(ntiles, t + STAGES); ++tt)
         mbar_wait(smem_u32(&bars[tt % STAGES]), (uint32_t)((tt / STAGES) & 1), P.err,
                   kErrWaitTileLoad);
-    return;
+    __syncthreads();  // every thread saw the failure (the barrier above)
+    // Leave this split empty (weight zero) but still take its merge ticket
+    // below, so that the workspace counters return to zero; the error word
+    // tells the caller the output is not valid.
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+      z[g] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NP; ++j) of[g][j] = make_float2(0.f, 0.f);
+    }
   }
   // the zero-point term adds the same amount to every channel
 #pragma unroll

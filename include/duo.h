@@ -178,7 +178,10 @@ duo_status duo_cache_reset(duo_cache *cache);
 duo_status duo_release_rows(duo_cache *cache, const int32_t *rows, int32_t n_rows);
 
 /* Append n_tokens tokens to one layer of every row (each row at its own
- * positions len .. len+n_tokens-1): retrieval heads write page (or block)
+ * positions len .. len+n_tokens-1).  Defined by "What is DuoAttention"
+ * (nav.superapi.store), section "Technical principles of DuoAttention": a
+ * full KV cache for retrieval heads, a fixed-length cache of attention sinks
+ * and recent tokens for streaming heads.  Retrieval heads write page (or block)
  * rows, streaming heads write only the positions that survive the chunk
  * (sinks and the last R positions) into their slots, evicting what was
  * there.  INT4 caches quantise each (token, head) row of head_dim channels
@@ -200,7 +203,10 @@ duo_status duo_append_kv_rows(duo_cache *cache, int32_t layer, const int32_t *ro
 
 /* Single-token decode attention for one layer: in every row, the query at
  * position len-1 (len = that row's length) of every query head attends to its
- * KV head's visible set.  Retrieval heads run split-K flash decoding
+ * KV head's visible set.  Defined by "DuoAttention: Efficient Long-Context
+ * LLM Inference with Retrieval and Streaming Heads" (hotpaper.ai), abstract:
+ * retrieval heads attend over all tokens, streaming heads over the attention
+ * sinks and recent tokens only.  Retrieval heads run split-K flash decoding
  * (per-split log-sum-exp partials in the workspace, merged by the last split
  * of each head; the tensor-core decode gives each row a split count in
  * proportion to its length); streaming heads run one pass over their slot
@@ -223,7 +229,10 @@ duo_status duo_decode_attn_rows(duo_cache *cache, int32_t layer, const int32_t *
                                 size_t workspace_bytes, duo_stream stream);
 
 /* One decode step for one layer in a single launch where the kernels allow
- * it: append each row's new token (k_new, v_new: [batch, n_kv_heads,
+ * it (the two operations of the abstract of "DuoAttention: Efficient
+ * Long-Context LLM Inference with Retrieval and Streaming Heads"
+ * (hotpaper.ai) and of section "Technical principles of DuoAttention" of
+ * "What is DuoAttention" (nav.superapi.store), in one pass): append each row's new token (k_new, v_new: [batch, n_kv_heads,
  * head_dim]) at position len and attend with q at that position, exactly as
  * duo_append_kv(.., 1, ..) followed by duo_decode_attn.  The warp whose key
  * tile holds the new token's row takes its K/V from the inputs and writes
@@ -245,8 +254,10 @@ duo_status duo_decode_step_rows(duo_cache *cache, int32_t layer, const int32_t *
                                 duo_stream stream);
 
 /* Decode attention like duo_decode_attn, but with no workspace argument and
- * no allocation of any kind: the split-K scratch (partial outputs, log-sum-exp
- * values, merge tickets) lives in a fixed array inside the library,
+ * no device memory allocation (no cudaMalloc, cudaFree or allocating library
+ * routine; the host-side planning uses a few small heap buffers, like every
+ * other call): the split-K scratch (partial outputs, log-sum-exp values,
+ * merge tickets) lives in a fixed array inside the library,
  * DUO_DECODE_STATIC_SCRATCH_BYTES in size, that every GPU loading the library
  * holds until the process exits.  The paper has no counterpart to this call.
  * It is for callers that cannot call cudaMalloc (or any allocator) to get a
@@ -271,7 +282,11 @@ duo_status duo_decode_attn_static(duo_cache *cache, int32_t layer, const void *q
 
 /* Chunked pre-fill attention for one layer: in every row, C queries at
  * positions len .. len+C-1 attend to the cache as it stands (positions below
- * len) plus the chunk's own k/v: causal for retrieval heads, Lambda mask
+ * len) plus the chunk's own k/v.  Defined by "DuoAttention: Efficient
+ * Long-Context LLM Inference with Retrieval and Streaming Heads"
+ * (hotpaper.ai), abstract (the split applies to pre-filling as well as
+ * decoding), and "韩松团队长上下文LLM推理高效框架" (cn.bg3.co), section "研究背景"
+ * (pre-fill cost quadratic in the context): causal for retrieval heads, Lambda mask
  * (sinks plus the R most recent positions) for streaming heads, with key tiles
  * outside the Lambda band skipped.  Runs on the sm_100a tensor cores
  * (tcgen05.mma, accumulators in tensor memory, operands loaded by TMA).  Does
@@ -396,7 +411,10 @@ duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
 
 /* Read and clear the device-side error word that bounded in-kernel waits set
  * when they give up.  Synchronises the device.  Returns DUO_ERR_TIMEOUT if it
- * was set, DUO_OK otherwise; *code (may be NULL) receives the raw word. */
+ * was set, DUO_OK otherwise; *code (may be NULL) receives the raw word.
+ * The outputs of a call whose wait gave up are undefined.  A decode CTA that
+ * gives up still leaves an empty partial and takes its merge ticket, so the
+ * decode workspace is left with its counters at zero and stays usable. */
 duo_status duo_poll_device_error(int32_t *code);
 
 const char *duo_status_string(duo_status status);

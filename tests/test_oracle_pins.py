@@ -307,6 +307,40 @@ def test_golden_ring_and_bytes():
     assert (kept, full) == (b["expected_kept"], b["expected_full"])
 
 
+def _position_rows(n, d=2):
+    """Row p = [p, 100 + p, ...]: every position's row is distinct."""
+    return np.array([[p + 100 * c for c in range(d)] for p in range(n)], dtype=np.int64)
+
+
+def test_expected_streaming_buffer_golden_ring():
+    """The golden ring case (S=2, R=3, n=10) written out by hand: after ten
+    appends slot s holds position expected_held[s], so buffer row s must be
+    position expected_held[s]'s row."""
+    c = _golden()["ring_slots"]
+    S, R, n = c["S"], c["R"], c["n"]
+    rows = _position_rows(n)
+    buf, filled = C.expected_streaming_buffer(rows, S, R)
+    hand = np.array([[0, 100], [1, 101], [8, 108], [9, 109], [7, 107]], dtype=np.int64)
+    assert [int(c["expected_held"][str(s)]) for s in range(S + R)] == [0, 1, 8, 9, 7]
+    np.testing.assert_array_equal(buf, hand)
+    assert filled.all()
+
+
+def test_expected_streaming_buffer_partial_and_no_sinks():
+    """Hand-built buffers where the ring has not wrapped yet (unwritten slots
+    stay zero and are marked unfilled), and with no sinks (S=0)."""
+    buf, filled = C.expected_streaming_buffer(_position_rows(3), 2, 3)
+    np.testing.assert_array_equal(buf, [[0, 100], [1, 101], [2, 102], [0, 0], [0, 0]])
+    assert filled.tolist() == [True, True, True, False, False]
+    # S=0, R=3, n=7: positions 6, 4, 5 sit in slots 0, 1, 2 (p mod 3)
+    buf, filled = C.expected_streaming_buffer(_position_rows(7), 0, 3)
+    np.testing.assert_array_equal(buf, [[6, 106], [4, 104], [5, 105]])
+    assert filled.all()
+    # R=1: only the newest position after the sinks survives
+    buf, filled = C.expected_streaming_buffer(_position_rows(9), 4, 1)
+    np.testing.assert_array_equal(buf[:, 0], [0, 1, 2, 3, 8])
+
+
 # ---------------------------------------------------------------- ring + bytes
 
 
@@ -472,3 +506,22 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(Q, "quantize_int4", floor_not_rint)
     with pytest.raises(AssertionError):
         test_golden_int4()
+    monkeypatch.setattr(Q, "quantize_int4", good_q)
+
+    good_buf = C.expected_streaming_buffer
+
+    def indexed_by_position(k_head, S, R):
+        # a slip: row p stored at row p mod W instead of at its ring slot
+        k_head = np.asarray(k_head)
+        W = S + R
+        buf = np.zeros((W,) + k_head.shape[1:], dtype=k_head.dtype)
+        filled = np.zeros(W, dtype=bool)
+        for p in range(k_head.shape[0]):
+            buf[p % W] = k_head[p]
+            filled[p % W] = True
+        return buf, filled
+
+    monkeypatch.setattr(C, "expected_streaming_buffer", indexed_by_position)
+    with pytest.raises(AssertionError):
+        test_expected_streaming_buffer_golden_ring()
+    monkeypatch.setattr(C, "expected_streaming_buffer", good_buf)
