@@ -8,9 +8,11 @@ one fused launch per layer (``duo_decode_step``): the token's K/V is appended
 (page row / ring slot) and the query attends (split-K retrieval heads,
 streaming heads, log-sum-exp merge by the last split).  The chunked pre-fill
 (32K prompt, 4K chunks, tcgen05 tensor cores) is measured in the same run and
-reported under "prefill"; ``--extra`` adds the other workloads (batch 4, MHA
-32K, 4-bit 1M, paged mixed lengths, one rank of a sharded sequence, pre-fill on
-a 4-bit cache).
+reported under "prefill", and the other decode configurations under "configs"
+(the same step at batch 4; Llama-2-7B-shaped MHA at 32K; 4-bit KV at 1M tokens,
+one layer; a paged batch of 8 sequences of mixed lengths), each with its own
+roofline and clock samples.  ``--extra`` adds one rank of a sequence-sharded
+decode and pre-fill on a 4-bit cache.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl duo|reference]
 
@@ -149,29 +151,42 @@ class ClockSampler:
 
 
 # DRAM traffic of one fused decode launch (dram__bytes_read.sum +
-# dram__bytes_write.sum) from an ncu capture of one layer of the 128K batch-1
-# GQA workload (4 retrieval + 4 streaming KV heads, context 131076), and that
-# launch's algorithmic bytes.  The ratio scales to the benchmark's launches; it
-# is reported only while the kernel's sources hash as they did when the
-# counters were taken (otherwise traffic is null).
+# dram__bytes_write.sum) from an ncu capture of one layer of a workload, and
+# that launch's algorithmic bytes, per cache type: bf16 from the 128K batch-1
+# GQA workload (4 retrieval + 4 streaming KV heads, context 131076); int4 from
+# the 1M GQA workload (2 retrieval + 6 streaming KV heads).  The ratio scales
+# to the benchmark's launches; it is reported only while the kernel's sources
+# hash as they did when the counters were taken (otherwise traffic is null).
+DECODE_TRAFFIC_SOURCES = ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h",
+                          "quant_int4.cuh")
 DECODE_TRAFFIC = {
-    "sources": ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h"),
-    "sha256": "abeb3a94fbd790f3cb6f27832eef02e415b99b53ec0fbd1e65e439171fe58b1c",
-    "dram_bytes": 269781760 + 4422400,
-    "algorithmic_bytes": 269120512,
+    "bf16": {"sha256": None, "dram_bytes": None, "algorithmic_bytes": None},
+    "int4": {"sha256": None, "dram_bytes": None, "algorithmic_bytes": None},
 }
 
 
-def decode_traffic(bytes_per_launch):
+def decode_traffic(kv_dtype, bytes_per_launch):
     """ncu DRAM bytes per launch scaled to this launch size, or None if the
-    kernel changed since the capture."""
+    kernel changed since the capture (or none was taken)."""
+    ref = DECODE_TRAFFIC.get(kv_dtype)
+    if not ref or ref["sha256"] is None:
+        return None
     h = hashlib.sha256()
-    for name in DECODE_TRAFFIC["sources"]:
+    for name in DECODE_TRAFFIC_SOURCES:
         with open(os.path.join(ROOT, "head_split_kv_decode_b200", "csrc", name), "rb") as f:
             h.update(f.read())
-    if h.hexdigest() != DECODE_TRAFFIC["sha256"]:
+    if h.hexdigest() != ref["sha256"]:
         return None
-    return DECODE_TRAFFIC["dram_bytes"] / DECODE_TRAFFIC["algorithmic_bytes"] * bytes_per_launch
+    return ref["dram_bytes"] / ref["algorithmic_bytes"] * bytes_per_launch
+
+
+def hbm_roofline(achieved_gbs, avg_launch_ms, bytes_per_launch, kernel, peaks, peak_kind,
+                 traffic=None):
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
+            "frac": achieved_gbs / peak, "traffic": traffic, "kernel": kernel,
+            "avg_launch_ms": avg_launch_ms, "bytes_per_launch": bytes_per_launch,
+            "peak_kind": peak_kind}
 
 
 def decode_bytes_per_layer(w, batch, n, n_ret, n_str):
@@ -240,9 +255,9 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K * w.layers)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K * w.layers)]
 
-    # bf16 head_dim-128 caches decode each layer in one fused launch
+    # bf16 and 4-bit head_dim-128 caches decode each layer in one fused launch
     # (duo_decode_step: append + attend); other caches append, then attend.
-    fused = w.kv_dtype == "bf16" and w.head_dim == 128
+    fused = w.kv_dtype in ("bf16", "int4") and w.head_dim == 128
 
     # The fused path's timed region holds nothing but its decode launches, back
     # to back (programmatic dependent launch overlaps each one's set-up with
@@ -355,8 +370,9 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
         "e2e_value": aggregate_rate(step_bytes, world, K, e2e_ms),
         "h2d": h2d, "d2h": d2h,
         "step_bytes": step_bytes,
-        "kernel": {"name": "decode_mma_kernel (fused append + attention)" if fused else
-                   "decode_mma_kernel", "avg_ms": avg_kern_ms, "launches": len(kern_ms),
+        "kernel": {"name": ("decode_mma_kernel %s (fused append + attention)" if fused else
+                            "decode_mma_kernel %s") % w.kv_dtype,
+                   "avg_ms": avg_kern_ms, "launches": len(kern_ms),
                    "bytes_per_launch": avg_launch_bytes, "achieved_gbs": achieved},
         "splits": splits,
         "fill_s": fill_s,
@@ -364,13 +380,17 @@ def run_decode(args, w, batch, rank, world, peaks, peak_kind, clock_gpu):
         "context": n_first,
         "gpu_launches": K * w.layers * (1 if fused else 2),
         "fused": fused,
+        "roofline": hbm_roofline(achieved, avg_kern_ms, avg_launch_bytes,
+                                 ("decode_mma_kernel %s (fused append + attention)" if fused else
+                                  "decode_mma_kernel %s") % w.kv_dtype, peaks, peak_kind,
+                                 decode_traffic(w.kv_dtype, avg_launch_bytes) if fused else None),
     }
     del cache
     torch.cuda.empty_cache()
     return res
 
 
-def run_paged_mixed(args, w, rank, world, peaks):
+def run_paged_mixed(args, w, rank, world, peaks, peak_kind, clock_gpu):
     """Decode of a mixed-length batch on the paged layout: every row (one
     sequence, w.row_lengths tokens of context) takes one fused step per layer,
     all rows in one launch, each at its own position."""
@@ -426,11 +446,13 @@ def run_paged_mixed(args, w, rank, world, peaks):
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(K):
-        step(Wm + i)
-    e1.record()
-    torch.cuda.synchronize()
+    with ClockSampler(clock_gpu) as clk:
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(K):
+            step(Wm + i)
+        e1.record()
+        torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     ms = max_over_ranks([ms], world, "cuda")[0]
     if B.duo_poll_device_error() != 0:
@@ -452,6 +474,11 @@ def run_paged_mixed(args, w, rank, world, peaks):
            "decode_splits": cache.decode_splits(0), "fill_s": fill_s}
     res["kernel_achieved_gbs"] = res["bytes_per_launch"] / (res["kernel_avg_launch_ms"] * 1e-3) / 1e9
     res["frac"] = res["kernel_achieved_gbs"] / peaks["hbm_gbs"]
+    res["roofline"] = hbm_roofline(res["kernel_achieved_gbs"], res["kernel_avg_launch_ms"],
+                                   res["bytes_per_launch"],
+                                   "decode_mma_kernel bf16 paged (fused append + attention)",
+                                   peaks, peak_kind)
+    res["clocks"] = clk.summary()
     del cache
     torch.cuda.empty_cache()
     return res
@@ -734,7 +761,11 @@ def main(argv=None):
                          "profiling; 0 = all layers)")
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--extra", action="store_true",
-                    help="also time batch 4 at 128K and the MHA 32K workload")
+                    help="also time one rank of a sequence-sharded decode and pre-fill on a "
+                         "4-bit cache")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline workload (and pre-fill), not the other "
+                         "decode configurations")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -764,25 +795,38 @@ def main(argv=None):
             clock_gpu = int(ids[local])
 
     res = run_decode(args, w, args.batch, rank, world, peaks, peak_kind, clock_gpu)
+
+    def decode_entry(wx, rx, note=None):
+        e = {"workload": wx.name, "batch": rx.get("batch", 1), "context": rx["context"],
+             "layers": wx.layers, "value": rx["value"], "unit": "GB/s",
+             "ms_per_step": rx["ms_per_step"], "roofline": rx["roofline"],
+             "clocks": rx["clocks"], "decode_splits": rx["splits"],
+             "gpu_launches": rx["gpu_launches"]}
+        if note:
+            e["note"] = note
+        return e
+
+    # The other decode configurations, each timed like the headline (the
+    # same step function, its own clock samples and roofline).
+    configs = {}
+    if not args.headline_only and not args.layers:
+        r4 = run_decode(args, w, 4, rank, world, peaks, peak_kind, clock_gpu)
+        r4["batch"] = 4
+        configs["llama3_8b_gqa_128k_b4"] = decode_entry(w, r4)
+        wm = synth.WORKLOADS["llama2_7b_mha_32k"]
+        configs["llama2_7b_mha_32k"] = decode_entry(
+            wm, run_decode(args, wm, 1, rank, world, peaks, peak_kind, clock_gpu))
+        wq = dataclasses.replace(synth.WORKLOADS["llama3_8b_gqa_int4_1m"], layers=1)
+        configs["llama3_8b_gqa_int4_1m"] = decode_entry(
+            wq, run_decode(args, wq, 1, rank, world, peaks, peak_kind, clock_gpu),
+            note="one layer of the 32-layer workload (layer 0's head mask), its 1M-token "
+                 "4-bit cache re-read every step (285 MB per launch, larger than L2); "
+                 "a 32-layer step is 32 such launches")
+        configs["llama3_8b_gqa_paged_mixed"] = run_paged_mixed(
+            args, synth.WORKLOADS["llama3_8b_gqa_paged_mixed"], rank, world, peaks, peak_kind,
+            clock_gpu)
     extra = {}
     if args.extra:
-        r4 = run_decode(args, w, 4, rank, world, peaks, peak_kind, clock_gpu)
-        extra["batch4"] = {"value": r4["value"], "unit": "GB/s", "ms_per_step": r4["ms_per_step"],
-                           "kernel_avg_launch_ms": r4["kernel"]["avg_ms"],
-                           "kernel_achieved_gbs": r4["kernel"]["achieved_gbs"],
-                           "frac": r4["kernel"]["achieved_gbs"] / peaks["hbm_gbs"],
-                           "decode_splits": r4["splits"], "gpu_launches": r4["gpu_launches"]}
-        for key in ("llama2_7b_mha_32k", "llama3_8b_gqa_int4_1m"):
-            wx = synth.WORKLOADS[key]
-            rx = run_decode(args, wx, 1, rank, world, peaks, peak_kind, clock_gpu)
-            extra[key] = {"workload": wx.name, "value": rx["value"], "unit": "GB/s",
-                          "ms_per_step": rx["ms_per_step"],
-                          "kernel_avg_launch_ms": rx["kernel"]["avg_ms"],
-                          "kernel_achieved_gbs": rx["kernel"]["achieved_gbs"],
-                          "frac": rx["kernel"]["achieved_gbs"] / peaks["hbm_gbs"],
-                          "decode_splits": rx["splits"], "gpu_launches": rx["gpu_launches"]}
-        extra["llama3_8b_gqa_paged_mixed"] = run_paged_mixed(
-            args, synth.WORKLOADS["llama3_8b_gqa_paged_mixed"], rank, world, peaks)
         extra["sequence_sharded_1m_rank0_of_8"] = run_shard_rank(args, w, 8, rank, peaks)
         pq = run_prefill(args, synth.WORKLOADS["llama3_8b_gqa_prefill_32k"], rank, world, peaks,
                          kv_dtype="int4")
@@ -803,7 +847,6 @@ def main(argv=None):
         if world > 1:
             torch.distributed.destroy_process_group()
         return 0
-    peak = peaks["hbm_gbs"]
     kern = res["kernel"]
     line = {
         "metric": METRIC,
@@ -820,17 +863,14 @@ def main(argv=None):
         "data": "synthetic",
         "config": workload_config(w, args.batch, world),
         "pct_of_8tbs": 100.0 * res["value"] / world / 8000.0,
-        "roofline": {"bound": "hbm", "achieved": kern["achieved_gbs"], "peak": peak,
-                     "unit": "GB/s", "frac": kern["achieved_gbs"] / peak,
-                     "traffic": decode_traffic(kern["bytes_per_launch"]) if res["fused"] else None,
-                     "kernel": kern["name"], "avg_launch_ms": kern["avg_ms"],
-                     "bytes_per_launch": kern["bytes_per_launch"], "peak_kind": peak_kind},
+        "roofline": res["roofline"],
         "e2e": {"value": res["e2e_value"], "unit": "GB/s", "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": res["gpu_launches"] + (prefill or {}).get("gpu_launches", 0),
         "clocks": res["clocks"],
         "decode_splits": res["splits"],
         "prefill": prefill,
+        "configs": configs,
     }
     line.update(extra)
     if world == 1 and not args.no_cpu_baseline:

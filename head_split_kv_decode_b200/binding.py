@@ -100,6 +100,8 @@ SIGNATURES = {
     "duo_layout_info": (_I32, [_P, _I32, ctypes.POINTER(duo_layout_view)]),
     "duo_set_decode_splits": (_I32, [_P, _I32]),
     "duo_set_decode_reproducible": (_I32, [_P, _I32]),
+    "duo_set_decode_output": (_I32, [_P, _I32]),
+    "duo_test_stall_next_prefill": (_I32, [_P, _I64]),
     "duo_decode_splits": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "duo_poll_device_error": (_I32, [ctypes.POINTER(_I32)]),
     "duo_status_string": (ctypes.c_char_p, [_I32]),
@@ -300,6 +302,17 @@ def duo_layout_info(handle, layer):
 
 def duo_set_decode_splits(handle, splits):
     _check(lib().duo_set_decode_splits(handle, splits), "duo_set_decode_splits")
+
+
+def duo_test_stall_next_prefill(handle, wait_ns):
+    """Testing hook: the next pre-fill loads nothing and its waits give up
+    after wait_ns (the timeout path, without any fault)."""
+    _check(lib().duo_test_stall_next_prefill(handle, int(wait_ns)), "duo_test_stall_next_prefill")
+
+
+def duo_set_decode_output(handle, dtype):
+    """dtype: "f32" or "bf16" (the element type of decode outputs)."""
+    _check(lib().duo_set_decode_output(handle, KV_DTYPES[dtype]), "duo_set_decode_output")
 
 
 def duo_set_decode_reproducible(handle, on):

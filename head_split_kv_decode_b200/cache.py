@@ -51,6 +51,7 @@ class DuoCache:
         self.n_q_heads, self.n_kv_heads, self.head_dim = n_q_heads, n_kv_heads, head_dim
         self.kv_dtype, self.capacity, self.S, self.R = kv_dtype, capacity, S, R
         self.io_dtype = _TORCH_DTYPE[kv_dtype]
+        self.out_dtype = self.io_dtype  # decode outputs (see set_decode_output)
         self.device = torch.device(device)
         if self.device.type == "cuda" and self.device.index is None:
             self.device = torch.device("cuda", torch.cuda.current_device())
@@ -101,8 +102,8 @@ class DuoCache:
         shape = (self.batch, self.n_q_heads, self.head_dim)
         self._check(q, shape, "q")
         if out is None:
-            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
-        self._check(out, shape, "out")
+            out = torch.empty(shape, dtype=self.out_dtype, device=q.device)
+        self._check(out, shape, "out", self.out_dtype)
         B.duo_decode_attn(self.handle, layer, q.data_ptr(), out.data_ptr(), float(scale),
                           self.ws_ptr, self.ws_bytes, _stream_handle(stream, self.device))
         return out
@@ -116,8 +117,8 @@ class DuoCache:
         self._check(k_new, kv_shape, "k_new")
         self._check(v_new, kv_shape, "v_new")
         if out is None:
-            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
-        self._check(out, shape, "out")
+            out = torch.empty(shape, dtype=self.out_dtype, device=q.device)
+        self._check(out, shape, "out", self.out_dtype)
         B.duo_decode_step(self.handle, layer, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
                           out.data_ptr(), float(scale), self.ws_ptr, self.ws_bytes,
                           _stream_handle(stream, self.device))
@@ -161,8 +162,8 @@ class DuoCache:
         shape = (len(rows), self.n_q_heads, self.head_dim)
         self._check(q, shape, "q")
         if out is None:
-            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
-        self._check(out, shape, "out")
+            out = torch.empty(shape, dtype=self.out_dtype, device=q.device)
+        self._check(out, shape, "out", self.out_dtype)
         B.duo_decode_attn_rows(self.handle, layer, rows, q.data_ptr(), out.data_ptr(), float(scale),
                                self.ws_ptr, self.ws_bytes, _stream_handle(stream, self.device))
         return out
@@ -176,8 +177,8 @@ class DuoCache:
         self._check(k_new, kv_shape, "k_new")
         self._check(v_new, kv_shape, "v_new")
         if out is None:
-            out = torch.empty(shape, dtype=self.io_dtype, device=q.device)
-        self._check(out, shape, "out")
+            out = torch.empty(shape, dtype=self.out_dtype, device=q.device)
+        self._check(out, shape, "out", self.out_dtype)
         B.duo_decode_step_rows(self.handle, layer, rows, q.data_ptr(), k_new.data_ptr(),
                                v_new.data_ptr(), out.data_ptr(), float(scale), self.ws_ptr,
                                self.ws_bytes, _stream_handle(stream, self.device))
@@ -245,6 +246,13 @@ class DuoCache:
 
     def set_decode_splits(self, splits):
         B.duo_set_decode_splits(self.handle, splits)
+
+    def set_decode_output(self, dtype):
+        """Element type of decode outputs: torch.float32 or torch.bfloat16
+        (bf16 and 4-bit caches; an fp32 cache always outputs float32)."""
+        name = {torch.float32: "f32", torch.bfloat16: "bf16"}[dtype]
+        B.duo_set_decode_output(self.handle, name)
+        self.out_dtype = dtype
 
     def set_decode_reproducible(self, on=True):
         """Fixed key shares per decode split: bit-identical repeated calls."""

@@ -11,6 +11,7 @@
 // survive the chunk: p < S (sinks) and the last R positions.  Those land in
 // distinct slots, so the result equals appending token by token.
 #include "common.cuh"
+#include "quant_int4.cuh"
 
 namespace duo {
 
@@ -52,10 +53,8 @@ __global__ void append_kernel(const __grid_constant__ AppendParams a, int row_by
 }
 
 // INT4: one warp per (token, KV head, K or V) row of D bf16 channels.  Lane l
-// owns channels [l*CPL, l*CPL + CPL).  The encoder performs, in this order,
-// correctly rounded fp32 operations:
-//   span = mx - mn; sc = fp16(span / 15); zp = fp16(mn);
-//   u = clamp(rint((x - zp) / sc), 0, 15), u = 0 when sc == 0.
+// owns channels [l*CPL, l*CPL + CPL); quantize_row_int4 performs the encoder's
+// correctly rounded fp32 operations.
 template <int D>
 __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
   constexpr int CPL = D / 32;
@@ -91,36 +90,15 @@ __global__ void append_int4_kernel(const __grid_constant__ AppendParams a) {
     const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(which ? a.v : a.k) +
                                (((int64_t)lr * a.n_tok + t) * a.Hkv + h) * D + lane * CPL;
     float x[CPL];
-    float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      x[j] = __bfloat162float(src[j]);
-      mn = fminf(mn, x[j]);
-      mx = fmaxf(mx, x[j]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    const __half sch = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
-    const __half zph = __float2half_rn(mn);
-    const float scf = __half2float(sch);
-    const float zpf = __half2float(zph);
-    uint32_t u[CPL];
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-      float q = 0.0f;
-      if (scf != 0.0f) q = fminf(15.0f, fmaxf(0.0f, rintf(__fdiv_rn(__fsub_rn(x[j], zpf), scf))));
-      u[j] = (uint32_t)q;
-    }
+    for (int j = 0; j < CPL; ++j) x[j] = __bfloat162float(src[j]);
+    __half sch, zph;
+    const uint32_t packed = quantize_row_int4<CPL>(x, &sch, &zph);
     uint8_t *dst = codes + row * (D / 2) + lane * (CPL / 2);
-    if (CPL == 4) {
-      const uint16_t packed = (uint16_t)(u[0] | (u[1] << 4) | (u[2] << 8) | (u[3] << 12));
-      *reinterpret_cast<uint16_t *>(dst) = packed;
-    } else {
-      *dst = (uint8_t)(u[0] | (u[1] << 4));
-    }
+    if (CPL == 4)
+      *reinterpret_cast<uint16_t *>(dst) = (uint16_t)packed;
+    else
+      *dst = (uint8_t)packed;
     if (lane == 0) {
       __half2 pair;
       pair.x = sch;

@@ -23,7 +23,11 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
                                                     int64_t unit, int64_t part0, int nsplit,
                                                     int split) {
   constexpr float kLn2 = 0.6931471805599453f;  // log-sum-exps leave in natural log
-  T *out = reinterpret_cast<T *>(P.out) + out_row * D;
+  // output element i of this head's rows, as T or (P.out_f32) as float
+  auto put = [&](int i, float v) {
+    if (P.out_f32) reinterpret_cast<float *>(P.out)[out_row * D + i] = v;
+    else store_out(reinterpret_cast<T *>(P.out) + out_row * D + i, v);
+  };
   constexpr int NT = NWARPS * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int &s_last = *s_last_p;
@@ -53,7 +57,7 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
       P.part_o[(out_row + g) * D + c] = empty ? 0.f : O / L;
       if (c == 0) P.part_lse[out_row + g] = empty ? -INFINITY : (M + fast_log2(L)) * kLn2;
     } else if (direct) {
-      store_out(out + g * D + c, O / L);
+      put(g * D + c, O / L);
     } else {
       // a split whose CTA claimed no keys leaves weight zero (lse -inf)
       const bool empty = L == 0.f;
@@ -168,7 +172,7 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
       P.part_o[(out_row + g) * D + c] = num / s_den[g];
       if (c == 0) P.part_lse[out_row + g] = (s_mx[g] + fast_log2(s_den[g])) * kLn2;
     } else {
-      store_out(out + g * D + c, num / s_den[g]);
+      put(g * D + c, num / s_den[g]);
     }
   }
   if (tid == 0) {  // leave the ticket (and chunk counter) ready for the next call

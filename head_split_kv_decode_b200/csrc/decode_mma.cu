@@ -1,6 +1,6 @@
 // Single-token decode attention with warp-level tensor-core MMAs
-// (mma.sync m16n8k16, bf16 in, fp32 accumulate), for head_dim 128 and a bf16
-// or 4-bit KV cache.
+// (mma.sync m16n8k16, fp32 accumulate), for head_dim 128 and a bf16 or 4-bit
+// KV cache.
 //
 // Same work split as the CUDA-core decode (split-K over retrieval pages, one
 // CTA per streaming slot buffer, last split merges); what changes is the inner
@@ -18,15 +18,27 @@
 // loaded straight from global memory into registers; nothing is staged in
 // shared memory except the final cross-warp combine.
 //
-// 4-bit cache: a nibble u becomes the bf16 128 + u by masking it under the bf16
-// pattern of 128 and is then reduced by 128 (exact), and the per-token scale
-// and zero are applied outside the products: s = sc*(q.u) + zp*sum(q),
-// sum p*v_hat = sum (p*sc)*u + (sum p*zp).
+// 4-bit cache (f16 operands): a nibble masked into the low bits of a 16-bit
+// half, all other bits zero, is the f16 subnormal u * 2^-24 exactly, and one
+// at bits 4..7 is 16u * 2^-24; so one AND per register turns packed codes into
+// MMA operands, with no offset to remove.  The factor 16 is taken out of the
+// query (K side, q/16 on those k-slots) or out of the output channel (V
+// side), both exact.  Scale and zero are applied outside the products:
+//   s = sc * (q . u) + zp * sum(q),   sum p*x_hat = sum (p*sc) * u + sum p*zp.
+// p*sc enters the V product as an f16 pair, high part plus residual (22
+// significant bits; one f16 alone, 11 bits, would leave up to 2^-11 of a V
+// row's range in the output), relative to a reference m - f: f is a
+// power-of-two headroom chosen from the largest V scale seen, so that
+// p*sc < 2^15 whatever the data (f16 overflows at 65504); lowering f rescales
+// the state exactly.  With the fused step the warp that owns the new token
+// quantises it (the append kernel's encoder), writes it to the cache and
+// attends to it from shared memory.
 //
 // Pages: "DuoAttention: Efficient Long-Context LLM Inference with Retrieval and
 // Streaming Heads" (hotpaper.ai), abstract and section "기술적 접근법".
 #include "common.cuh"
 #include "decode_finish.cuh"
+#include "quant_int4.cuh"
 
 namespace duo {
 
@@ -35,18 +47,35 @@ namespace dm {
 constexpr int D = 128;
 constexpr int NWARPS = 16;
 // Key groups of 16 per warp iteration: the 4-bit rows are 4x smaller, so a
-// warp takes two groups to keep as many bytes in flight as the bf16 path.
+// warp takes two groups to keep as many bytes in flight as the bf16 path
+// (measured: one group plus bulk L2 prefetches of the warp's later tiles is
+// slower than two groups in registers).
 template <bool Q4>
 struct Keys {
   static constexpr int KG = Q4 ? 2 : 1;
   static constexpr int STEP = NWARPS * 16 * KG;  // keys per CTA iteration
 };
 
+// 4-bit codes as f16 subnormals: masks of the nibbles at bits 0..3 (value
+// u * 2^-24) and 4..7 (16u * 2^-24) of both 16-bit halves.
+constexpr uint32_t kNib0 = 0x000F000Fu, kNib1 = 0x00F000F0u;
+constexpr float kTwo24 = 16777216.f, kTwo20 = 1048576.f;
+
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
                                          uint32_t b1) {
   // rows g+8 of A are zero (a1 = a3 = 0)
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                             uint32_t b1) {
+  // f16 operands; rows g+8 of A are zero
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
@@ -71,6 +100,20 @@ __device__ __forceinline__ uint2 ldg64(const void *p) {
   return v;
 }
 
+// Loads of the 4-bit tile: read-only global memory, or (GEN) any address
+// space through a generic pointer (the new token staged in shared memory).
+template <bool GEN>
+__device__ __forceinline__ uint4 ld16(const uint8_t *p) {
+  if constexpr (GEN) return *reinterpret_cast<const uint4 *>(p);
+  else return ldg128(p);
+}
+
+template <bool GEN>
+__device__ __forceinline__ uint2 ld8(const uint8_t *p) {
+  if constexpr (GEN) return *reinterpret_cast<const uint2 *>(p);
+  else return ldg64(p);
+}
+
 // Fetch [ptr, ptr + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void *ptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
@@ -81,12 +124,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Two 4-bit codes u (at bit s and bit s+16 of x) -> bf16x2 of 128 + u (exact):
-// the code is masked under the bit pattern of 128.0, whose mantissa is zero.
-// The offset of 128 is removed after the products (see the callers).
-__device__ __forceinline__ uint32_t nib2(uint32_t x, int s) {
-  return ((x >> s) & 0x000F000Fu) | 0x43004300u;
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
 }
+
+__device__ __forceinline__ float2 half2_bits_to_f2(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+}
+
+// 2^e for an integer e in [-126, 127], exactly.
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
 
 __device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                               uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -97,10 +145,28 @@ __device__ __forceinline__ void mma16816_full(float (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma16816_full_f16(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3, uint32_t b0,
+                                                  uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 template <bool Q4, int G>
 __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid_constant__ DecodeParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_last;
+  // 4-bit fused step: the new token of the head as quantised by its owning
+  // warp: K codes [0, 64), V codes [64, 128), K (scale, zero) at 128 and V's
+  // at 136, each padded to 8 bytes
+  __shared__ __align__(16) uint8_t s_new[Q4 ? 144 : 16];
+  // 4-bit: the query fragments, the same in every warp (they depend on the
+  // lane only), as [4][32 lanes][4 words]; the tile reloads them instead of
+  // holding 16 registers through it
+  __shared__ __align__(16) uint32_t s_q[Q4 ? 4 * 32 * 4 : 4];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
@@ -167,49 +233,53 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const int first = split_head ? (split * ts + warp) * T : k0 + warp * T;
   const int last = split_head ? min(keys, t1 * T) : k1;
 
+  // Bring rows [kb, min(kb + T, last)) of this head (one tile, inside one
+  // block) into L2 with bulk prefetches (lane 0 of the calling warp).  A
+  // block-table entry may be read here before the wait below; it only aims a
+  // prefetch, and is clamped to the pool so the address stays valid.
+  auto prefetch_tile = [&](int kb) {
+    const int rows = min(T, last - kb);
+    int64_t row = srow0() + kb;
+    const uint8_t *pk = P.p.str_k, *pv = P.p.str_v, *psk = P.p.str_k_sz, *psv = P.p.str_v_sz;
+    if (retrieval) {
+      pk = P.p.ret_k;
+      pv = P.p.ret_v;
+      psk = P.p.ret_k_sz;
+      psv = P.p.ret_v_sz;
+      if (P.ret.table) {
+        int64_t blk = P.ret.table[(int64_t)b * P.ret.stride + (kb >> kPageShift)];
+        blk = blk < 0 ? 0 : (blk >= P.ret.blocks ? P.ret.blocks - 1 : blk);
+        row = ((blk * P.n_ret + pidx) << kPageShift) + (kb & (kPageTokens - 1));
+      } else {
+        row = ret_row(P.ret, b, pidx, kb);
+      }
+    }
+    prefetch_l2(pk + row * RB, (uint32_t)(rows * RB));
+    prefetch_l2(pv + row * RB, (uint32_t)(rows * RB));
+    if (Q4) {  // 4-byte (scale, zero) rows; buffers hold a multiple of 4 rows
+      const uint32_t sz = (uint32_t)(((rows + 3) & ~3) * 4);
+      prefetch_l2(psk + row * 4, sz);
+      prefetch_l2(psv + row * 4, sz);
+    }
+  };
   // Launched with programmatic dependent launch, so this may run while the
   // previous kernel in the stream finishes.  Bring this warp's first two
   // tiles into L2 meanwhile: every global write lands in L2, so a line
   // fetched now cannot be stale when the loads below (after the wait) use it.
-  // A block-table entry read now may be stale; it only aims a prefetch, and
-  // is clamped to the pool so the address stays valid.
   if (lane == 0) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int kb = first + i * NWARPS * T;
-      if (kb < last) {
-        const int rows = min(T, last - kb);
-        int64_t row = srow0() + kb;
-        const uint8_t *pk = P.p.str_k, *pv = P.p.str_v, *psk = P.p.str_k_sz, *psv = P.p.str_v_sz;
-        if (retrieval) {
-          pk = P.p.ret_k;
-          pv = P.p.ret_v;
-          psk = P.p.ret_k_sz;
-          psv = P.p.ret_v_sz;
-          if (P.ret.table) {
-            int64_t blk = P.ret.table[(int64_t)b * P.ret.stride + (kb >> kPageShift)];
-            blk = blk < 0 ? 0 : (blk >= P.ret.blocks ? P.ret.blocks - 1 : blk);
-            row = ((blk * P.n_ret + pidx) << kPageShift) + (kb & (kPageTokens - 1));
-          } else {
-            row = ret_row(P.ret, b, pidx, kb);
-          }
-        }
-        prefetch_l2(pk + row * RB, (uint32_t)(rows * RB));
-        prefetch_l2(pv + row * RB, (uint32_t)(rows * RB));
-        if (Q4) {  // 4-byte (scale, zero) rows; buffers hold a multiple of 4 rows
-          const uint32_t sz = (uint32_t)(((rows + 3) & ~3) * 4);
-          prefetch_l2(psk + row * 4, sz);
-          prefetch_l2(psv + row * 4, sz);
-        }
-      }
+      if (kb < last) prefetch_tile(kb);
     }
   }
   // Nothing the previous kernel may have written is read before this.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // Fused append (bf16 cache): the token at position n-1 is not in the cache
-  // yet.  The warp whose tile holds its row writes it there, skips that row,
-  // and adds the key at the end from the inputs.
+  // Fused append: the token at position n-1 is not in the cache yet.  The
+  // warp whose tile holds its row writes it there, skips that row, and adds
+  // the key at the end from the inputs (bf16) or from its shared-memory copy
+  // (4-bit).
   // In partial mode a rank that does not own the streaming heads leaves
   // their rows empty (another shard contributes them).
   if (P.part_o && !retrieval && !P.own_str) {
@@ -218,17 +288,43 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     if (tid < G) P.part_lse[row0 + tid] = -INFINITY;
     return;
   }
-  const bool fused = !Q4 && P.knew != nullptr && new_here_shard;
+  const bool fused = P.knew != nullptr && new_here_shard;
   const int newk = retrieval ? n - 1 - (int)P.shard_lo : (int)ring_slot(n - 1, P.S, P.R);  // its row
   const bool owns_new = fused && !split_head && newk >= k0 && newk < k1;
-  auto write_new = [&]() {  // one warp copies the new K and V rows into the cache
-    const int64_t off = ((int64_t)r * P.Hkv + kvh) * (int64_t)RB;
-    const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
-    const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + off;
+  const int64_t in_off = ((int64_t)r * P.Hkv + kvh) * (int64_t)(D * 2);  // its K/V in the inputs (bf16)
+  auto write_new = [&]() {  // one warp writes the new K and V rows into the cache
     const int64_t row = retrieval ? ret_row(P.ret, b, pidx, newk) : srow0() + newk;
-    uint8_t *dst = const_cast<uint8_t *>(lane < 16 ? (retrieval ? P.p.ret_k : P.p.str_k)
-                                                   : (retrieval ? P.p.ret_v : P.p.str_v)) + row * RB;
-    reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
+    if constexpr (Q4) {
+      // lane l quantises channels 4l .. 4l+3 of each row, as the append does
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint2 raw = ldg64(reinterpret_cast<const uint8_t *>(which ? P.vnew : P.knew) + in_off + 8 * lane);
+        const float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
+                            __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u)};
+        __half sch, zph;
+        const uint32_t packed = quantize_row_int4<4>(x, &sch, &zph);
+        uint8_t *codes = which ? (retrieval ? P.p.ret_v : P.p.str_v) : (retrieval ? P.p.ret_k : P.p.str_k);
+        uint8_t *sz = which ? (retrieval ? P.p.ret_v_sz : P.p.str_v_sz)
+                            : (retrieval ? P.p.ret_k_sz : P.p.str_k_sz);
+        *reinterpret_cast<uint16_t *>(codes + row * RB + 2 * lane) = (uint16_t)packed;
+        *reinterpret_cast<uint16_t *>(s_new + 64 * which + 2 * lane) = (uint16_t)packed;
+        if (lane == 0) {
+          __half2 pair;
+          pair.x = sch;
+          pair.y = zph;
+          reinterpret_cast<__half2 *>(sz)[row] = pair;
+          *reinterpret_cast<uint2 *>(s_new + 128 + 8 * which) =
+              make_uint2(*reinterpret_cast<const uint32_t *>(&pair), 0u);
+        }
+      }
+      __syncwarp();
+    } else {
+      const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
+      const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + in_off;
+      uint8_t *dst = (lane < 16 ? (retrieval ? P.p.ret_k : P.p.str_k)
+                                : (retrieval ? P.p.ret_v : P.p.str_v)) + row * RB;
+      reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
+    }
   };
   if (owns_new && warp == 0) write_new();
 
@@ -236,42 +332,71 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   uint32_t qa[8][2];
   float qsum = 0.f;  // sum of the query's channels (4-bit zero-point term)
   const bool live = g < G;
+  const float sl2 = P.scale_log2;
+  // 4-bit: score (log2 units) = raw * (sc * c1) + zp * c2, raw = the MMA sum
+  float c1 = sl2, c2 = 0.f;
   {
     const __nv_bfloat16 *qrow =
         reinterpret_cast<const __nv_bfloat16 *>(P.q) + ((int64_t)r * P.Hq + (int64_t)kvh * G + g) * D;
+    if constexpr (Q4) {
+      // Thread column t holds channels 32t .. 32t+31 of its key rows: word w
+      // of the 16-byte load covers 32t + 8w .. +7, and k-steps 2w and 2w+1
+      // take its four registers: (c0, c4), (c1, c5)x16, (c2, c6), (c3, c7)x16
+      // (see kNib0 / kNib1); the x16 slots get q/16.
+      float qv[32];
+      float amax = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      int c0, c1, c2, c3;  // channels behind k-slots 2t, 2t+1, 2t+8, 2t+9
-      if (Q4) {
-        const int w = k >> 1, tt = k & 1;
-        c0 = 32 * t + 8 * w + 2 * tt;
-        c1 = c0 + 4;
-        c2 = c0 + 1;
-        c3 = c0 + 5;
-      } else {
-        const int s = k >> 1, tt = k & 1;
-        c0 = 32 * s + 8 * t + 4 * tt;
-        c1 = c0 + 1;
-        c2 = c0 + 2;
-        c3 = c0 + 3;
+      for (int i = 0; i < 32; ++i) {
+        qv[i] = live ? __bfloat162float(qrow[32 * t + i]) : 0.f;
+        amax = fmaxf(amax, fabsf(qv[i]));
+        qsum += qv[i];
       }
-      const float q0 = live ? __bfloat162float(qrow[c0]) : 0.f;
-      const float q1 = live ? __bfloat162float(qrow[c1]) : 0.f;
-      const float q2 = live ? __bfloat162float(qrow[c2]) : 0.f;
-      const float q3 = live ? __bfloat162float(qrow[c3]) : 0.f;
-      qa[k][0] = pack_bf16(q0, q1);  // exact: the inputs are bf16
-      qa[k][1] = pack_bf16(q2, q3);
-      qsum += (q0 + q1) + (q2 + q3);
+      qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+      qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // a power of two keeps |q| below 2^15 in f16 (taken back in c1)
+      const int ex = ((__float_as_int(amax) >> 23) & 0xff) - 127;
+      const int eq = ex > 14 ? ex - 14 : 0;
+      const float qs = exp2i(-eq), qs16 = qs * 0.0625f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float *c = qv + 8 * w;
+        qa[2 * w][0] = pack_f16(c[0] * qs, c[4] * qs);
+        qa[2 * w][1] = pack_f16(c[1] * qs16, c[5] * qs16);
+        qa[2 * w + 1][0] = pack_f16(c[2] * qs, c[6] * qs);
+        qa[2 * w + 1][1] = pack_f16(c[3] * qs16, c[7] * qs16);
+      }
+      c1 = sl2 * kTwo24 * exp2i(eq);
+      c2 = qsum * sl2;
+      if (warp == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4 *>(&s_q[(j * 32 + lane) * 4]) =
+              make_uint4(qa[2 * j][0], qa[2 * j][1], qa[2 * j + 1][0], qa[2 * j + 1][1]);
+      }
+      __syncthreads();
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        // channels behind k-slots 2t, 2t+1, 2t+8, 2t+9
+        const int s = k >> 1, tt = k & 1;
+        const int c0 = 32 * s + 8 * t + 4 * tt;
+        const float q0 = live ? __bfloat162float(qrow[c0]) : 0.f;
+        const float q1 = live ? __bfloat162float(qrow[c0 + 1]) : 0.f;
+        const float q2 = live ? __bfloat162float(qrow[c0 + 2]) : 0.f;
+        const float q3 = live ? __bfloat162float(qrow[c0 + 3]) : 0.f;
+        qa[k][0] = pack_bf16(q0, q1);  // exact: the inputs are bf16
+        qa[k][1] = pack_bf16(q2, q3);
+      }
     }
-    qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
-    qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   }
-  const float sl2 = P.scale_log2;
 
   // O^T accumulators: tile mt holds channels vchan(mt) (rows g) and
   // vchan(mt) + 1 (rows g+8) for queries 2t and 2t+1.  bf16: the thread's V
   // channels are the 16-byte chunks g and 8+g of a row (so the eight lanes of
-  // a key read 128 contiguous bytes); 4-bit: code bytes 8g..8g+7.
+  // a key read 128 contiguous bytes); 4-bit: code bytes 8g..8g+7, and the
+  // rows g+8 accumulate 16x (the nibble at bits 4..7).
   auto vchan = [&](int mt) {
     return Q4 ? 16 * g + 2 * mt : 64 * (mt >> 2) + 8 * g + 2 * (mt & 3);
   };
@@ -279,99 +404,58 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   // softmax state of query g (identical in the four threads of a row); for the
-  // 4-bit cache z = sum p*zp and cs = sum p*sc (as multiplied, see below)
-  float m = -INFINITY, l = 0.f, z = 0.f, cs = 0.f;
+  // 4-bit cache z = sum p*zp, and p is taken relative to m - f (f: headroom
+  // exponent, the same in every lane; at most 20, which the smallest scales
+  // allow)
+  float m = -INFINITY, l = 0.f, z = 0.f;
+  int f = 20;
 
-  // One warp, keys [kb0, kb0 + 16*KG) below hi of the buffers Kx/Vx (and, for
-  // the 4-bit cache, the (scale, zero) rows Ksx/Vsx), row index = key, except
-  // `skip_key`.
-  // `full` (a compile-time flag) promises that all keys of the tile lie below
-  // hi and none is skip_key, so no load or score needs a bounds test.
-  auto tile = [&](auto full, const uint8_t *Kx, const uint8_t *Vx, const uint8_t *Ksx,
-                  const uint8_t *Vsx, int kb0, int hi, int skip_key) {
+  // bf16 cache, one warp: keys [kb0, kb0 + 16) below hi of the buffers Kx/Vx,
+  // row index = key, except `skip_key`.  `full` (a compile-time flag)
+  // promises that all keys of the tile lie below hi and none is skip_key, so
+  // no load or score needs a bounds test.
+  auto tile = [&](auto full, const uint8_t *Kx, const uint8_t *Vx, int kb0, int hi, int skip_key) {
     constexpr bool FULL = decltype(full)::value;
     // ------------------------------------------------------------ loads (all up front)
-    // group kg covers keys kb = kb0 + 16*kg ..: K of key kb + 8*nt + g (this
-    // thread's column of S); V of keys kb + {2t, 2t+1, 8+2t, 9+2t} (the k-slots
-    // of the P^T fragment) at this thread's channels (see vchan below).
-    uint4 kr[KG][2][Q4 ? 1 : 4];
-    uint2 ksz[KG][2], vsz[KG][2];
-    uint4 vr[KG][4][Q4 ? 1 : 2];
+    // K of key kb0 + 8*nt + g (this thread's column of S); V of keys
+    // kb0 + {2t, 2t+1, 8+2t, 9+2t} (the k-slots of the P^T fragment) at this
+    // thread's channels (see vchan).
+    uint4 kr[2][4];
+    uint4 vr[4][2];
 #pragma unroll
-    for (int kg = 0; kg < KG; ++kg) {
-      const int kb = kb0 + 16 * kg;
+    for (int nt = 0; nt < 2; ++nt) {
+      const int key = kb0 + 8 * nt + g;
+      const bool ok = FULL || (key < hi && key != skip_key);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int key = kb + 8 * nt + g;
-        const bool ok = FULL || (key < hi && key != skip_key);
-        if (Q4) {
-          kr[kg][nt][0] = ok ? ldg128(Kx + key * RB + 16 * t) : make_uint4(0, 0, 0, 0);
-          const int key2 = kb + 8 * nt + 2 * t;
-          ksz[kg][nt] = (FULL || key2 < hi) ? ldg64(Ksx + key2 * 4) : make_uint2(0, 0);
-          vsz[kg][nt] = (FULL || key2 < hi) ? ldg64(Vsx + key2 * 4) : make_uint2(0, 0);
-        } else {
+      for (int sp = 0; sp < 4; ++sp)
+        kr[nt][sp] = ok ? ldg128(Kx + key * RB + (32 * sp + 8 * t) * 2) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-          for (int sp = 0; sp < 4; ++sp)
-            kr[kg][nt][sp] = ok ? ldg128(Kx + key * RB + (32 * sp + 8 * t) * 2) : make_uint4(0, 0, 0, 0);
-        }
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int key = kb0 + 2 * t + (i & 1) + 8 * (i >> 1);
+      const bool ok = FULL || (key < hi && key != skip_key);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
-        const bool ok = FULL || (key < hi && key != skip_key);
-        if (Q4) {
-          const uint2 x = ok ? ldg64(Vx + key * RB + 8 * g) : make_uint2(0, 0);
-          vr[kg][i][0] = make_uint4(x.x, x.y, 0, 0);
-        } else {
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            vr[kg][i][h] = ok ? ldg128(Vx + key * RB + 16 * (8 * h + g)) : make_uint4(0, 0, 0, 0);
-        }
-      }
+      for (int h = 0; h < 2; ++h)
+        vr[i][h] = ok ? ldg128(Vx + key * RB + 16 * (8 * h + g)) : make_uint4(0, 0, 0, 0);
     }
     // ------------------------------------------------------------ S = Q K^T
-    float sc[KG][2][2];
+    float sc[2][2];
 #pragma unroll
-    for (int kg = 0; kg < KG; ++kg) {
-      const int kb = kb0 + 16 * kg;
+    for (int nt = 0; nt < 2; ++nt) {
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        if (Q4) {
-          const uint32_t w4[4] = {kr[kg][nt][0].x, kr[kg][nt][0].y, kr[kg][nt][0].z, kr[kg][nt][0].w};
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            mma16816(s, qa[2 * w][0], qa[2 * w][1], nib2(w4[w], 0), nib2(w4[w], 4));
-            mma16816(s, qa[2 * w + 1][0], qa[2 * w + 1][1], nib2(w4[w], 8), nib2(w4[w], 12));
-          }
-        } else {
-#pragma unroll
-          for (int sp = 0; sp < 4; ++sp) {
-            mma16816(s, qa[2 * sp][0], qa[2 * sp][1], kr[kg][nt][sp].x, kr[kg][nt][sp].y);
-            mma16816(s, qa[2 * sp + 1][0], qa[2 * sp + 1][1], kr[kg][nt][sp].z, kr[kg][nt][sp].w);
-          }
-        }
-        // scores of query g at keys kb + 8*nt + 2t + e
-        const int key = kb + 8 * nt + 2 * t;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float raw = s[e];
-          if (Q4) {
-            const __half2 kp = *reinterpret_cast<const __half2 *>(e ? &ksz[kg][nt].y : &ksz[kg][nt].x);
-            // q.(128 + u) = q.u + 128*sum(q):  s = sc*q.u + zp*sum(q)
-            const float ksc = __low2float(kp);
-            raw = ksc * raw + (__high2float(kp) - 128.f * ksc) * qsum;
-          }
-          sc[kg][nt][e] =
-              (live && (FULL || (key + e < hi && key + e != skip_key))) ? raw * sl2 : -INFINITY;
-        }
+      for (int sp = 0; sp < 4; ++sp) {
+        mma16816(s, qa[2 * sp][0], qa[2 * sp][1], kr[nt][sp].x, kr[nt][sp].y);
+        mma16816(s, qa[2 * sp + 1][0], qa[2 * sp + 1][1], kr[nt][sp].z, kr[nt][sp].w);
       }
+      // scores of query g at keys kb0 + 8*nt + 2t + e
+      const int key = kb0 + 8 * nt + 2 * t;
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        sc[nt][e] = (live && (FULL || (key + e < hi && key + e != skip_key))) ? s[e] * sl2 : -INFINITY;
     }
     // ------------------------------------------------------------ online softmax
-    float mx = -INFINITY;
-#pragma unroll
-    for (int kg = 0; kg < KG; ++kg)
-      mx = fmaxf(mx, fmaxf(fmaxf(sc[kg][0][0], sc[kg][0][1]), fmaxf(sc[kg][1][0], sc[kg][1][1])));
+    float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     // Rescale only when the running max grows by more than 2^8 (numerator and
@@ -381,8 +465,6 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     if (grow) {
       alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
       l *= alpha;
-      z *= alpha;
-      cs *= alpha;
       m = mx;
     }
     if (__any_sync(0xffffffffu, grow)) {
@@ -398,78 +480,195 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         o[i][3] *= a1;
       }
     }
+    float p[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        p[nt][e] = (sc[nt][e] == -INFINITY) ? 0.f : fast_exp2(sc[nt][e] - m);
+        l += p[nt][e];
+      }
+    // P^T fragment: b0 = keys 2t, 2t+1 (tile 0), b1 = keys 8+2t, 9+2t (tile 1)
+    const uint32_t pb0 = pack_bf16(p[0][0], p[0][1]);
+    const uint32_t pb1 = pack_bf16(p[1][0], p[1][1]);
+    // ---------------------------------------------------------- O^T += V^T P^T
+    const uint4 *va = vr[0], *vb = vr[1], *vc = vr[2], *vd = vr[3];
+    const uint32_t wa[8] = {va[0].x, va[0].y, va[0].z, va[0].w, va[1].x, va[1].y, va[1].z, va[1].w};
+    const uint32_t wb[8] = {vb[0].x, vb[0].y, vb[0].z, vb[0].w, vb[1].x, vb[1].y, vb[1].z, vb[1].w};
+    const uint32_t wc[8] = {vc[0].x, vc[0].y, vc[0].z, vc[0].w, vc[1].x, vc[1].y, vc[1].z, vc[1].w};
+    const uint32_t wd[8] = {vd[0].x, vd[0].y, vd[0].z, vd[0].w, vd[1].x, vd[1].y, vd[1].z, vd[1].w};
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)  // word mt holds channels vchan(mt), +1
+      mma16816_full(o[mt], __byte_perm(wa[mt], wb[mt], 0x5410u), __byte_perm(wa[mt], wb[mt], 0x7632u),
+                    __byte_perm(wc[mt], wd[mt], 0x5410u), __byte_perm(wc[mt], wd[mt], 0x7632u), pb0,
+                    pb1);
+  };
+
+  // 4-bit cache, one warp: keys [kb0, kb0 + 32) below hi, except `skip_key`.
+  // The pointers are this thread's own starting points in the tile: K codes
+  // at the tile's first row + g rows + 16t bytes, V codes at + 2t rows + 8g
+  // bytes, (scale, zero) rows at + 2t rows; every load of the tile is then an
+  // immediate offset from one of them.  `full` as above; `gen` reads through
+  // generic pointers (the staged new token).
+  auto tile_q4 = [&](auto full, auto gen, const uint8_t *Kt, const uint8_t *Vt, const uint8_t *Kst,
+                     const uint8_t *Vst, int kb0, int hi, int skip_key) {
+    constexpr bool FULL = decltype(full)::value;
+    constexpr bool GEN = decltype(gen)::value;
+    // ------------------------------------------------------------ loads (all up front)
+    // group kg covers keys kb = kb0 + 16*kg ..: K codes of key kb + 8*nt + g
+    // (bytes 16t..16t+15: channels 32t..32t+31); (scale, zero) of keys
+    // kb + 8*nt + 2t, +1 (this thread's score columns); V codes of keys
+    // kb + {2t, 2t+1, 8+2t, 9+2t} at bytes 8g..8g+7 (channels 16g..16g+15).
+    uint4 kr[KG][2];
+    uint2 ksz[KG][2], vsz[KG][2];
+    uint2 vr[KG][4];
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
-      float p[2][2];
+      const int kb = kb0 + 16 * kg;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt) {
+        const int r0 = 16 * kg + 8 * nt;  // tile row of this thread's group
+        const int key = kb + 8 * nt + g;
+        const bool ok = FULL || (key < hi && key != skip_key);
+        kr[kg][nt] = ok ? ld16<GEN>(Kt + r0 * RB) : make_uint4(0, 0, 0, 0);
+        const int key2 = kb + 8 * nt + 2 * t;
+        ksz[kg][nt] = (FULL || key2 < hi) ? ld8<GEN>(Kst + r0 * 4) : make_uint2(0, 0);
+        vsz[kg][nt] = (FULL || key2 < hi) ? ld8<GEN>(Vst + r0 * 4) : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r0 = 16 * kg + (i & 1) + 8 * (i >> 1);
+        const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
+        const bool ok = FULL || (key < hi && key != skip_key);
+        vr[kg][i] = ok ? ld8<GEN>(Vt + r0 * RB) : make_uint2(0, 0);
+      }
+    }
+    // ------------------------------------------------------------ headroom
+    // The largest V scale of the tile bounds p*sc: with p < 2^(8+f) (the lazy
+    // rescale below) and sc < 2^(E-14) for an fp16 exponent field E >= 1,
+    // f = 21 - E keeps p*sc < 2^15.  Positive fp16 values order as integers.
+    uint32_t vm = 0;
+#pragma unroll
+    for (int kg = 0; kg < KG; ++kg)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) vm = __vmaxu2(vm, __vmaxu2(vsz[kg][nt].x, vsz[kg][nt].y));
+    vm &= 0xffffu;  // the scales (low halves)
+    vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, 1));
+    vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, 2));
+    const int ftile = 21 - max((int)(vm >> 10), 1);
+    // ------------------------------------------------------------ S = Q K^T
+    float sc[KG][2][2];
+#pragma unroll
+    for (int kg = 0; kg < KG; ++kg) {
+      const int kb = kb0 + 16 * kg;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t w4[4] = {kr[kg][nt].x, kr[kg][nt].y, kr[kg][nt].z, kr[kg][nt].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
+          const uint32_t x = w4[w], y = x >> 8;
+          mma16816_f16(s, qf.x, qf.y, x & kNib0, x & kNib1);
+          mma16816_f16(s, qf.z, qf.w, y & kNib0, y & kNib1);
+        }
+        // scores of query g at keys kb + 8*nt + 2t + e
+        const int key = kb + 8 * nt + 2 * t;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          p[nt][e] = (sc[kg][nt][e] == -INFINITY) ? 0.f : fast_exp2(sc[kg][nt][e] - m);
-          l += p[nt][e];
-          if (Q4) {  // the key's V (scale, zero), unpacked where used
-            const __half2 vp = *reinterpret_cast<const __half2 *>(e ? &vsz[kg][nt].y : &vsz[kg][nt].x);
-            z += p[nt][e] * __high2float(vp);
-            p[nt][e] *= __low2float(vp);
-          }
+          const float2 kp = half2_bits_to_f2(e ? ksz[kg][nt].y : ksz[kg][nt].x);  // (scale, zero)
+          const float v = fmaf(s[e], kp.x * c1, kp.y * c2);
+          sc[kg][nt][e] = (FULL || (key + e < hi && key + e != skip_key)) ? v : -INFINITY;
         }
-      // P^T fragment: b0 = keys 2t, 2t+1 (tile 0), b1 = keys 8+2t, 9+2t (tile 1)
-      const uint32_t pb0 = pack_bf16(p[0][0], p[0][1]);
-      const uint32_t pb1 = pack_bf16(p[1][0], p[1][1]);
-      // 4-bit cache: p*sc multiplies codes up to 15 whose sum is offset by the
-      // zero point, so bf16's 8-bit mantissa alone is too coarse; the residual
-      // p*sc - bf16(p*sc) goes through a second product (16 mantissa bits).
-      uint32_t pl0 = 0u, pl1 = 0u;
-      if (Q4) {
-        const __nv_bfloat162 h0 = *reinterpret_cast<const __nv_bfloat162 *>(&pb0);
-        const __nv_bfloat162 h1 = *reinterpret_cast<const __nv_bfloat162 *>(&pb1);
-        pl0 = pack_bf16(p[0][0] - __low2float(h0), p[0][1] - __high2float(h0));
-        pl1 = pack_bf16(p[1][0] - __low2float(h1), p[1][1] - __high2float(h1));
-        // The V codes enter as 128 + u: remember exactly what was multiplied
-        // so that 128 * sum(p*sc) can be removed from O afterwards.
-        const __nv_bfloat162 l0 = *reinterpret_cast<const __nv_bfloat162 *>(&pl0);
-        const __nv_bfloat162 l1 = *reinterpret_cast<const __nv_bfloat162 *>(&pl1);
-        cs += ((__low2float(h0) + __low2float(l0)) + (__high2float(h0) + __high2float(l0))) +
-              ((__low2float(h1) + __low2float(l1)) + (__high2float(h1) + __high2float(l1)));
       }
-      // ---------------------------------------------------------- O^T += V^T P^T
-      if (Q4) {
+    }
+    // ------------------------------------------------------------ online softmax
+    float mx = -INFINITY;
 #pragma unroll
-        for (int wi = 0; wi < 2; ++wi) {
-          const uint32_t xa = wi ? vr[kg][0][0].y : vr[kg][0][0].x, xb = wi ? vr[kg][1][0].y : vr[kg][1][0].x;
-          const uint32_t xc = wi ? vr[kg][2][0].y : vr[kg][2][0].x, xd = wi ? vr[kg][3][0].y : vr[kg][3][0].x;
+    for (int kg = 0; kg < KG; ++kg)
+      mx = fmaxf(mx, fmaxf(fmaxf(sc[kg][0][0], sc[kg][0][1]), fmaxf(sc[kg][1][0], sc[kg][1][1])));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    // Rescale when the running max grows by more than 2^8 or the headroom
+    // must shrink (numerator and denominator scale together).
+    const bool grow = mx > m + 8.f || (m == -INFINITY && mx > -INFINITY);
+    const bool shrink = ftile < f;  // the same in every lane
+    if (__any_sync(0xffffffffu, grow) || shrink) {
+      float alpha = 1.f;
+      if (grow) {
+        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
+        m = mx;
+      }
+      if (shrink) {
+        alpha *= exp2i(ftile - f);
+        f = ftile;
+      }
+      l *= alpha;
+      z *= alpha;
+      const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * t) << 2);
+      const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) << 2);
 #pragma unroll
-          for (int j = 0; j < 4; j += 2) {
-            const uint32_t sel = j ? 0x7632u : 0x5410u;
-            const uint32_t ab = __byte_perm(xa, xb, sel);  // [A_j, A_j+1, B_j, B_j+1]
-            const uint32_t cd = __byte_perm(xc, xd, sel);
+      for (int i = 0; i < 8; ++i) {
+        o[i][0] *= a0;
+        o[i][2] *= a0;
+        o[i][1] *= a1;
+        o[i][3] *= a1;
+      }
+    }
+    const float ref = m - (float)f;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int mt = 4 * wi + j + h;  // code byte 8g + mt: channels 16g + 2mt, +1
-              const uint32_t a0 = nib2(ab, 8 * h), a1 = nib2(ab, 8 * h + 4);
-              const uint32_t a2 = nib2(cd, 8 * h), a3 = nib2(cd, 8 * h + 4);
-              mma16816_full(o[mt], a0, a1, a2, a3, pb0, pb1);
-              mma16816_full(o[mt], a0, a1, a2, a3, pl0, pl1);
-            }
-          }
+    for (int kg = 0; kg < KG; ++kg) {
+      float pv[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float x = sc[kg][nt][e];
+          // a full tile has finite scores in every row, so ref is finite
+          const float p = (FULL || x != -INFINITY) ? fast_exp2(x - ref) : 0.f;
+          const float2 vp = half2_bits_to_f2(e ? vsz[kg][nt].y : vsz[kg][nt].x);  // (scale, zero)
+          l += p;
+          z = fmaf(p, vp.y, z);
+          pv[nt][e] = p * vp.x;
         }
-      } else {
-        const uint4 *va = vr[kg][0], *vb = vr[kg][1], *vc = vr[kg][2], *vd = vr[kg][3];
-        const uint32_t wa[8] = {va[0].x, va[0].y, va[0].z, va[0].w, va[1].x, va[1].y, va[1].z, va[1].w};
-        const uint32_t wb[8] = {vb[0].x, vb[0].y, vb[0].z, vb[0].w, vb[1].x, vb[1].y, vb[1].z, vb[1].w};
-        const uint32_t wc[8] = {vc[0].x, vc[0].y, vc[0].z, vc[0].w, vc[1].x, vc[1].y, vc[1].z, vc[1].w};
-        const uint32_t wd[8] = {vd[0].x, vd[0].y, vd[0].z, vd[0].w, vd[1].x, vd[1].y, vd[1].z, vd[1].w};
+      }
+      // P^T fragment (p*sc as f16 high part and residual): b0 = keys 2t,
+      // 2t+1, b1 = keys 8+2t, 9+2t
+      const uint32_t pb0 = pack_f16(pv[0][0], pv[0][1]);
+      const uint32_t pb1 = pack_f16(pv[1][0], pv[1][1]);
+      const float2 h0 = half2_bits_to_f2(pb0), h1 = half2_bits_to_f2(pb1);
+      const uint32_t pl0 = pack_f16(pv[0][0] - h0.x, pv[0][1] - h0.y);
+      const uint32_t pl1 = pack_f16(pv[1][0] - h1.x, pv[1][1] - h1.y);
+      // ---------------------------------------------------------- O^T += V^T P^T
+      // A rows g / g+8 are channels vchan(mt) / vchan(mt)+1; cols are keys
+      // (2t, 2t+1) from ab and (8+2t, 9+2t) from cd, two bytes (4 channels)
+      // of each key per byte_perm.
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)  // word mt holds channels vchan(mt), +1
-          mma16816_full(o[mt], __byte_perm(wa[mt], wb[mt], 0x5410u), __byte_perm(wa[mt], wb[mt], 0x7632u),
-                        __byte_perm(wc[mt], wd[mt], 0x5410u), __byte_perm(wc[mt], wd[mt], 0x7632u), pb0,
-                        pb1);
+      for (int wi = 0; wi < 2; ++wi) {
+        const uint32_t xa = wi ? vr[kg][0].y : vr[kg][0].x, xb = wi ? vr[kg][1].y : vr[kg][1].x;
+        const uint32_t xc = wi ? vr[kg][2].y : vr[kg][2].x, xd = wi ? vr[kg][3].y : vr[kg][3].x;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t sel = hh ? 0x7632u : 0x5410u;
+          const uint32_t ab = __byte_perm(xa, xb, sel), cd = __byte_perm(xc, xd, sel);
+          const uint32_t ab8 = ab >> 8, cd8 = cd >> 8;
+          const int mt = 4 * wi + 2 * hh;
+          const uint32_t a0 = ab & kNib0, a1 = ab & kNib1, a2 = cd & kNib0, a3 = cd & kNib1;
+          mma16816_full_f16(o[mt], a0, a1, a2, a3, pb0, pb1);
+          mma16816_full_f16(o[mt], a0, a1, a2, a3, pl0, pl1);
+          const uint32_t b0 = ab8 & kNib0, b1 = ab8 & kNib1, b2 = cd8 & kNib0, b3 = cd8 & kNib1;
+          mma16816_full_f16(o[mt + 1], b0, b1, b2, b3, pb0, pb1);
+          mma16816_full_f16(o[mt + 1], b0, b1, b2, b3, pl0, pl1);
+        }
       }
     }
   };
+
   // A tile of keys [kb0, kb0 + T) below hi: retrieval keys through the block
   // that holds them (indices local to the block), streaming keys in the slot
   // buffer.
+  // this thread's offsets within a 4-bit tile (see tile_q4)
+  const int k_off = g * RB + 16 * t, v_off = 2 * t * RB + 8 * g, s_off = 8 * t;
   auto run_tile = [&](int kb0, int hi, int skip_key) {
     int64_t row;
     int base = 0;
@@ -482,17 +681,21 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       row = srow0();
       pk = P.p.str_k, pv = P.p.str_v, psk = P.p.str_k_sz, psv = P.p.str_v_sz;
     }
-    // 4-bit only: on the bf16 path a second copy of the tile costs more in
-    // registers than the bounds tests it saves
+    const int lo_k = kb0 - base, hi_k = hi - base, sk = skip_key < 0 ? -1 : skip_key - base;
     if constexpr (Q4) {
-      const int lo_k = kb0 - base, hi_k = hi - base, sk = skip_key < 0 ? -1 : skip_key - base;
-      if (lo_k + T <= hi_k && (sk < lo_k || sk >= lo_k + T)) {
-        tile(BoolC<true>{}, pk + row * RB, pv + row * RB, psk + row * 4, psv + row * 4, lo_k, hi_k, sk);
-        return;
-      }
+      // tiles wholly inside the visible range skip every bounds test (4-bit
+      // only: on the bf16 path a second copy costs more in registers than the
+      // tests it saves)
+      const int64_t r = row + lo_k;  // the tile's first storage row
+      const uint8_t *Kt = pk + r * RB + k_off, *Vt = pv + r * RB + v_off;
+      const uint8_t *Kst = psk + r * 4 + s_off, *Vst = psv + r * 4 + s_off;
+      if (lo_k + T <= hi_k && (sk < lo_k || sk >= lo_k + T))
+        tile_q4(BoolC<true>{}, BoolC<false>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk);
+      else
+        tile_q4(BoolC<false>{}, BoolC<false>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk);
+    } else {
+      tile(BoolC<false>{}, pk + row * RB, pv + row * RB, lo_k, hi_k, sk);
     }
-    tile(BoolC<false>{}, pk + row * RB, pv + row * RB, Q4 ? psk + row * 4 : nullptr,
-         Q4 ? psv + row * 4 : nullptr, kb0 - base, hi - base, skip_key < 0 ? -1 : skip_key - base);
   };
   bool new_here = owns_new && warp == 0;  // this warp adds the new token at the end
   if (split_head) {
@@ -512,6 +715,30 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     unsigned c = 0;
     int tt = split * ts + warp;
     if (pooled && tt >= t1 && lane == 0) c = atomicAdd(next, 1u);
+    if constexpr (Q4) {
+      if (!P.ret.table) {
+        // Packed layout: the warp's tiles of its share lie NWARPS tiles apart
+        // in one contiguous page, so the walk only advances four pointers.
+        // Tiles holding the new token or the page's ragged end take the
+        // general path.
+        const int64_t r0 = ret_row(P.ret, b, pidx, (int64_t)tt * T);
+        const uint8_t *Kt = P.p.ret_k + r0 * RB + k_off, *Vt = P.p.ret_v + r0 * RB + v_off;
+        const uint8_t *Kst = P.p.ret_k_sz + r0 * 4 + s_off, *Vst = P.p.ret_v_sz + r0 * 4 + s_off;
+        constexpr int kStep = NWARPS * T;  // rows between a warp's tiles
+        for (; tt < t1; tt += NWARPS) {
+          if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
+          const int kb0 = tt * T;
+          if (kb0 + T <= keys && !(fused && newk >= kb0 && newk < kb0 + T))
+            tile_q4(BoolC<true>{}, BoolC<false>{}, Kt, Vt, Kst, Vst, kb0, keys, -1);
+          else
+            visit(tt);
+          Kt += kStep * RB;
+          Vt += kStep * RB;
+          Kst += kStep * 4;
+          Vst += kStep * 4;
+        }
+      }
+    }
     for (; tt < t1; tt += NWARPS) {
       if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
       visit(tt);
@@ -528,11 +755,14 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       run_tile(kb0, k1, owns_new ? newk : -1);
   }
   if (new_here) {
-    // the new token, straight from the inputs (key 0 of a one-row buffer)
-    const int64_t off = ((int64_t)r * P.Hkv + kvh) * (int64_t)RB;
-    tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + off,
-         reinterpret_cast<const uint8_t *>(P.vnew) + off,
-         nullptr, nullptr, 0, 1, -1);
+    // the new token: key 0 of a one-row buffer, the inputs (bf16) or the
+    // warp's quantised copy in shared memory (4-bit)
+    if constexpr (Q4)
+      tile_q4(BoolC<false>{}, BoolC<true>{}, s_new + k_off, s_new + 64 + v_off, s_new + 128 + s_off,
+              s_new + 136 + s_off, 0, 1, -1);
+    else
+      tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + in_off,
+           reinterpret_cast<const uint8_t *>(P.vnew) + in_off, 0, 1, -1);
   }
 
   // the next kernel in the stream may start its set-up now
@@ -544,9 +774,6 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   if (Q4) {
     z += __shfl_xor_sync(0xffffffffu, z, 1);
     z += __shfl_xor_sync(0xffffffffu, z, 2);
-    cs += __shfl_xor_sync(0xffffffffu, cs, 1);
-    cs += __shfl_xor_sync(0xffffffffu, cs, 2);
-    z -= 128.f * cs;  // the codes were multiplied as 128 + u
   }
   float *red_m = reinterpret_cast<float *>(smem);
   float *red_l = red_m + NWARPS * G;
@@ -555,20 +782,22 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const float z0 = __shfl_sync(0xffffffffu, z, (2 * t) << 2);
   const float z1 = __shfl_sync(0xffffffffu, z, (2 * t + 1) << 2);
   if (live && t == 0) {
-    red_m[warp * G + g] = m;
+    red_m[warp * G + g] = Q4 ? m - (float)f : m;  // the reference of l and O
     red_l[warp * G + g] = l;
   }
+  // 4-bit: rows g carry u * 2^-24, rows g+8 16u * 2^-24
+  const float e0 = Q4 ? kTwo24 : 1.f, e1 = Q4 ? kTwo20 : 1.f;
   const int q0 = 2 * t, q1 = 2 * t + 1;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
     const int ch = vchan(mt);
     if (q0 < G) {
-      red_o[(warp * G + q0) * D + ch] = o[mt][0] + z0;
-      red_o[(warp * G + q0) * D + ch + 1] = o[mt][2] + z0;
+      red_o[(warp * G + q0) * D + ch] = fmaf(o[mt][0], e0, z0);
+      red_o[(warp * G + q0) * D + ch + 1] = fmaf(o[mt][2], e1, z0);
     }
     if (q1 < G) {
-      red_o[(warp * G + q1) * D + ch] = o[mt][1] + z1;
-      red_o[(warp * G + q1) * D + ch + 1] = o[mt][3] + z1;
+      red_o[(warp * G + q1) * D + ch] = fmaf(o[mt][1], e0, z1);
+      red_o[(warp * G + q1) * D + ch + 1] = fmaf(o[mt][3], e1, z1);
     }
   }
   __syncthreads();
@@ -637,9 +866,8 @@ bool decode_mma_supported(int kv_type, int D, int G) {
   return D == 128 && (kv_type == kBF16 || kv_type == kINT4) && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
-bool decode_can_fuse_append(int kv_type, int D, int G) {
-  return kv_type == kBF16 && decode_mma_supported(kv_type, D, G);
-}
+// Both the bf16 and the 4-bit tensor-core decode take the new token themselves.
+bool decode_can_fuse_append(int kv_type, int D, int G) { return decode_mma_supported(kv_type, D, G); }
 
 cudaError_t decode_mma_config(int kv_type, int G, DecodeConfig *cfg) {
   DecodeParams dummy{};

@@ -64,6 +64,8 @@ struct duo_cache {
   int forced_splits;
   int64_t shard_lo, shard_hi;  // retrieval heads keep positions [lo, hi) (sequence shard)
   bool reproducible;       // decode splits take fixed key shares only
+  int32_t out_dtype;       // decode output element type (DUO_F32 or DUO_BF16)
+  int64_t stall_ns;        // testing hook: the next pre-fill loads nothing, waits this long
   bool have_cfg;           // decode launch facts, queried once per cache
   duo::DecodeConfig cfg;
 };
@@ -358,6 +360,8 @@ duo_status create(duo_cache **out, const duo_cache_desc *desc, const uint8_t *he
   c->shard_lo = 0;
   c->shard_hi = kNoShardEnd;
   c->reproducible = false;
+  c->out_dtype = desc->kv_dtype == DUO_F32 ? DUO_F32 : DUO_BF16;
+  c->stall_ns = 0;
   c->have_cfg = false;
   c->row_bytes = d.kv_dtype == DUO_INT4 ? d.head_dim / 2 : d.head_dim * elem_bytes(d.kv_dtype);
   c->pool_blocks = paged ? pool_blocks : 0;
@@ -485,6 +489,7 @@ void fill_decode_common(const duo_cache *c, int32_t layer, const void *q, void *
   p->scale_log2 = sc * 1.4426950408889634f;
   p->err = duo::device_error_word();
   p->pool = c->reproducible ? 0 : 1;
+  p->out_f32 = (d.kv_dtype != DUO_F32 && c->out_dtype == DUO_F32) ? 1 : 0;
   p->shard_lo = c->shard_lo;
   p->shard_hi = c->shard_hi;
 }
@@ -589,7 +594,8 @@ duo_status decode_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &
 
   // Tensor-core decode: plan every launch (up to DUO_MAX_LAUNCH_ROWS rows
   // each) and check its scratch before anything is enqueued.
-  const int64_t q_row = (int64_t)d.n_q_heads * d.head_dim * 2;   // bf16 q / out per row
+  const int64_t q_row = (int64_t)d.n_q_heads * d.head_dim * 2;   // bf16 q per row
+  const int64_t o_row = (int64_t)d.n_q_heads * d.head_dim * (c->out_dtype == DUO_F32 ? 4 : 2);
   const int64_t kv_row = (int64_t)d.n_kv_heads * d.head_dim * 2;  // bf16 k_new / v_new per row
   std::vector<duo::DecodeParams> plans((rows.size() + duo::kMaxLaunchRows - 1) / duo::kMaxLaunchRows);
   std::vector<char> needs(plans.size(), 0);
@@ -598,7 +604,7 @@ duo_status decode_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &
     const int nr = (int)std::min<size_t>(duo::kMaxLaunchRows, rows.size() - g0);
     duo::DecodeParams &p = plans[i];
     fill_decode_common(c, layer, static_cast<const uint8_t *>(q) + (int64_t)g0 * q_row,
-                       out ? static_cast<uint8_t *>(out) + (int64_t)g0 * q_row : nullptr, scale, &p);
+                       out ? static_cast<uint8_t *>(out) + (int64_t)g0 * o_row : nullptr, scale, &p);
     p.rows.n = nr;
     int32_t rlen[duo::kMaxLaunchRows];  // retrieval keys of each row in this shard
     for (int r = 0; r < nr; ++r) {
@@ -750,6 +756,9 @@ duo_status prefill_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> 
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)d.head_dim);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.err = duo::device_error_word();
+  p.wait_ns = c->stall_ns > 0 ? (uint64_t)c->stall_ns : duo::kPrefillWaitNs;
+  p.skip_loads = c->stall_ns > 0 ? 1 : 0;
+  c->stall_ns = 0;  // one call only
   const int64_t q_row = (int64_t)C * d.n_q_heads * d.head_dim * 2;
   const int64_t kv_row = (int64_t)C * d.n_kv_heads * d.head_dim * 2;
   for (size_t g0 = 0; g0 < rows.size(); g0 += duo::kMaxLaunchRows) {
@@ -1049,6 +1058,19 @@ duo_status duo_layout_info(const duo_cache *c, int32_t layer, duo_layout_view *o
 duo_status duo_set_decode_splits(duo_cache *c, int32_t splits) {
   if (!c || splits < 0 || splits > DUO_MAX_SPLITS) return DUO_ERR_ARG;
   c->forced_splits = splits;
+  return DUO_OK;
+}
+
+duo_status duo_test_stall_next_prefill(duo_cache *c, int64_t wait_ns) {
+  if (!c || wait_ns < 1000 || wait_ns > 1000000000LL) return DUO_ERR_ARG;
+  c->stall_ns = wait_ns;
+  return DUO_OK;
+}
+
+duo_status duo_set_decode_output(duo_cache *c, int32_t dtype) {
+  if (!c || (dtype != DUO_F32 && dtype != DUO_BF16)) return DUO_ERR_ARG;
+  if (c->desc.kv_dtype == DUO_F32 && dtype != DUO_F32) return DUO_ERR_UNSUPPORTED;
+  c->out_dtype = dtype;
   return DUO_OK;
 }
 

@@ -23,6 +23,9 @@ constexpr int kMaxLaunchRows = 128;
 
 enum KvType : int { kF32 = 0, kBF16 = 1, kINT4 = 2 };
 
+// Limit of the pre-fill kernel's bounded waits (ns) unless a test shortens it.
+constexpr uint64_t kPrefillWaitNs = 1000000000ull;
+
 // Error word set by bounded in-kernel waits that give up (bit flags).
 enum DeviceError : int {
   kErrWaitTileLoad = 1,
@@ -123,6 +126,7 @@ struct DecodeParams {
   // writes it to the cache.
   const void *knew, *vnew;
   int pdl;             // launched with programmatic dependent launch
+  int out_f32;         // bf16 and 4-bit caches: out is float32 instead of bf16
   int pool;            // tensor-core decode: the last eighth of a split head's
                        // tiles is claimed at run time (0: every split gets an
                        // even, fixed share)
@@ -139,6 +143,8 @@ struct PrefillParams {
   int64_t retrieval_rows; // storage rows of each retrieval buffer of the layer
   float scale_log2;
   int *err;
+  uint64_t wait_ns;       // limit of every bounded wait (normally kWaitNs)
+  int skip_loads;         // testing hook: issue no TMA loads (every wait then gives up)
 };
 
 // 4-bit history expanded to bf16 for the pre-fill: retrieval rows keep their

@@ -356,7 +356,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 8) {
     // =============================================================== TMA producer
-    if (lane == 0) {
+    // (testing hook: with P.skip_loads nothing is loaded, so every wait of
+    // the other roles runs out and the CTA unwinds)
+    if (lane == 0 && !P.skip_loads) {
       const int qz = b * P.C + q0;
       mbar_arrive_expect_tx(bar(Q_FULL), 2 * TILE);
       tma_load3(base + kQA, &M.q, 0, hq, qz, bar(Q_FULL));
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue = [&](int j, bool is_v) -> bool {
         const int st = j & 1;
         if (j >= 2 && !mbar_wait(bar((is_v ? V_EMPTY0 : K_EMPTY0) + st), (uint32_t)(((j - 2) >> 1) & 1),
-                                 P.err, kErrWaitPrefillLoad))
+                                 P.err, kErrWaitPrefillLoad, P.wait_ns))
           return false;
         int seg, idx;
         sc.get(j, seg, idx);
@@ -407,9 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Copies still in flight land before the CTA can exit (bounded waits;
       // an already completed phase returns at once).
       for (int jj = max(0, issued_k - 2); jj < issued_k; ++jj)
-        mbar_wait(bar(K_FULL0 + (jj & 1)), (uint32_t)((jj >> 1) & 1), P.err, kErrWaitPrefillLoad);
+        mbar_wait(bar(K_FULL0 + (jj & 1)), (uint32_t)((jj >> 1) & 1), P.err, kErrWaitPrefillLoad,
+                  P.wait_ns);
       for (int jj = max(0, issued_v - 2); jj < issued_v; ++jj)
-        mbar_wait(bar(V_FULL0 + (jj & 1)), (uint32_t)((jj >> 1) & 1), P.err, kErrWaitPrefillLoad);
+        mbar_wait(bar(V_FULL0 + (jj & 1)), (uint32_t)((jj >> 1) & 1), P.err, kErrWaitPrefillLoad,
+                  P.wait_ns);
     }
   } else if (warp == 9) {
     // =============================================================== MMA issuer
@@ -434,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < BN / 16; ++k)
           mma_ts(tO[x], tS[x] + 8u * k, dv[st] + (uint32_t)((k * 2048) >> 4), kIdescPV, (j > 0 || k > 0));
       };
-      bool ok = mbar_wait(bar(Q_FULL), 0, P.err, kErrWaitMma) &&
-                mbar_wait(bar(K_FULL0), 0, P.err, kErrWaitMma);
+      bool ok = mbar_wait(bar(Q_FULL), 0, P.err, kErrWaitMma, P.wait_ns) &&
+                mbar_wait(bar(K_FULL0), 0, P.err, kErrWaitMma, P.wait_ns);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -447,13 +451,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j & 1;
         const bool more = j + 1 < n_tiles;
-        ok = mbar_wait(bar(V_FULL0 + st), (uint32_t)((j >> 1) & 1), P.err, kErrWaitMma) &&
-             mbar_wait(bar(P_FULL_A), (uint32_t)(j & 1), P.err, kErrWaitMma);
+        ok = mbar_wait(bar(V_FULL0 + st), (uint32_t)((j >> 1) & 1), P.err, kErrWaitMma, P.wait_ns) &&
+             mbar_wait(bar(P_FULL_A), (uint32_t)(j & 1), P.err, kErrWaitMma, P.wait_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, st, j);
         if (more) {
-          ok = mbar_wait(bar(K_FULL0 + (st ^ 1)), (uint32_t)(((j + 1) >> 1) & 1), P.err, kErrWaitMma);
+          ok = mbar_wait(bar(K_FULL0 + (st ^ 1)), (uint32_t)(((j + 1) >> 1) & 1), P.err, kErrWaitMma,
+                         P.wait_ns);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, st ^ 1);
@@ -461,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           mma_commit(bar(O_FULL_A));
         }
-        ok = mbar_wait(bar(P_FULL_B), (uint32_t)(j & 1), P.err, kErrWaitMma);
+        ok = mbar_wait(bar(P_FULL_B), (uint32_t)(j & 1), P.err, kErrWaitMma, P.wait_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(1, st, j);
@@ -477,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) *abort_flag = 1;
       // nothing may still be writing tensor memory when it is freed
       mma_commit(bar(DRAIN));
-      mbar_wait(bar(DRAIN), 0, P.err, kErrWaitMma);
+      mbar_wait(bar(DRAIN), 0, P.err, kErrWaitMma, P.wait_ns);
     }
   }
   } else {
@@ -499,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      ok = mbar_wait(bar(s_bar), (uint32_t)(j & 1), P.err, kErrWaitMma);
+      ok = mbar_wait(bar(s_bar), (uint32_t)(j & 1), P.err, kErrWaitMma, P.wait_ns);
       if (!__all_sync(0xffffffffu, ok) || abort_set(abort_flag)) {
         ok = false;
         break;
@@ -624,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(p_bar));
     }
     const float l = (l2[0].x + l2[0].y) + (l2[1].x + l2[1].y);
-    if (ok) ok = mbar_wait(bar(o_bar), 0, P.err, kErrWaitMma);
+    if (ok) ok = mbar_wait(bar(o_bar), 0, P.err, kErrWaitMma, P.wait_ns);
     if (__all_sync(0xffffffffu, ok) && !abort_set(abort_flag)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;

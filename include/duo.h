@@ -34,7 +34,9 @@
  *      append  k, v     [batch, n_tokens, n_kv_heads, head_dim]
  *      prefill q, out   [batch, C, n_q_heads, head_dim]; k, v [batch, C, n_kv_heads, head_dim]
  *    Element type: float32 for a DUO_F32 cache; bfloat16 for DUO_BF16 and for
- *    the K/V/Q/O of a DUO_INT4 cache (K/V are quantised on append).
+ *    the K/V/Q/O of a DUO_INT4 cache (K/V are quantised on append).  Decode
+ *    outputs of bf16 and 4-bit caches can be float32 instead
+ *    (duo_set_decode_output).
  *  - Every call with a stream is asynchronous on that stream.  Argument,
  *    capacity and layout errors are detected on the host and returned before
  *    anything is enqueued; a failed launch returns DUO_ERR_CUDA.  Nothing
@@ -404,10 +406,30 @@ duo_status duo_set_decode_splits(duo_cache *cache, int32_t splits);
  * cache or on outside {0, 1}. */
 duo_status duo_set_decode_reproducible(duo_cache *cache, int32_t on);
 
+/* Element type of decode outputs: DUO_BF16 (the default for DUO_BF16 and
+ * DUO_INT4 caches) or DUO_F32 (float32; the only type of a DUO_F32 cache).
+ * Applies to duo_decode_attn, duo_decode_step, duo_decode_attn_static and
+ * their *_rows forms: out is then [rows, n_q_heads, head_dim] of that type.
+ * The kernels accumulate in float32 either way; DUO_F32 skips the final
+ * rounding to bf16 (whose half-ulp exceeds 2e-2 once |out| passes 8).
+ * Errors: DUO_ERR_ARG (null cache, other types), DUO_ERR_UNSUPPORTED (DUO_BF16
+ * for a DUO_F32 cache). */
+duo_status duo_set_decode_output(duo_cache *cache, int32_t dtype);
+
 /* Split count the next decode of this layer will use (tensor-core decode: the
  * largest any row gets at the current lengths). */
 duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
                              int32_t *splits);
+
+/* Testing hook for the failure path of the bounded in-kernel waits (the
+ * pages have no counterpart).  The next duo_prefill_attn or
+ * duo_prefill_attn_rows on this cache issues none of its tile loads, and its
+ * waits give up after wait_ns nanoseconds (1000 .. 1e9) instead of a second:
+ * every CTA records the timeout in the device error word, frees its tensor
+ * memory and returns without writing its output, and duo_poll_device_error
+ * then returns DUO_ERR_TIMEOUT.  Nothing faults, traps or hangs; the next call
+ * runs normally.  Errors: DUO_ERR_ARG. */
+duo_status duo_test_stall_next_prefill(duo_cache *cache, int64_t wait_ns);
 
 /* Read and clear the device-side error word that bounded in-kernel waits set
  * when they give up.  Synchronises the device.  Returns DUO_ERR_TIMEOUT if it

@@ -5,34 +5,47 @@ existed): fp32 max |err| <= 1e-5; bf16 max |err| <= 2e-2 and mean |err| <= 2e-3;
 INT4 (against an oracle fed the identically dequantised K/V) max |err| <= 2e-2;
 cache contents and INT4 codes bit-exact.
 
-INT4 outputs are bf16.  The 4-bit workload has x10 outlier channels, so an
-output element can reach |O| ~ 40, and bf16 cannot hold such a value to within
-2e-2: rounding alone moves it by up to half an ulp, 2^-9 |O| (0.078 at 40).
-The INT4 bound is therefore the absolute 2e-2 plus that half-ulp of the
-reference value, 2e-2 + 2^-9 |ref|, elementwise.  No other slack is allowed.
+INT4 parity is checked on float32 outputs (duo_set_decode_output), against the
+absolute 2e-2 as stated.  The default bf16 output of a 4-bit cache is checked
+too, and there the bound also allows the output's own rounding and nothing
+more: half an ulp of bf16 at the element, 2^(floor(log2 |x|) - 8) for
+x = max(|ref|, |got|).  The 4-bit workload's x10 outlier channels give
+|O| ~ 40, where that half-ulp (0.125 at 32..64) is larger than 2e-2 by itself.
 """
 
 import numpy as np
 import torch
 
-BF16_HALF_ULP_REL = 2.0 ** -9
-
 TOL = {
     "f32": dict(max=1e-5, mean=None, bf16_rounding=False),
     "bf16": dict(max=2e-2, mean=2e-3, bf16_rounding=False),
-    "int4": dict(max=2e-2, mean=None, bf16_rounding=True),
+    "int4": dict(max=2e-2, mean=None, bf16_rounding=False),
+    "int4_bf16": dict(max=2e-2, mean=None, bf16_rounding=True),
 }
 
 
+def bf16_half_ulp(x):
+    """Half an ulp of bf16 (8 significant bits) at |x|, elementwise; 0 at 0."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(e - 8.0), 0.0)
+
+
+def _np(t):
+    if isinstance(t, torch.Tensor):
+        return t.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(t, np.float64)
+
+
 def parity_errors(got, ref, bf16_rounding=False):
-    """(max, mean) of |got - ref|; with bf16_rounding the error of each
-    element first loses the output's own rounding allowance, 2^-9 |ref|, so
-    that the result compares directly with the absolute bound."""
-    g = got.detach().to("cpu", torch.float64).numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
+    """(max, mean) of |got - ref|; with bf16_rounding each element's error
+    first loses half an ulp of bf16 at max(|ref|, |got|) (the rounding of the
+    output itself), so that the result compares directly with the bound."""
+    g = _np(got)
     r = np.asarray(ref, dtype=np.float64)
     err = np.abs(g - r)
     if bf16_rounding:
-        err = np.maximum(err - BF16_HALF_ULP_REL * np.abs(r), 0.0)
+        err = np.maximum(err - bf16_half_ulp(np.maximum(np.abs(r), np.abs(g))), 0.0)
     return float(err.max()), float(err.mean())
 
 
@@ -41,16 +54,15 @@ def assert_parity(got, ref, kind, what=""):
     mx, mean = parity_errors(got, ref, tol["bf16_rounding"])
     assert np.isfinite(mx), "%s: non-finite output" % what
     assert mx <= tol["max"], "%s: max |err| %.3g > %.3g%s" % (
-        what, mx, tol["max"], " (+ 2^-9 |ref|)" if tol["bf16_rounding"] else "")
+        what, mx, tol["max"], " (+ bf16 half-ulp)" if tol["bf16_rounding"] else "")
     if tol["mean"] is not None:
         assert mean <= tol["mean"], "%s: mean |err| %.3g > %.3g" % (what, mean, tol["mean"])
     return mx, mean
 
 
 def raw_max_error(got, ref):
-    """Plain max |got - ref| (reported next to the bound in test output)."""
-    g = got.detach().to("cpu", torch.float64).numpy() if isinstance(got, torch.Tensor) else np.asarray(got, np.float64)
-    return float(np.abs(g - np.asarray(ref, dtype=np.float64)).max())
+    """Plain max |got - ref|."""
+    return float(np.abs(_np(got) - np.asarray(ref, dtype=np.float64)).max())
 
 
 def seeded_mask(seed, n_kv, n_ret):

@@ -166,11 +166,19 @@ def test_llama3_gqa_prefill_32k_sampled_rows():
 
 def test_llama3_int4_1m_decode_sampled_heads():
     w = synth.WORKLOADS["llama3_8b_gqa_int4_1m"]
-    cache, q, out, row = _fill_decode(w, 1, chunk=65536)
+    cache, q, out_bf16, row = _fill_decode(w, 1, chunk=65536)
+    cache.set_decode_output(torch.float32)
+    out = cache.decode(0, q)
+    torch.cuda.synchronize()
     ret = [h for h in range(w.n_kv_heads) if row[h]][:1]
     strm = [h for h in range(w.n_kv_heads) if not row[h]][:1]
     G = w.group
+    worst = 0.0
     for h in ret + strm:
-        got = out[0, h * G:(h + 1) * G].float().cpu()
+        got = out[0, h * G:(h + 1) * G].cpu()
         ref = _oracle_head(w, 0, 0, h, row, q, quantised=True)
-        assert_parity(got, ref, "int4", "1M INT4 decode head %d" % h)
+        mx, _ = assert_parity(got, ref, "int4", "1M INT4 decode head %d (fp32 output)" % h)
+        worst = max(worst, mx)
+        assert_parity(out_bf16[0, h * G:(h + 1) * G].cpu(), ref, "int4_bf16",
+                      "1M INT4 decode head %d (bf16 output)" % h)
+    print("1M INT4 decode: max |err| %.3g (fp32 output)" % worst)

@@ -196,7 +196,9 @@ def test_paged_int4_rows_decode():
     cache.append_rows(0, [2], hist[2][0][:, 400:].contiguous(), hist[2][1][:, 400:].contiguous())
     rows = [1, 2, 0]
     q = torch.cat([_seq(60 + r, lens[r], HQ)[:, -1] for r in rows]).contiguous()
+    cache.set_decode_output(torch.float32)
     out = cache.decode_rows(0, rows, q)
+    assert out.dtype == torch.float32
     for i, r in enumerate(rows):
         K, V = hist[r]
         kd = OQ.dequantize_int4(*OQ.quantize_int4(K[0].float().cpu().numpy()))

@@ -157,3 +157,34 @@ def test_prefill_int4_needs_workspace():
         Bd.duo_prefill_attn(c4.handle, 0, qb.data_ptr(), kb.data_ptr(), kb.data_ptr(), 128,
                             qb.data_ptr(), 0.0, None, 0)
     assert e.value.name == "DUO_ERR_WORKSPACE"
+
+
+def test_prefill_bounded_wait_gives_up_and_recovers():
+    """The failure path of the bounded waits, with no fault: the testing hook
+    makes the next pre-fill issue no tile loads and shortens its wait limit to
+    2 ms, so every wait of the MMA and softmax roles runs out.  Each CTA
+    records the timeout, frees its tensor memory and returns; the output is
+    left as it was; duo_poll_device_error reports DUO_ERR_TIMEOUT.  The same
+    process then runs a normal pre-fill that matches the oracle."""
+    from head_split_kv_decode_b200 import binding as Bd
+    B, Hq, Hkv, C, S, R = 1, 8, 2, 256, 4, 64
+    Q, K, V = _prompt(91, B, C, Hq, Hkv)
+    mask = torch.tensor([1, 0], dtype=torch.uint8)
+    cache = DuoCache(1, B, Hq, Hkv, 128, "bf16", C, mask[None], S, R)
+    assert Bd.duo_poll_device_error() == 0
+    with pytest.raises(Bd.DuoError):
+        Bd.duo_test_stall_next_prefill(cache.handle, 10)  # below the allowed range
+    Bd.duo_test_stall_next_prefill(cache.handle, 2_000_000)
+    sentinel = torch.full((B, C, Hq, 128), 7.0, dtype=BF, device="cuda")
+    cache.prefill(0, Q, K, V, out=sentinel)
+    torch.cuda.synchronize()
+    code = Bd.duo_poll_device_error()
+    assert code != 0, "the stalled pre-fill did not report a timeout"
+    assert (code & 2) != 0  # kErrWaitMma: the MMA / softmax waits gave up
+    assert torch.all(sentinel == 7.0)  # no CTA wrote its output
+    assert Bd.duo_poll_device_error() == 0  # polling clears the word
+    out = cache.prefill(0, Q, K, V)  # the hook was one-shot
+    torch.cuda.synchronize()
+    assert Bd.duo_poll_device_error() == 0
+    ref = OA.prefill_reference(f64(Q), f64(K), f64(V), 0, mask.numpy(), S, R)
+    assert_parity(out, ref, "bf16", "pre-fill after a stalled call")

@@ -27,12 +27,12 @@ def _seq(seed, B_, n, heads):
     return synth.kv_field(seed, range(B_), range(n), heads, D, device="cuda").to(BF)
 
 
-def _merged(caches, q, layer=0):
+def _merged(caches, q, layer=0, out_dtype=BF):
     parts = [c.decode_partial(layer, q, owns_streaming=shard.owns_streaming(i))
              for i, c in enumerate(caches)]
     o = torch.stack([p[0] for p in parts]).contiguous()
     lse = torch.stack([p[1] for p in parts]).contiguous()
-    return merge_partials(o, lse, torch.empty(q.shape, dtype=BF, device="cuda")), parts
+    return merge_partials(o, lse, torch.empty(q.shape, dtype=out_dtype, device="cuda")), parts
 
 
 @pytest.mark.parametrize("world,paged", [(3, False), (2, True), (4, False)])
@@ -85,7 +85,7 @@ def test_sharded_int4_decode():
         c.append(0, K.contiguous(), V.contiguous())
         caches.append(c)
     q = Q[:, n - 1].contiguous()
-    got, _ = _merged(caches, q)
+    got, _ = _merged(caches, q, out_dtype=torch.float32)
     kd = OQ.dequantize_int4(*OQ.quantize_int4(K.float().cpu().numpy()))
     vd = OQ.dequantize_int4(*OQ.quantize_int4(V.float().cpu().numpy()))
     ref = OA.decode_reference(f64(q), kd, vd, mask.numpy(), S, R)

@@ -50,8 +50,8 @@ def _two_calls(cache, mask, K, V, Q, n, kind, dequant=None, exact=False):
         t = n + step
         cache.append(0, K[:, t:t + 1].contiguous(), V[:, t:t + 1].contiguous())
         q = Q[:, t].contiguous()
-        ref = torch.empty_like(q)
-        got = torch.full_like(q, float("nan"))
+        ref = torch.empty(q.shape, dtype=cache.out_dtype, device=q.device)
+        got = torch.full(q.shape, float("nan"), dtype=cache.out_dtype, device=q.device)
         B.duo_decode_attn(cache.handle, 0, q.data_ptr(), ref.data_ptr(), 0.0,
                           cache.ws_ptr, cache.ws_bytes)
         B.duo_decode_attn_static(cache.handle, 0, q.data_ptr(), got.data_ptr(), 0.0)
@@ -99,6 +99,7 @@ def test_static_decode_cuda_core_f32_d64():
 def test_static_decode_int4_cache():
     batch, n = 1, 12000
     cache, mask, K, V, Q = _cache(batch, n, 560, kv="int4")
+    cache.set_decode_output(torch.float32)  # the 4-bit bound is absolute
     assert cache.decode_splits(0) > 1
 
     def dequant(x):
