@@ -70,7 +70,7 @@ class DuoCache:
         if self.prefill_ws_bytes == 0:
             return None, 0
         if self._pf_ws is None:
-            self._pf_ws, off = _aligned_buffer(self.prefill_ws_bytes, self.device, zero=True)
+            self._pf_ws, off = _aligned_buffer(self.prefill_ws_bytes, self.device, zero=False)
             self.pf_ws_ptr = self._pf_ws.data_ptr() + off
         return self.pf_ws_ptr, self.prefill_ws_bytes
 

@@ -21,7 +21,11 @@
 // 4-bit cache (f16 operands): a nibble masked into the low bits of a 16-bit
 // half, all other bits zero, is the f16 subnormal u * 2^-24 exactly, and one
 // at bits 4..7 is 16u * 2^-24; so one AND per register turns packed codes into
-// MMA operands, with no offset to remove.  The factor 16 is taken out of the
+// MMA operands, with no offset to remove.  The scores are computed transposed,
+// S^T[16 x 8] = K[16 x 128] . Q^T, so that the codes fill the whole A operand
+// (16 keys per product) and Q is the two-register B operand; each thread then
+// holds two keys for its queries 2t and 2t+1, and P^T for the V product comes
+// from S^T by an 8x8 transpose (movmatrix) per 8 keys.  The factor 16 is taken out of the
 // query (K side, q/16 on those k-slots) or out of the output channel (V
 // side), both exact.  Scale and zero are applied outside the products:
 //   s = sc * (q . u) + zp * sum(q),   sum p*x_hat = sum (p*sc) * u + sum p*zp.
@@ -114,6 +118,59 @@ __device__ __forceinline__ uint2 ld8(const uint8_t *p) {
   else return ldg64(p);
 }
 
+template <bool GEN>
+__device__ __forceinline__ uint32_t ld4(const uint8_t *p) {
+  if constexpr (GEN) return *reinterpret_cast<const uint32_t *>(p);
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Per-thread asynchronous copies global -> shared (no registers held while in
+// flight); completion is per thread, tracked by commit groups.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+template <int N>
+struct IntC {
+  static constexpr int value = N;
+};
+
+// 4-bit decode, copies staged in shared memory: each thread owns 10 chunks of
+// 16 bytes per stage (K codes of its 4 key rows; V codes of its 8 key rows, 8
+// bytes each; the (scale, zero) words of its 4 key rows for K and for V),
+// chunk c of thread i at (c * threads + i) * 16, so that the 16-byte reads of
+// a quarter-warp are contiguous.  Two stages.
+constexpr int kQ4Chunks = 10;
+constexpr uint32_t kQ4Chunk = NWARPS * 32 * 16;      // bytes between a thread's chunks
+constexpr uint32_t kQ4Stage = kQ4Chunks * kQ4Chunk;  // bytes per stage
+
+// Transpose of an 8x8 matrix of 16-bit elements held as the warp's
+// fragments (thread 4i+j holds row i, columns 2j and 2j+1).
+__device__ __forceinline__ uint32_t movm_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 // Fetch [ptr, ptr + bytes) into L2 (16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void *ptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
@@ -170,8 +227,19 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
-  // ---- work item: retrieval CTAs first (launch row r, head, split), then
-  // one CTA per (launch row, streaming head)
+  // ---- work items: retrieval CTAs first (launch row r, head, split), one
+  // item each; then streaming CTAs, each taking P.str_per_cta consecutive
+  // (launch row, streaming head) items in turn (a streaming head's window is
+  // short, so one CTA per head would leave SMs idle that retrieval splits can
+  // use)
+  // The item counter of a streaming CTA lives in shared memory, so that no
+  // register carries it through the body.
+  __shared__ int s_item;
+  if (tid == 0)
+    s_item = (int)blockIdx.x < P.cta0[P.rows.n] ? 0
+                                                 : ((int)blockIdx.x - P.cta0[P.rows.n]) * P.str_per_cta;
+  __syncthreads();
+  for (;;) {
   const int n_ret_ctas = P.cta0[P.rows.n];
   int r, kvh, pidx, split, nsplit;
   bool retrieval;
@@ -189,7 +257,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     kvh = P.h.ret_heads[pidx];
     retrieval = true;
   } else {
-    const int x = (int)blockIdx.x - n_ret_ctas;
+    const int x = s_item;
     r = x / P.n_str;
     pidx = x % P.n_str;
     kvh = P.h.str_heads[pidx];
@@ -197,6 +265,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     split = 0;
     nsplit = 1;
   }
+  {  // the item
   const int b = P.rows.row[r];
   // Key indices and tile counts are 32-bit (a row holds fewer than 2^31
   // tokens); byte offsets are formed in 64 bits.
@@ -286,19 +355,21 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     const int64_t row0 = (int64_t)r * P.Hq + (int64_t)kvh * G;
     for (int i = tid; i < G * D; i += NWARPS * 32) P.part_o[row0 * D + i] = 0.f;
     if (tid < G) P.part_lse[row0 + tid] = -INFINITY;
-    return;
+    goto next_item;  // the same for every thread of the CTA
   }
   const bool fused = P.knew != nullptr && new_here_shard;
   const int newk = retrieval ? n - 1 - (int)P.shard_lo : (int)ring_slot(n - 1, P.S, P.R);  // its row
   const bool owns_new = fused && !split_head && newk >= k0 && newk < k1;
-  const int64_t in_off = ((int64_t)r * P.Hkv + kvh) * (int64_t)(D * 2);  // its K/V in the inputs (bf16)
+  // its K/V in the inputs (bf16); recomputed where used rather than held
+  // through the main loop
+  auto in_off = [&]() { return ((int64_t)r * P.Hkv + kvh) * (int64_t)(D * 2); };
   auto write_new = [&]() {  // one warp writes the new K and V rows into the cache
     const int64_t row = retrieval ? ret_row(P.ret, b, pidx, newk) : srow0() + newk;
     if constexpr (Q4) {
       // lane l quantises channels 4l .. 4l+3 of each row, as the append does
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint2 raw = ldg64(reinterpret_cast<const uint8_t *>(which ? P.vnew : P.knew) + in_off + 8 * lane);
+        const uint2 raw = ldg64(reinterpret_cast<const uint8_t *>(which ? P.vnew : P.knew) + in_off() + 8 * lane);
         const float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
                             __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u)};
         __half sch, zph;
@@ -320,7 +391,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       __syncwarp();
     } else {
       const int c = lane & 15;  // 16 lanes x 16 bytes = one 256-byte row
-      const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + in_off;
+      const uint8_t *src = reinterpret_cast<const uint8_t *>(lane < 16 ? P.knew : P.vnew) + in_off();
       uint8_t *dst = (lane < 16 ? (retrieval ? P.p.ret_k : P.p.str_k)
                                 : (retrieval ? P.p.ret_v : P.p.str_v)) + row * RB;
       reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
@@ -333,8 +404,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   float qsum = 0.f;  // sum of the query's channels (4-bit zero-point term)
   const bool live = g < G;
   const float sl2 = P.scale_log2;
-  // 4-bit: score (log2 units) = raw * (sc * c1) + zp * c2, raw = the MMA sum
-  float c1 = sl2, c2 = 0.f;
+  // 4-bit: score (log2 units) = raw * (sc * c1) + zp * c2, raw = the MMA sum;
+  // c2q: c2 of the queries 2t, 2t+1 this thread scores
+  float c1 = sl2, c2 = 0.f, c2q[2] = {0.f, 0.f};
   {
     const __nv_bfloat16 *qrow =
         reinterpret_cast<const __nv_bfloat16 *>(P.q) + ((int64_t)r * P.Hq + (int64_t)kvh * G + g) * D;
@@ -353,9 +425,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       }
       qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
       qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      // a power of two keeps |q| below 2^15 in f16 (taken back in c1)
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      // one power of two for all the CTA's queries keeps |q| below 2^15 in
+      // f16 (taken back in c1)
       const int ex = ((__float_as_int(amax) >> 23) & 0xff) - 127;
       const int eq = ex > 14 ? ex - 14 : 0;
       const float qs = exp2i(-eq), qs16 = qs * 0.0625f;
@@ -369,6 +442,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       }
       c1 = sl2 * kTwo24 * exp2i(eq);
       c2 = qsum * sl2;
+      // S^T: this thread scores queries 2t and 2t+1
+      c2q[0] = __shfl_sync(0xffffffffu, c2, (2 * t) << 2);
+      c2q[1] = __shfl_sync(0xffffffffu, c2, (2 * t + 1) << 2);
       if (warp == 0) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -403,11 +479,13 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   float o[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  // softmax state of query g (identical in the four threads of a row); for the
-  // 4-bit cache z = sum p*zp, and p is taken relative to m - f (f: headroom
-  // exponent, the same in every lane; at most 20, which the smallest scales
-  // allow)
-  float m = -INFINITY, l = 0.f, z = 0.f;
+  // bf16: softmax state of query g (identical in the four threads of a row).
+  // 4-bit: state of queries 2t and 2t+1 (m the same in the eight threads of a
+  // column; l and the zero-point sums z partial over this thread's keys), p
+  // taken relative to m - f (f: headroom exponent, the same in every lane; at
+  // most 20, which the smallest scales allow)
+  float m = -INFINITY, l = 0.f;
+  float mq[2] = {-INFINITY, -INFINITY}, lq[2] = {0.f, 0.f}, zq[2] = {0.f, 0.f};
   int f = 20;
 
   // bf16 cache, one warp: keys [kb0, kb0 + 16) below hi of the buffers Kx/Vx,
@@ -507,40 +585,59 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // 4-bit cache, one warp: keys [kb0, kb0 + 32) below hi, except `skip_key`.
   // The pointers are this thread's own starting points in the tile: K codes
   // at the tile's first row + g rows + 16t bytes, V codes at + 2t rows + 8g
-  // bytes, (scale, zero) rows at + 2t rows; every load of the tile is then an
+  // bytes, (scale, zero) rows at + g rows; every load of the tile is then an
   // immediate offset from one of them.  `full` as above; `gen` reads through
   // generic pointers (the staged new token).
-  auto tile_q4 = [&](auto full, auto gen, const uint8_t *Kt, const uint8_t *Vt, const uint8_t *Kst,
-                     const uint8_t *Vst, int kb0, int hi, int skip_key) {
+  auto tile_q4 = [&](auto full, auto src, const uint8_t *Kt, const uint8_t *Vt, const uint8_t *Kst,
+                     const uint8_t *Vst, int kb0, int hi, int skip_key, uint32_t slot) {
     constexpr bool FULL = decltype(full)::value;
-    constexpr bool GEN = decltype(gen)::value;
+    constexpr int SRC = decltype(src)::value;  // 0 global, 1 generic pointers, 2 staged (slot)
+    constexpr bool GEN = SRC == 1;
     // ------------------------------------------------------------ loads (all up front)
-    // group kg covers keys kb = kb0 + 16*kg ..: K codes of key kb + 8*nt + g
-    // (bytes 16t..16t+15: channels 32t..32t+31); (scale, zero) of keys
-    // kb + 8*nt + 2t, +1 (this thread's score columns); V codes of keys
-    // kb + {2t, 2t+1, 8+2t, 9+2t} at bytes 8g..8g+7 (channels 16g..16g+15).
+    // group kg covers keys kb = kb0 + 16*kg ..: K codes and (scale, zero) of
+    // keys kb + 8*h + g (this thread's rows of S^T; codes at bytes 16t..16t+15,
+    // channels 32t..32t+31); V codes of keys kb + {2t, 2t+1, 8+2t, 9+2t} at
+    // bytes 8g..8g+7 (channels 16g..16g+15).
     uint4 kr[KG][2];
-    uint2 ksz[KG][2], vsz[KG][2];
+    uint32_t ksz[KG][2], vsz[KG][2];
     uint2 vr[KG][4];
+    if constexpr (SRC == 2) {
+      static_assert(KG == 2 || SRC != 2, "the staged layout holds two key groups");
+      // this thread's chunks of the stage (see kQ4Chunks)
 #pragma unroll
-    for (int kg = 0; kg < KG; ++kg) {
-      const int kb = kb0 + 16 * kg;
+      for (int kg = 0; kg < KG; ++kg) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int r0 = 16 * kg + 8 * nt;  // tile row of this thread's group
-        const int key = kb + 8 * nt + g;
-        const bool ok = FULL || (key < hi && key != skip_key);
-        kr[kg][nt] = ok ? ld16<GEN>(Kt + r0 * RB) : make_uint4(0, 0, 0, 0);
-        const int key2 = kb + 8 * nt + 2 * t;
-        ksz[kg][nt] = (FULL || key2 < hi) ? ld8<GEN>(Kst + r0 * 4) : make_uint2(0, 0);
-        vsz[kg][nt] = (FULL || key2 < hi) ? ld8<GEN>(Vst + r0 * 4) : make_uint2(0, 0);
+        for (int h = 0; h < 2; ++h) kr[kg][h] = lds128(slot + (2 * kg + h) * kQ4Chunk);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint4 v = lds128(slot + (4 + 2 * kg + j) * kQ4Chunk);
+          vr[kg][2 * j] = make_uint2(v.x, v.y);
+          vr[kg][2 * j + 1] = make_uint2(v.z, v.w);
+        }
       }
+      const uint4 ks = lds128(slot + 8 * kQ4Chunk), vs = lds128(slot + 9 * kQ4Chunk);
+      ksz[0][0] = ks.x, ksz[0][1] = ks.y, ksz[1][0] = ks.z, ksz[1][1] = ks.w;
+      vsz[0][0] = vs.x, vsz[0][1] = vs.y, vsz[1][0] = vs.z, vsz[1][1] = vs.w;
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r0 = 16 * kg + (i & 1) + 8 * (i >> 1);
-        const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
-        const bool ok = FULL || (key < hi && key != skip_key);
-        vr[kg][i] = ok ? ld8<GEN>(Vt + r0 * RB) : make_uint2(0, 0);
+      for (int kg = 0; kg < KG; ++kg) {
+        const int kb = kb0 + 16 * kg;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r0 = 16 * kg + 8 * h;  // tile row of this thread's group
+          const int key = kb + 8 * h + g;
+          const bool ok = FULL || (key < hi && key != skip_key);
+          kr[kg][h] = ok ? ld16<GEN>(Kt + r0 * RB) : make_uint4(0, 0, 0, 0);
+          ksz[kg][h] = (FULL || key < hi) ? ld4<GEN>(Kst + r0 * 4) : 0u;
+          vsz[kg][h] = (FULL || key < hi) ? ld4<GEN>(Vst + r0 * 4) : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r0 = 16 * kg + (i & 1) + 8 * (i >> 1);
+          const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
+          const bool ok = FULL || (key < hi && key != skip_key);
+          vr[kg][i] = ok ? ld8<GEN>(Vt + r0 * RB) : make_uint2(0, 0);
+        }
       }
     }
     // ------------------------------------------------------------ headroom
@@ -549,96 +646,103 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     // f = 21 - E keeps p*sc < 2^15.  Positive fp16 values order as integers.
     uint32_t vm = 0;
 #pragma unroll
-    for (int kg = 0; kg < KG; ++kg)
+    for (int kg = 0; kg < KG; ++kg) vm = max(vm, max(vsz[kg][0] & 0xffffu, vsz[kg][1] & 0xffffu));
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) vm = __vmaxu2(vm, __vmaxu2(vsz[kg][nt].x, vsz[kg][nt].y));
-    vm &= 0xffffu;  // the scales (low halves)
-    vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, 1));
-    vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, 2));
+    for (int off = 4; off < 32; off <<= 1) vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, off));
     const int ftile = 21 - max((int)(vm >> 10), 1);
-    // ------------------------------------------------------------ S = Q K^T
-    float sc[KG][2][2];
+    // ------------------------------------------------------------ S^T = K Q^T
+    // A rows g / g+8 are keys kb + g / kb + 8 + g; k-slots follow the channel
+    // order of the query fragments (see the set-up)
+    float sc[KG][2][2];  // [group][key g / 8+g][query 2t / 2t+1]
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
       const int kb = kb0 + 16 * kg;
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t w0[4] = {kr[kg][0].x, kr[kg][0].y, kr[kg][0].z, kr[kg][0].w};
+      const uint32_t w1[4] = {kr[kg][1].x, kr[kg][1].y, kr[kg][1].z, kr[kg][1].w};
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t w4[4] = {kr[kg][nt].x, kr[kg][nt].y, kr[kg][nt].z, kr[kg][nt].w};
+      for (int w = 0; w < 4; ++w) {
+        const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
+        const uint32_t x0 = w0[w], x1 = w1[w], y0 = x0 >> 8, y1 = x1 >> 8;
+        mma16816_full_f16(s, x0 & kNib0, x1 & kNib0, x0 & kNib1, x1 & kNib1, qf.x, qf.y);
+        mma16816_full_f16(s, y0 & kNib0, y1 & kNib0, y0 & kNib1, y1 & kNib1, qf.z, qf.w);
+      }
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
-          const uint32_t x = w4[w], y = x >> 8;
-          mma16816_f16(s, qf.x, qf.y, x & kNib0, x & kNib1);
-          mma16816_f16(s, qf.z, qf.w, y & kNib0, y & kNib1);
-        }
-        // scores of query g at keys kb + 8*nt + 2t + e
-        const int key = kb + 8 * nt + 2 * t;
+      for (int h = 0; h < 2; ++h) {
+        const float2 kp = half2_bits_to_f2(ksz[kg][h]);  // (scale, zero)
+        const float a = kp.x * c1;
+        const int key = kb + 8 * h + g;
+        const bool valid = FULL || (key < hi && key != skip_key);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float2 kp = half2_bits_to_f2(e ? ksz[kg][nt].y : ksz[kg][nt].x);  // (scale, zero)
-          const float v = fmaf(s[e], kp.x * c1, kp.y * c2);
-          sc[kg][nt][e] = (FULL || (key + e < hi && key + e != skip_key)) ? v : -INFINITY;
-        }
+        for (int e = 0; e < 2; ++e)
+          sc[kg][h][e] = valid ? fmaf(s[2 * h + e], a, kp.y * c2q[e]) : -INFINITY;
       }
     }
     // ------------------------------------------------------------ online softmax
-    float mx = -INFINITY;
+    float mx[2];
 #pragma unroll
-    for (int kg = 0; kg < KG; ++kg)
-      mx = fmaxf(mx, fmaxf(fmaxf(sc[kg][0][0], sc[kg][0][1]), fmaxf(sc[kg][1][0], sc[kg][1][1])));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    // Rescale when the running max grows by more than 2^8 or the headroom
-    // must shrink (numerator and denominator scale together).
-    const bool grow = mx > m + 8.f || (m == -INFINITY && mx > -INFINITY);
+    for (int e = 0; e < 2; ++e) {
+      float x = -INFINITY;
+#pragma unroll
+      for (int kg = 0; kg < KG; ++kg) x = fmaxf(x, fmaxf(sc[kg][0][e], sc[kg][1][e]));
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+      mx[e] = x;
+    }
+    // Rescale when a running max grows by more than 2^8 or the headroom must
+    // shrink (numerator and denominator scale together).
+    bool grow[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) grow[e] = mx[e] > mq[e] + 8.f || (mq[e] == -INFINITY && mx[e] > -INFINITY);
     const bool shrink = ftile < f;  // the same in every lane
-    if (__any_sync(0xffffffffu, grow) || shrink) {
-      float alpha = 1.f;
-      if (grow) {
-        alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mx);
-        m = mx;
+    if (__any_sync(0xffffffffu, grow[0] || grow[1]) || shrink) {
+      float alpha[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        alpha[e] = 1.f;
+        if (grow[e]) {
+          alpha[e] = (mq[e] == -INFINITY) ? 0.f : fast_exp2(mq[e] - mx[e]);
+          mq[e] = mx[e];
+        }
+        if (shrink) alpha[e] *= exp2i(ftile - f);
+        lq[e] *= alpha[e];
+        zq[e] *= alpha[e];
       }
-      if (shrink) {
-        alpha *= exp2i(ftile - f);
-        f = ftile;
-      }
-      l *= alpha;
-      z *= alpha;
-      const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * t) << 2);
-      const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) << 2);
+      if (shrink) f = ftile;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        o[i][0] *= a0;
-        o[i][2] *= a0;
-        o[i][1] *= a1;
-        o[i][3] *= a1;
+        o[i][0] *= alpha[0];
+        o[i][2] *= alpha[0];
+        o[i][1] *= alpha[1];
+        o[i][3] *= alpha[1];
       }
     }
-    const float ref = m - (float)f;
+    const float ref[2] = {mq[0] - (float)f, mq[1] - (float)f};
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
-      float pv[2][2];
+      // p*sc per (key, query) as an f16 high part and residual, packed per key
+      // row of P (queries 2t, 2t+1), then transposed to P^T fragments
+      uint32_t ph[2], pl[2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
+      for (int h = 0; h < 2; ++h) {
+        const float2 vp = half2_bits_to_f2(vsz[kg][h]);  // (scale, zero)
+        float pv[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float x = sc[kg][nt][e];
-          // a full tile has finite scores in every row, so ref is finite
-          const float p = (FULL || x != -INFINITY) ? fast_exp2(x - ref) : 0.f;
-          const float2 vp = half2_bits_to_f2(e ? vsz[kg][nt].y : vsz[kg][nt].x);  // (scale, zero)
-          l += p;
-          z = fmaf(p, vp.y, z);
-          pv[nt][e] = p * vp.x;
+          const float x = sc[kg][h][e];
+          // a full tile has finite scores in every column, so ref is finite
+          const float p = (FULL || x != -INFINITY) ? fast_exp2(x - ref[e]) : 0.f;
+          lq[e] += p;
+          zq[e] = fmaf(p, vp.y, zq[e]);
+          pv[e] = p * vp.x;
         }
+        ph[h] = pack_f16(pv[0], pv[1]);
+        const float2 hf = half2_bits_to_f2(ph[h]);
+        pl[h] = pack_f16(pv[0] - hf.x, pv[1] - hf.y);
       }
-      // P^T fragment (p*sc as f16 high part and residual): b0 = keys 2t,
-      // 2t+1, b1 = keys 8+2t, 9+2t
-      const uint32_t pb0 = pack_f16(pv[0][0], pv[0][1]);
-      const uint32_t pb1 = pack_f16(pv[1][0], pv[1][1]);
-      const float2 h0 = half2_bits_to_f2(pb0), h1 = half2_bits_to_f2(pb1);
-      const uint32_t pl0 = pack_f16(pv[0][0] - h0.x, pv[0][1] - h0.y);
-      const uint32_t pl1 = pack_f16(pv[1][0] - h1.x, pv[1][1] - h1.y);
+      // P^T fragment: b0 = keys 2t, 2t+1, b1 = keys 8+2t, 9+2t, of query g
+      const uint32_t pb0 = movm_trans(ph[0]), pb1 = movm_trans(ph[1]);
+      const uint32_t pl0 = movm_trans(pl[0]), pl1 = movm_trans(pl[1]);
       // ---------------------------------------------------------- O^T += V^T P^T
       // A rows g / g+8 are channels vchan(mt) / vchan(mt)+1; cols are keys
       // (2t, 2t+1) from ab and (8+2t, 9+2t) from cd, two bytes (4 channels)
@@ -668,7 +772,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // that holds them (indices local to the block), streaming keys in the slot
   // buffer.
   // this thread's offsets within a 4-bit tile (see tile_q4)
-  const int k_off = g * RB + 16 * t, v_off = 2 * t * RB + 8 * g, s_off = 8 * t;
+  const int k_off = g * RB + 16 * t, v_off = 2 * t * RB + 8 * g, s_off = 4 * g;
   auto run_tile = [&](int kb0, int hi, int skip_key) {
     int64_t row;
     int base = 0;
@@ -690,9 +794,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       const uint8_t *Kt = pk + r * RB + k_off, *Vt = pv + r * RB + v_off;
       const uint8_t *Kst = psk + r * 4 + s_off, *Vst = psv + r * 4 + s_off;
       if (lo_k + T <= hi_k && (sk < lo_k || sk >= lo_k + T))
-        tile_q4(BoolC<true>{}, BoolC<false>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk);
+        tile_q4(BoolC<true>{}, IntC<0>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk, 0u);
       else
-        tile_q4(BoolC<false>{}, BoolC<false>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk);
+        tile_q4(BoolC<false>{}, IntC<0>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk, 0u);
     } else {
       tile(BoolC<false>{}, pk + row * RB, pv + row * RB, lo_k, hi_k, sk);
     }
@@ -718,24 +822,49 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     if constexpr (Q4) {
       if (!P.ret.table) {
         // Packed layout: the warp's tiles of its share lie NWARPS tiles apart
-        // in one contiguous page, so the walk only advances four pointers.
-        // Tiles holding the new token or the page's ragged end take the
-        // general path.
+        // in one contiguous page.  Its full tiles (all but the one holding
+        // the new token or the page's ragged end) stream through two
+        // shared-memory stages: each thread copies asynchronously exactly
+        // the bytes it will use, so the next tile is in flight while this
+        // one is computed, and no register holds a load in flight.
+        const int tend = min(t1, (keys - (fused ? 1 : 0)) / T);  // tiles below are full
         const int64_t r0 = ret_row(P.ret, b, pidx, (int64_t)tt * T);
+        // the next tile to copy
         const uint8_t *Kt = P.p.ret_k + r0 * RB + k_off, *Vt = P.p.ret_v + r0 * RB + v_off;
         const uint8_t *Kst = P.p.ret_k_sz + r0 * 4 + s_off, *Vst = P.p.ret_v_sz + r0 * 4 + s_off;
         constexpr int kStep = NWARPS * T;  // rows between a warp's tiles
-        for (; tt < t1; tt += NWARPS) {
-          if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
-          const int kb0 = tt * T;
-          if (kb0 + T <= keys && !(fused && newk >= kb0 && newk < kb0 + T))
-            tile_q4(BoolC<true>{}, BoolC<false>{}, Kt, Vt, Kst, Vst, kb0, keys, -1);
-          else
-            visit(tt);
+        const uint32_t slot0 = smem_u32(smem) + (uint32_t)tid * 16u;
+        auto issue = [&](int stage) {
+          const uint32_t sl = slot0 + (uint32_t)stage * kQ4Stage;
+#pragma unroll
+          for (int kg = 0; kg < KG; ++kg) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int rr = 16 * kg + 8 * h;
+              cp_async16(sl + (2 * kg + h) * kQ4Chunk, Kt + rr * RB);
+              cp_async4(sl + 8 * kQ4Chunk + 4 * (2 * kg + h), Kst + rr * 4);
+              cp_async4(sl + 9 * kQ4Chunk + 4 * (2 * kg + h), Vst + rr * 4);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              cp_async8(sl + (4 + 2 * kg + (i >> 1)) * kQ4Chunk + 8 * (i & 1),
+                        Vt + (16 * kg + (i & 1) + 8 * (i >> 1)) * RB);
+          }
+          cp_async_commit();
           Kt += kStep * RB;
           Vt += kStep * RB;
           Kst += kStep * 4;
           Vst += kStep * 4;
+        };
+        if (tt < tend) issue(0);
+        if (tt + NWARPS < tend) issue(1);
+        for (int stage = 0; tt < tend; tt += NWARPS, stage ^= 1) {
+          if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
+          if (tt + NWARPS < tend) cp_async_wait<1>();
+          else cp_async_wait<0>();
+          tile_q4(BoolC<true>{}, IntC<2>{}, nullptr, nullptr, nullptr, nullptr, tt * T, keys, -1,
+                  slot0 + (uint32_t)stage * kQ4Stage);
+          if (tt + 2 * NWARPS < tend) issue(stage);  // this stage is read (by this thread)
         }
       }
     }
@@ -758,32 +887,50 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     // the new token: key 0 of a one-row buffer, the inputs (bf16) or the
     // warp's quantised copy in shared memory (4-bit)
     if constexpr (Q4)
-      tile_q4(BoolC<false>{}, BoolC<true>{}, s_new + k_off, s_new + 64 + v_off, s_new + 128 + s_off,
-              s_new + 136 + s_off, 0, 1, -1);
+      tile_q4(BoolC<false>{}, IntC<1>{}, s_new + k_off, s_new + 64 + v_off, s_new + 128 + s_off,
+              s_new + 136 + s_off, 0, 1, -1, 0u);
     else
-      tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + in_off,
-           reinterpret_cast<const uint8_t *>(P.vnew) + in_off, 0, 1, -1);
+      tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + in_off(),
+           reinterpret_cast<const uint8_t *>(P.vnew) + in_off(), 0, 1, -1);
   }
 
   // the next kernel in the stream may start its set-up now
   asm volatile("griddepcontrol.launch_dependents;");
 
-  // ---- per-warp state -> shared memory (queries < G only)
-  l += __shfl_xor_sync(0xffffffffu, l, 1);
-  l += __shfl_xor_sync(0xffffffffu, l, 2);
-  if (Q4) {
-    z += __shfl_xor_sync(0xffffffffu, z, 1);
-    z += __shfl_xor_sync(0xffffffffu, z, 2);
-  }
+  // ---- per-warp state -> shared memory (queries < G only).  The 4-bit
+  // copy stages share this memory: every warp must be past its main loop.
+  if constexpr (Q4) __syncthreads();
   float *red_m = reinterpret_cast<float *>(smem);
   float *red_l = red_m + NWARPS * G;
   float *red_o = red_l + NWARPS * G;
   // the zero-point sums of this thread's two O^T columns (queries 2t, 2t+1)
-  const float z0 = __shfl_sync(0xffffffffu, z, (2 * t) << 2);
-  const float z1 = __shfl_sync(0xffffffffu, z, (2 * t + 1) << 2);
-  if (live && t == 0) {
-    red_m[warp * G + g] = Q4 ? m - (float)f : m;  // the reference of l and O
-    red_l[warp * G + g] = l;
+  float z0 = 0.f, z1 = 0.f;
+  if constexpr (Q4) {
+    // sums over the eight key rows g of each query column
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        lq[e] += __shfl_xor_sync(0xffffffffu, lq[e], off);
+        zq[e] += __shfl_xor_sync(0xffffffffu, zq[e], off);
+      }
+    z0 = zq[0];
+    z1 = zq[1];
+    if (g == 0) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (2 * t + e < G) {
+          red_m[warp * G + 2 * t + e] = mq[e] - (float)f;  // the reference of l and O
+          red_l[warp * G + 2 * t + e] = lq[e];
+        }
+    }
+  } else {
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (live && t == 0) {
+      red_m[warp * G + g] = m;
+      red_l[warp * G + g] = l;
+    }
   }
   // 4-bit: rows g carry u * 2^-24, rows g+8 16u * 2^-24
   const float e0 = Q4 ? kTwo24 : 1.f, e1 = Q4 ? kTwo20 : 1.f;
@@ -802,16 +949,29 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   }
   __syncthreads();
   decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(
-      P, smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
+      epi_ptrs(P), smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
       (int64_t)r * P.n_ret + pidx, (int64_t)(retrieval ? P.cta0[r] : 0) + (int64_t)pidx * nsplit,
       nsplit, split);
+  }
+  next_item:
+  if ((int)blockIdx.x < P.cta0[P.rows.n]) break;  // a retrieval CTA has one item
+  __syncthreads();  // the item's epilogue read shared memory; the counter moves on
+  if (tid == 0) ++s_item;
+  __syncthreads();
+  {
+    const int x = s_item, first = ((int)blockIdx.x - P.cta0[P.rows.n]) * P.str_per_cta;
+    if (x >= first + P.str_per_cta || x >= P.rows.n * P.n_str) break;
+  }
+  }  // items
 }
 
 template <bool Q4, int G>
 cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
   auto kern = decode_mma_kernel<Q4, G>;
-  // staging: 2*NWARPS*G + NWARPS*G*D floats; merge: nsplit*G + G (+align) + NWARPS*G*D floats
-  const int smem = (int)sizeof(float) * (kMaxSplits * G + 8 + NWARPS * G * D + 2 * NWARPS * G);
+  // staging: 2*NWARPS*G + NWARPS*G*D floats; merge: nsplit*G + G (+align) + NWARPS*G*D floats;
+  // 4-bit: the two copy stages of the main loop share the same memory
+  const int red = (int)sizeof(float) * (kMaxSplits * G + 8 + NWARPS * G * D + 2 * NWARPS * G);
+  const int smem = Q4 ? max(red, (int)(2 * kQ4Stage)) : red;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -829,7 +989,7 @@ cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
     cfg->num_sms = sms;
     return cudaSuccess;
   }
-  const int grid = d.cta0[d.rows.n] + d.rows.n * d.n_str;
+  const int grid = d.cta0[d.rows.n] + (d.rows.n * d.n_str + d.str_per_cta - 1) / d.str_per_cta;
   if (grid == 0) return cudaSuccess;
   if (!d.pdl) {
     kern<<<grid, NWARPS * 32, smem, s>>>(d);

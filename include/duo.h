@@ -105,7 +105,7 @@ typedef struct duo_cache_desc {
   int32_t n_kv_heads;  /* <= DUO_MAX_KV_HEADS, divides n_q_heads */
   int32_t head_dim;    /* 64 or 128 */
   int32_t kv_dtype;    /* duo_kv_dtype */
-  int64_t capacity;    /* max tokens of one row (INT4: rounded up to 4) */
+  int64_t capacity;    /* max tokens of one row (INT4: rounded up to 128) */
 } duo_cache_desc;
 
 typedef struct duo_cache duo_cache;
@@ -299,10 +299,9 @@ duo_status duo_decode_attn_static(duo_cache *cache, int32_t layer, const void *q
  * row's length, filled streaming slots) is first expanded to bf16, x = sc*u+zp
  * rounded to bf16, in the workspace (duo_prefill_workspace_bytes, 256-byte
  * aligned), which the tensor-core pass then reads; the chunk's own k/v enter
- * exactly as given.  The workspace must be zero-filled before its first use:
- * key tiles are 128 rows, so a tile can cover rows past a row's length whose
- * probabilities are 0, and those rows must hold finite values (zeros or an
- * earlier call's expansion) for 0 * value to stay 0.
+ * exactly as given.  Key tiles are 128 rows, so a tile can cover rows past a
+ * row's length (probability 0); the expansion writes zeros there, so the
+ * workspace needs no initialisation.
  * Errors: DUO_ERR_CAPACITY if len + C would pass capacity in a row;
  * DUO_ERR_WORKSPACE if an INT4 cache gets a missing or small workspace. */
 duo_status duo_prefill_attn(duo_cache *cache, int32_t layer, const void *q,

@@ -137,6 +137,10 @@ def test_int4_constant_rows_and_prefill_limits():
     assert (Kh == 0.75).all()
     ref = OA.decode_reference(f64(q), Kh, _dequant_history(V)[0], mask.numpy(), 2, 8)
     assert_parity(out, ref, "int4", "constant rows")
+    cap = cache.layout(0).capacity  # 4-bit caches round capacity up to one 128-key tile
+    assert cap == 128
+    zeros = torch.zeros(B, cap - n, Hkv, D, dtype=BF, device="cuda")
+    cache.append(0, zeros, zeros)
     with pytest.raises(DuoError) as e:  # the cache is full
         cache.prefill(0, torch.zeros(B, 8, Hq, D, dtype=BF, device="cuda"),
                       torch.zeros(B, 8, Hkv, D, dtype=BF, device="cuda"),

@@ -129,7 +129,10 @@ def _int4_view(x):
 @pytest.mark.parametrize("paged", [False, True])
 def test_prefill_int4_cache(B, Hq, Hkv, S, R, paged):
     """Chunks attend to a 4-bit cache (expanded to bf16 for the tensor cores)
-    plus their own bf16 k/v; the oracle reads the dequantised history exactly."""
+    plus their own bf16 k/v; the oracle reads the dequantised history exactly.
+    The expansion workspace starts full of NaN bytes: the library writes every
+    row the tensor-core pass reads (keys, then zeros to the tile's end), so the
+    caller needs no zero fill."""
     bounds = [(0, 300), (300, 812), (812, 1500)]
     n = bounds[-1][1]
     seed = 41 + Hkv + S
@@ -138,6 +141,8 @@ def test_prefill_int4_cache(B, Hq, Hkv, S, R, paged):
     kw = dict(pool_blocks=B * 8) if paged else {}
     cache = DuoCache(1, B, Hq, Hkv, 128, "int4", n, mask[None], S, R, **kw)
     assert cache.prefill_ws_bytes > 0
+    cache._prefill_ws()
+    cache._pf_ws.fill_(0xFF)  # every bf16 in it is a NaN
     outs = _run_chunks(cache, Q, K, V, bounds)
     Kq, Vq = _int4_view(K), _int4_view(V)
     for (c0, o), (_, c1) in zip(outs, bounds):
