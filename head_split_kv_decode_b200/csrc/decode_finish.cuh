@@ -9,47 +9,24 @@
 
 namespace duo {
 
-// The pointers the epilogue writes through, read from the kernel parameters
-// in one place.
-struct EpiPtrs {
-  void *out;
-  float *part_o, *part_lse;
-  float *ws_o, *ws_lse;
-  unsigned *ws_cnt, *ws_next;
-  int out_f32;
-};
-
-__device__ __forceinline__ EpiPtrs epi_ptrs(const DecodeParams &P) {
-  EpiPtrs e;
-  e.out = P.out;
-  e.part_o = P.part_o;
-  e.part_lse = P.part_lse;
-  e.ws_o = P.ws_o;
-  e.ws_lse = P.ws_lse;
-  e.ws_cnt = P.ws_cnt;
-  e.ws_next = P.ws_next;
-  e.out_f32 = P.out_f32;
-  return e;
-}
-
 // Second half of the epilogue: the per-warp states of the CTA are staged in
 // shared memory as red_m [NWARPS][G], red_l [NWARPS][G] (log2 units) and
 // red_o [NWARPS][G][D] (unnormalised), all starting at `smem`.  Combines them,
 // writes the result of this KV head's G query heads (rows out_row ..
-// out_row + G - 1 of the output, or of E.part_o / E.part_lse in partial mode)
+// out_row + G - 1 of the output, or of P.part_o / P.part_lse in partial mode)
 // when `direct`, or else this split's normalised partial and log-sum-exp
 // into slot part0 + split, and lets the last of the nsplit splits of the head
 // (merge ticket `unit`) merge slots part0 .. part0 + nsplit - 1.
 template <typename T, int D, int G, int NWARPS>
-__device__ __forceinline__ void decode_reduce_store(const EpiPtrs &E, uint8_t *smem,
+__device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8_t *smem,
                                                     int *s_last_p, bool direct, int64_t out_row,
                                                     int64_t unit, int64_t part0, int nsplit,
                                                     int split) {
   constexpr float kLn2 = 0.6931471805599453f;  // log-sum-exps leave in natural log
-  // output element i of this head's rows, as T or (E.out_f32) as float
+  // output element i of this head's rows, as T or (P.out_f32) as float
   auto put = [&](int i, float v) {
-    if (E.out_f32) reinterpret_cast<float *>(E.out)[out_row * D + i] = v;
-    else store_out(reinterpret_cast<T *>(E.out) + out_row * D + i, v);
+    if (P.out_f32) reinterpret_cast<float *>(P.out)[out_row * D + i] = v;
+    else store_out(reinterpret_cast<T *>(P.out) + out_row * D + i, v);
   };
   constexpr int NT = NWARPS * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -75,17 +52,17 @@ __device__ __forceinline__ void decode_reduce_store(const EpiPtrs &E, uint8_t *s
     float O = 0.f;
 #pragma unroll
     for (int w = 0; w < NWARPS; ++w) O += red_o[(w * G + g) * D + c] * __shfl_sync(0xffffffffu, sw, w);
-    if (direct && E.part_o) {
+    if (direct && P.part_o) {
       const bool empty = L == 0.f;  // this shard holds no key of the head
-      E.part_o[(out_row + g) * D + c] = empty ? 0.f : O / L;
-      if (c == 0) E.part_lse[out_row + g] = empty ? -INFINITY : (M + fast_log2(L)) * kLn2;
+      P.part_o[(out_row + g) * D + c] = empty ? 0.f : O / L;
+      if (c == 0) P.part_lse[out_row + g] = empty ? -INFINITY : (M + fast_log2(L)) * kLn2;
     } else if (direct) {
       put(g * D + c, O / L);
     } else {
       // a split whose CTA claimed no keys leaves weight zero (lse -inf)
       const bool empty = L == 0.f;
-      E.ws_o[(part * G + g) * D + c] = empty ? 0.f : O / L;
-      if (c == 0) E.ws_lse[part * G + g] = empty ? -INFINITY : M + fast_log2(L);
+      P.ws_o[(part * G + g) * D + c] = empty ? 0.f : O / L;
+      if (c == 0) P.ws_lse[part * G + g] = empty ? -INFINITY : M + fast_log2(L);
     }
   }
   if (direct) return;
@@ -96,7 +73,7 @@ __device__ __forceinline__ void decode_reduce_store(const EpiPtrs &E, uint8_t *s
   // the last ticket fences again before the barrier that lets its threads
   // read the other splits' partials.
   __syncthreads();
-  unsigned *cnt = E.ws_cnt + unit;
+  unsigned *cnt = P.ws_cnt + unit;
   if (tid == 0) {
     __threadfence();
     s_last = (atomicAdd(cnt, 1u) == (unsigned)(nsplit - 1));
@@ -117,7 +94,7 @@ __device__ __forceinline__ void decode_reduce_store(const EpiPtrs &E, uint8_t *s
   constexpr int L4 = D / 4;
   constexpr int U = G >= 8 ? 2 : 4;
   const bool owns = lane < L4;
-  const float4 *src = reinterpret_cast<const float4 *>(E.ws_o + part0 * G * D) + (owns ? lane : 0);
+  const float4 *src = reinterpret_cast<const float4 *>(P.ws_o + part0 * G * D) + (owns ? lane : 0);
   const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 v[U][G];
 #pragma unroll
@@ -132,7 +109,7 @@ __device__ __forceinline__ void decode_reduce_store(const EpiPtrs &E, uint8_t *s
   for (int g = warp; g < G; g += NWARPS) {
     float M = -INFINITY;
     for (int sp = lane; sp < nsplit; sp += 32) {
-      const float x = __ldcg(E.ws_lse + (part0 + sp) * G + g);
+      const float x = __ldcg(P.ws_lse + (part0 + sp) * G + g);
       s_w[sp * G + g] = x;
       M = fmaxf(M, x);
     }
@@ -191,16 +168,16 @@ __device__ __forceinline__ void decode_reduce_store(const EpiPtrs &E, uint8_t *s
     float num = 0.f;
 #pragma unroll
     for (int w = 0; w < NWARPS; ++w) num += s_acc[(w * G + g) * D + c];
-    if (E.part_o) {
-      E.part_o[(out_row + g) * D + c] = num / s_den[g];
-      if (c == 0) E.part_lse[out_row + g] = (s_mx[g] + fast_log2(s_den[g])) * kLn2;
+    if (P.part_o) {
+      P.part_o[(out_row + g) * D + c] = num / s_den[g];
+      if (c == 0) P.part_lse[out_row + g] = (s_mx[g] + fast_log2(s_den[g])) * kLn2;
     } else {
       put(g * D + c, num / s_den[g]);
     }
   }
   if (tid == 0) {  // leave the ticket (and chunk counter) ready for the next call
     *cnt = 0u;
-    if (E.ws_next) E.ws_next[unit * kChunkCounterStride] = 0u;
+    if (P.ws_next) P.ws_next[unit * kChunkCounterStride] = 0u;
   }
 }
 
@@ -259,7 +236,7 @@ __device__ __forceinline__ void decode_finish(const DecodeParams &P, uint8_t *sm
   // CUDA-core decode: packed layout, every batch row at length P.n, the
   // retrieval CTAs enumerated as ((b*n_ret + head)*nsplit + split).
   const int64_t unit = (int64_t)b * P.n_ret + (retrieval ? pidx : 0);
-  decode_reduce_store<T, D, G, NWARPS>(epi_ptrs(P), smem, s_last_p, !retrieval || P.nsplit == 1,
+  decode_reduce_store<T, D, G, NWARPS>(P, smem, s_last_p, !retrieval || P.nsplit == 1,
                                        (int64_t)b * P.Hq + (int64_t)kvh * G, unit,
                                        unit * P.nsplit, P.nsplit, split);
 }

@@ -126,42 +126,10 @@ __device__ __forceinline__ uint32_t ld4(const uint8_t *p) {
   return v;
 }
 
-// Per-thread asynchronous copies global -> shared (no registers held while in
-// flight); completion is per thread, tracked by commit groups.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-
 template <int N>
 struct IntC {
   static constexpr int value = N;
 };
-
-// 4-bit decode, copies staged in shared memory: each thread owns 10 chunks of
-// 16 bytes per stage (K codes of its 4 key rows; V codes of its 8 key rows, 8
-// bytes each; the (scale, zero) words of its 4 key rows for K and for V),
-// chunk c of thread i at (c * threads + i) * 16, so that the 16-byte reads of
-// a quarter-warp are contiguous.  Two stages.
-constexpr int kQ4Chunks = 10;
-constexpr uint32_t kQ4Chunk = NWARPS * 32 * 16;      // bytes between a thread's chunks
-constexpr uint32_t kQ4Stage = kQ4Chunks * kQ4Chunk;  // bytes per stage
 
 // Transpose of an 8x8 matrix of 16-bit elements held as the warp's
 // fragments (thread 4i+j holds row i, columns 2j and 2j+1).
@@ -227,19 +195,8 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
-  // ---- work items: retrieval CTAs first (launch row r, head, split), one
-  // item each; then streaming CTAs, each taking P.str_per_cta consecutive
-  // (launch row, streaming head) items in turn (a streaming head's window is
-  // short, so one CTA per head would leave SMs idle that retrieval splits can
-  // use)
-  // The item counter of a streaming CTA lives in shared memory, so that no
-  // register carries it through the body.
-  __shared__ int s_item;
-  if (tid == 0)
-    s_item = (int)blockIdx.x < P.cta0[P.rows.n] ? 0
-                                                 : ((int)blockIdx.x - P.cta0[P.rows.n]) * P.str_per_cta;
-  __syncthreads();
-  for (;;) {
+  // ---- work item: retrieval CTAs first (launch row r, head, split), then
+  // one CTA per (launch row, streaming head)
   const int n_ret_ctas = P.cta0[P.rows.n];
   int r, kvh, pidx, split, nsplit;
   bool retrieval;
@@ -257,7 +214,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     kvh = P.h.ret_heads[pidx];
     retrieval = true;
   } else {
-    const int x = s_item;
+    const int x = (int)blockIdx.x - n_ret_ctas;
     r = x / P.n_str;
     pidx = x % P.n_str;
     kvh = P.h.str_heads[pidx];
@@ -265,7 +222,6 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     split = 0;
     nsplit = 1;
   }
-  {  // the item
   const int b = P.rows.row[r];
   // Key indices and tile counts are 32-bit (a row holds fewer than 2^31
   // tokens); byte offsets are formed in 64 bits.
@@ -355,7 +311,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     const int64_t row0 = (int64_t)r * P.Hq + (int64_t)kvh * G;
     for (int i = tid; i < G * D; i += NWARPS * 32) P.part_o[row0 * D + i] = 0.f;
     if (tid < G) P.part_lse[row0 + tid] = -INFINITY;
-    goto next_item;  // the same for every thread of the CTA
+    return;
   }
   const bool fused = P.knew != nullptr && new_here_shard;
   const int newk = retrieval ? n - 1 - (int)P.shard_lo : (int)ring_slot(n - 1, P.S, P.R);  // its row
@@ -588,58 +544,63 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // bytes, (scale, zero) rows at + g rows; every load of the tile is then an
   // immediate offset from one of them.  `full` as above; `gen` reads through
   // generic pointers (the staged new token).
-  auto tile_q4 = [&](auto full, auto src, const uint8_t *Kt, const uint8_t *Vt, const uint8_t *Kst,
-                     const uint8_t *Vst, int kb0, int hi, int skip_key, uint32_t slot) {
+  // Registers of one 4-bit tile: K codes and (scale, zero) of keys
+  // kb + 8*h + g (this thread's rows of S^T; codes at bytes 16t..16t+15,
+  // channels 32t..32t+31); V codes of keys kb + {2t, 2t+1, 8+2t, 9+2t} at
+  // bytes 8g..8g+7 (channels 16g..16g+15); group kg covers keys
+  // kb = kb0 + 16*kg.  The K part is dead once the scores are computed, the
+  // V part once O is updated, so a pipelined walk refills each as it dies.
+  uint4 kr[KG][2];
+  uint32_t ksz[KG][2], vsz[KG][2];
+  uint2 vr[KG][4];
+  // Loads of a 4-bit tile, keys [kb0, kb0 + 32) below hi except `skip_key`.
+  // The pointers are this thread's own starting points in the tile: K codes
+  // at the tile's first row + g rows + 16t bytes, V codes at + 2t rows + 8g
+  // bytes, (scale, zero) rows at + g rows; every load of the tile is then an
+  // immediate offset from one of them.  `full` promises that all keys lie
+  // below hi and none is skip_key; `src` 1 reads through generic pointers
+  // (the staged new token), 0 through the read-only global path.
+  auto q4_load_k = [&](auto full, auto src, const uint8_t *Kt, const uint8_t *Kst, int kb0, int hi,
+                       int skip_key) {
     constexpr bool FULL = decltype(full)::value;
-    constexpr int SRC = decltype(src)::value;  // 0 global, 1 generic pointers, 2 staged (slot)
-    constexpr bool GEN = SRC == 1;
-    // ------------------------------------------------------------ loads (all up front)
-    // group kg covers keys kb = kb0 + 16*kg ..: K codes and (scale, zero) of
-    // keys kb + 8*h + g (this thread's rows of S^T; codes at bytes 16t..16t+15,
-    // channels 32t..32t+31); V codes of keys kb + {2t, 2t+1, 8+2t, 9+2t} at
-    // bytes 8g..8g+7 (channels 16g..16g+15).
-    uint4 kr[KG][2];
-    uint32_t ksz[KG][2], vsz[KG][2];
-    uint2 vr[KG][4];
-    if constexpr (SRC == 2) {
-      static_assert(KG == 2 || SRC != 2, "the staged layout holds two key groups");
-      // this thread's chunks of the stage (see kQ4Chunks)
+    constexpr bool GEN = decltype(src)::value == 1;
 #pragma unroll
-      for (int kg = 0; kg < KG; ++kg) {
+    for (int kg = 0; kg < KG; ++kg)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) kr[kg][h] = lds128(slot + (2 * kg + h) * kQ4Chunk);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint4 v = lds128(slot + (4 + 2 * kg + j) * kQ4Chunk);
-          vr[kg][2 * j] = make_uint2(v.x, v.y);
-          vr[kg][2 * j + 1] = make_uint2(v.z, v.w);
-        }
+      for (int h = 0; h < 2; ++h) {
+        const int r0 = 16 * kg + 8 * h;  // tile row of this thread's group
+        const int key = kb0 + r0 + g;
+        const bool ok = FULL || (key < hi && key != skip_key);
+        kr[kg][h] = ok ? ld16<GEN>(Kt + r0 * RB) : make_uint4(0, 0, 0, 0);
+        ksz[kg][h] = (FULL || key < hi) ? ld4<GEN>(Kst + r0 * 4) : 0u;
       }
-      const uint4 ks = lds128(slot + 8 * kQ4Chunk), vs = lds128(slot + 9 * kQ4Chunk);
-      ksz[0][0] = ks.x, ksz[0][1] = ks.y, ksz[1][0] = ks.z, ksz[1][1] = ks.w;
-      vsz[0][0] = vs.x, vsz[0][1] = vs.y, vsz[1][0] = vs.z, vsz[1][1] = vs.w;
-    } else {
+  };
+  auto q4_load_v = [&](auto full, auto src, const uint8_t *Vt, const uint8_t *Vst, int kb0, int hi,
+                       int skip_key) {
+    constexpr bool FULL = decltype(full)::value;
+    constexpr bool GEN = decltype(src)::value == 1;
 #pragma unroll
-      for (int kg = 0; kg < KG; ++kg) {
-        const int kb = kb0 + 16 * kg;
+    for (int kg = 0; kg < KG; ++kg) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r0 = 16 * kg + 8 * h;  // tile row of this thread's group
-          const int key = kb + 8 * h + g;
-          const bool ok = FULL || (key < hi && key != skip_key);
-          kr[kg][h] = ok ? ld16<GEN>(Kt + r0 * RB) : make_uint4(0, 0, 0, 0);
-          ksz[kg][h] = (FULL || key < hi) ? ld4<GEN>(Kst + r0 * 4) : 0u;
-          vsz[kg][h] = (FULL || key < hi) ? ld4<GEN>(Vst + r0 * 4) : 0u;
-        }
+      for (int h = 0; h < 2; ++h) {
+        const int r0 = 16 * kg + 8 * h;
+        vsz[kg][h] = (FULL || kb0 + r0 + g < hi) ? ld4<GEN>(Vst + r0 * 4) : 0u;
+      }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r0 = 16 * kg + (i & 1) + 8 * (i >> 1);
-          const int key = kb + 2 * t + (i & 1) + 8 * (i >> 1);
-          const bool ok = FULL || (key < hi && key != skip_key);
-          vr[kg][i] = ok ? ld8<GEN>(Vt + r0 * RB) : make_uint2(0, 0);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const int r0 = 16 * kg + (i & 1) + 8 * (i >> 1);
+        const int key = kb0 + 16 * kg + 2 * t + (i & 1) + 8 * (i >> 1);
+        const bool ok = FULL || (key < hi && key != skip_key);
+        vr[kg][i] = ok ? ld8<GEN>(Vt + r0 * RB) : make_uint2(0, 0);
       }
     }
+  };
+  // Scores of the loaded tile (S^T = K Q^T, log2 units; -inf where not
+  // visible) and the tile's headroom exponent.
+  float sc[KG][2][2];  // [group][key g / 8+g][query 2t / 2t+1]
+  int ftile = 0;
+  auto q4_scores = [&](auto full, int kb0, int hi, int skip_key) {
+    constexpr bool FULL = decltype(full)::value;
     // ------------------------------------------------------------ headroom
     // The largest V scale of the tile bounds p*sc: with p < 2^(8+f) (the lazy
     // rescale below) and sc < 2^(E-14) for an fp16 exponent field E >= 1,
@@ -649,24 +610,28 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     for (int kg = 0; kg < KG; ++kg) vm = max(vm, max(vsz[kg][0] & 0xffffu, vsz[kg][1] & 0xffffu));
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-    const int ftile = 21 - max((int)(vm >> 10), 1);
+    ftile = 21 - max((int)(vm >> 10), 1);
     // ------------------------------------------------------------ S^T = K Q^T
     // A rows g / g+8 are keys kb + g / kb + 8 + g; k-slots follow the channel
     // order of the query fragments (see the set-up)
-    float sc[KG][2][2];  // [group][key g / 8+g][query 2t / 2t+1]
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
       const int kb = kb0 + 16 * kg;
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      // two accumulators (channels 32t..32t+15 and +16..+31) halve the chain
+      // of dependent products
+      float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t w0[4] = {kr[kg][0].x, kr[kg][0].y, kr[kg][0].z, kr[kg][0].w};
       const uint32_t w1[4] = {kr[kg][1].x, kr[kg][1].y, kr[kg][1].z, kr[kg][1].w};
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
         const uint32_t x0 = w0[w], x1 = w1[w], y0 = x0 >> 8, y1 = x1 >> 8;
-        mma16816_full_f16(s, x0 & kNib0, x1 & kNib0, x0 & kNib1, x1 & kNib1, qf.x, qf.y);
-        mma16816_full_f16(s, y0 & kNib0, y1 & kNib0, y0 & kNib1, y1 & kNib1, qf.z, qf.w);
+        float(&acc)[4] = w < 2 ? s : s2;
+        mma16816_full_f16(acc, x0 & kNib0, x1 & kNib0, x0 & kNib1, x1 & kNib1, qf.x, qf.y);
+        mma16816_full_f16(acc, y0 & kNib0, y1 & kNib0, y0 & kNib1, y1 & kNib1, qf.z, qf.w);
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[i] += s2[i];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float2 kp = half2_bits_to_f2(ksz[kg][h]);  // (scale, zero)
@@ -678,7 +643,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
           sc[kg][h][e] = valid ? fmaf(s[2 * h + e], a, kp.y * c2q[e]) : -INFINITY;
       }
     }
-    // ------------------------------------------------------------ online softmax
+  };
+  // Online softmax of the scored tile, then O^T += V^T P^T.
+  auto q4_update = [&](auto full) {
+    constexpr bool FULL = decltype(full)::value;
     float mx[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -767,6 +735,14 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       }
     }
   };
+  // One 4-bit tile (pointers as for the loads).
+  auto tile_q4 = [&](auto full, auto src, const uint8_t *Kt, const uint8_t *Vt, const uint8_t *Kst,
+                     const uint8_t *Vst, int kb0, int hi, int skip_key) {
+    q4_load_k(full, src, Kt, Kst, kb0, hi, skip_key);
+    q4_load_v(full, src, Vt, Vst, kb0, hi, skip_key);
+    q4_scores(full, kb0, hi, skip_key);
+    q4_update(full);
+  };
 
   // A tile of keys [kb0, kb0 + T) below hi: retrieval keys through the block
   // that holds them (indices local to the block), streaming keys in the slot
@@ -794,9 +770,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       const uint8_t *Kt = pk + r * RB + k_off, *Vt = pv + r * RB + v_off;
       const uint8_t *Kst = psk + r * 4 + s_off, *Vst = psv + r * 4 + s_off;
       if (lo_k + T <= hi_k && (sk < lo_k || sk >= lo_k + T))
-        tile_q4(BoolC<true>{}, IntC<0>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk, 0u);
+        tile_q4(BoolC<true>{}, IntC<0>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk);
       else
-        tile_q4(BoolC<false>{}, IntC<0>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk, 0u);
+        tile_q4(BoolC<false>{}, IntC<0>{}, Kt, Vt, Kst, Vst, lo_k, hi_k, sk);
     } else {
       tile(BoolC<false>{}, pk + row * RB, pv + row * RB, lo_k, hi_k, sk);
     }
@@ -822,49 +798,36 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     if constexpr (Q4) {
       if (!P.ret.table) {
         // Packed layout: the warp's tiles of its share lie NWARPS tiles apart
-        // in one contiguous page.  Its full tiles (all but the one holding
-        // the new token or the page's ragged end) stream through two
-        // shared-memory stages: each thread copies asynchronously exactly
-        // the bytes it will use, so the next tile is in flight while this
-        // one is computed, and no register holds a load in flight.
+        // in one contiguous page, so the walk only advances four pointers.
+        // Its full tiles (all but one holding the new token or the page's
+        // ragged end, which take the general path) are software-pipelined
+        // in the tile's own registers: the next tile's K part is loaded as
+        // soon as this tile's scores are computed, its V part as soon as O
+        // is updated, so each load has half a tile of work to arrive.
         const int tend = min(t1, (keys - (fused ? 1 : 0)) / T);  // tiles below are full
         const int64_t r0 = ret_row(P.ret, b, pidx, (int64_t)tt * T);
-        // the next tile to copy
         const uint8_t *Kt = P.p.ret_k + r0 * RB + k_off, *Vt = P.p.ret_v + r0 * RB + v_off;
         const uint8_t *Kst = P.p.ret_k_sz + r0 * 4 + s_off, *Vst = P.p.ret_v_sz + r0 * 4 + s_off;
         constexpr int kStep = NWARPS * T;  // rows between a warp's tiles
-        const uint32_t slot0 = smem_u32(smem) + (uint32_t)tid * 16u;
-        auto issue = [&](int stage) {
-          const uint32_t sl = slot0 + (uint32_t)stage * kQ4Stage;
-#pragma unroll
-          for (int kg = 0; kg < KG; ++kg) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int rr = 16 * kg + 8 * h;
-              cp_async16(sl + (2 * kg + h) * kQ4Chunk, Kt + rr * RB);
-              cp_async4(sl + 8 * kQ4Chunk + 4 * (2 * kg + h), Kst + rr * 4);
-              cp_async4(sl + 9 * kQ4Chunk + 4 * (2 * kg + h), Vst + rr * 4);
+        if (tt < tend) {
+          q4_load_k(BoolC<true>{}, IntC<0>{}, Kt, Kst, 0, 0, -1);
+          q4_load_v(BoolC<true>{}, IntC<0>{}, Vt, Vst, 0, 0, -1);
+          for (; tt < tend; tt += NWARPS) {
+            // (the pool claim belongs to the last tile of the share: only
+            // then can the condition hold)
+            if (pooled && tt + NWARPS >= t1) {
+              if (lane == 0) c = atomicAdd(next, 1u);
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              cp_async8(sl + (4 + 2 * kg + (i >> 1)) * kQ4Chunk + 8 * (i & 1),
-                        Vt + (16 * kg + (i & 1) + 8 * (i >> 1)) * RB);
+            const bool more = tt + NWARPS < tend;
+            q4_scores(BoolC<true>{}, tt * T, keys, -1);
+            Kt += kStep * RB;
+            Kst += kStep * 4;
+            if (more) q4_load_k(BoolC<true>{}, IntC<0>{}, Kt, Kst, 0, 0, -1);
+            q4_update(BoolC<true>{});
+            Vt += kStep * RB;
+            Vst += kStep * 4;
+            if (more) q4_load_v(BoolC<true>{}, IntC<0>{}, Vt, Vst, 0, 0, -1);
           }
-          cp_async_commit();
-          Kt += kStep * RB;
-          Vt += kStep * RB;
-          Kst += kStep * 4;
-          Vst += kStep * 4;
-        };
-        if (tt < tend) issue(0);
-        if (tt + NWARPS < tend) issue(1);
-        for (int stage = 0; tt < tend; tt += NWARPS, stage ^= 1) {
-          if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
-          if (tt + NWARPS < tend) cp_async_wait<1>();
-          else cp_async_wait<0>();
-          tile_q4(BoolC<true>{}, IntC<2>{}, nullptr, nullptr, nullptr, nullptr, tt * T, keys, -1,
-                  slot0 + (uint32_t)stage * kQ4Stage);
-          if (tt + 2 * NWARPS < tend) issue(stage);  // this stage is read (by this thread)
         }
       }
     }
@@ -888,7 +851,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     // warp's quantised copy in shared memory (4-bit)
     if constexpr (Q4)
       tile_q4(BoolC<false>{}, IntC<1>{}, s_new + k_off, s_new + 64 + v_off, s_new + 128 + s_off,
-              s_new + 136 + s_off, 0, 1, -1, 0u);
+              s_new + 136 + s_off, 0, 1, -1);
     else
       tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + in_off(),
            reinterpret_cast<const uint8_t *>(P.vnew) + in_off(), 0, 1, -1);
@@ -897,9 +860,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // the next kernel in the stream may start its set-up now
   asm volatile("griddepcontrol.launch_dependents;");
 
-  // ---- per-warp state -> shared memory (queries < G only).  The 4-bit
-  // copy stages share this memory: every warp must be past its main loop.
-  if constexpr (Q4) __syncthreads();
+  // ---- per-warp state -> shared memory (queries < G only)
   float *red_m = reinterpret_cast<float *>(smem);
   float *red_l = red_m + NWARPS * G;
   float *red_o = red_l + NWARPS * G;
@@ -932,46 +893,34 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       red_l[warp * G + g] = l;
     }
   }
-  // 4-bit: rows g carry u * 2^-24, rows g+8 16u * 2^-24
-  const float e0 = Q4 ? kTwo24 : 1.f, e1 = Q4 ? kTwo20 : 1.f;
+  // 4-bit: rows g carry u * 2^-24, rows g+8 16u * 2^-24, plus the zero-point
+  // term; bf16: the accumulators as they are
+  auto fin = [&](float x, float e, float zz) { return Q4 ? fmaf(x, e, zz) : x; };
   const int q0 = 2 * t, q1 = 2 * t + 1;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) {
     const int ch = vchan(mt);
     if (q0 < G) {
-      red_o[(warp * G + q0) * D + ch] = fmaf(o[mt][0], e0, z0);
-      red_o[(warp * G + q0) * D + ch + 1] = fmaf(o[mt][2], e1, z0);
+      red_o[(warp * G + q0) * D + ch] = fin(o[mt][0], kTwo24, z0);
+      red_o[(warp * G + q0) * D + ch + 1] = fin(o[mt][2], kTwo20, z0);
     }
     if (q1 < G) {
-      red_o[(warp * G + q1) * D + ch] = fmaf(o[mt][1], e0, z1);
-      red_o[(warp * G + q1) * D + ch + 1] = fmaf(o[mt][3], e1, z1);
+      red_o[(warp * G + q1) * D + ch] = fin(o[mt][1], kTwo24, z1);
+      red_o[(warp * G + q1) * D + ch + 1] = fin(o[mt][3], kTwo20, z1);
     }
   }
   __syncthreads();
   decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(
-      epi_ptrs(P), smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
+      P, smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
       (int64_t)r * P.n_ret + pidx, (int64_t)(retrieval ? P.cta0[r] : 0) + (int64_t)pidx * nsplit,
       nsplit, split);
-  }
-  next_item:
-  if ((int)blockIdx.x < P.cta0[P.rows.n]) break;  // a retrieval CTA has one item
-  __syncthreads();  // the item's epilogue read shared memory; the counter moves on
-  if (tid == 0) ++s_item;
-  __syncthreads();
-  {
-    const int x = s_item, first = ((int)blockIdx.x - P.cta0[P.rows.n]) * P.str_per_cta;
-    if (x >= first + P.str_per_cta || x >= P.rows.n * P.n_str) break;
-  }
-  }  // items
 }
 
 template <bool Q4, int G>
 cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
   auto kern = decode_mma_kernel<Q4, G>;
-  // staging: 2*NWARPS*G + NWARPS*G*D floats; merge: nsplit*G + G (+align) + NWARPS*G*D floats;
-  // 4-bit: the two copy stages of the main loop share the same memory
-  const int red = (int)sizeof(float) * (kMaxSplits * G + 8 + NWARPS * G * D + 2 * NWARPS * G);
-  const int smem = Q4 ? max(red, (int)(2 * kQ4Stage)) : red;
+  // staging: 2*NWARPS*G + NWARPS*G*D floats; merge: nsplit*G + G (+align) + NWARPS*G*D floats
+  const int smem = (int)sizeof(float) * (kMaxSplits * G + 8 + NWARPS * G * D + 2 * NWARPS * G);
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -989,7 +938,7 @@ cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
     cfg->num_sms = sms;
     return cudaSuccess;
   }
-  const int grid = d.cta0[d.rows.n] + (d.rows.n * d.n_str + d.str_per_cta - 1) / d.str_per_cta;
+  const int grid = d.cta0[d.rows.n] + d.rows.n * d.n_str;
   if (grid == 0) return cudaSuccess;
   if (!d.pdl) {
     kern<<<grid, NWARPS * 32, smem, s>>>(d);

@@ -199,36 +199,14 @@ int choose_splits(const duo_cache *c, int layer, int64_t n, const duo::DecodeCon
   return (int)want;
 }
 
-// Tensor-core decode: (launch row, streaming head) items per streaming CTA.
-// A streaming head's window is short, so one CTA per head would leave SMs
-// with little to do; instead the streaming CTAs get a share of the SMs in
-// proportion to the streaming keys (at least one CTA), and each takes its
-// items in turn.  lens: each launch row's length (the query included).
-int str_items_per_cta(const duo_cache *c, int layer, const int32_t *lens, int nrows,
-                      const duo::DecodeConfig &cfg) {
-  const auto &L = c->layers[layer];
-  const int64_t items = (int64_t)nrows * L.n_str;
-  if (items == 0) return 1;
-  int64_t ret_keys = 0, str_keys = 0;
-  for (int r = 0; r < nrows; ++r) {
-    const int64_t n = std::max<int32_t>(1, lens[r]);
-    ret_keys += L.n_ret * n;
-    str_keys += L.n_str * std::min<int64_t>(n, c->W);
-  }
-  const int64_t slots = (int64_t)cfg.num_sms * (cfg.ctas_per_sm > 0 ? cfg.ctas_per_sm : 1);
-  int64_t ctas = slots * str_keys / std::max<int64_t>(1, ret_keys + str_keys);
-  ctas = std::max<int64_t>(1, std::min(ctas, items));
-  return (int)((items + ctas - 1) / ctas);
-}
-
 // Tensor-core decode: splits per retrieval head of each launch row.  The
-// SMs' CTA slots left after the streaming CTAs (str_ctas) are handed out one
-// split at a time to the row whose splits currently hold the most keys (every
-// row starts with one), which minimises the longest split; a row gets at most
-// one split per two CTA iterations of keys and at most DUO_MAX_SPLITS.  A
-// forced count applies to every row, capped by its length.
+// SMs' CTA slots left after the streaming heads are handed out one split at
+// a time to the row whose splits currently hold the most keys (every row
+// starts with one), which minimises the longest split; a row gets at most one
+// split per two CTA iterations of keys and at most DUO_MAX_SPLITS.  A forced
+// count applies to every row, capped by its length.
 void choose_row_splits(const duo_cache *c, int layer, const int32_t *lens, int nrows,
-                       int64_t str_ctas, const duo::DecodeConfig &cfg, int16_t *out) {
+                       const duo::DecodeConfig &cfg, int16_t *out) {
   const auto &L = c->layers[layer];
   std::vector<int64_t> cap(nrows);
   for (int r = 0; r < nrows; ++r) {
@@ -241,7 +219,7 @@ void choose_row_splits(const duo_cache *c, int layer, const int32_t *lens, int n
   }
   if (L.n_ret == 0 || c->forced_splits > 0) return;
   const int64_t slots = (int64_t)cfg.num_sms * (cfg.ctas_per_sm > 0 ? cfg.ctas_per_sm : 1);
-  const int64_t budget = (slots - str_ctas) / L.n_ret;  // splits over all rows
+  const int64_t budget = (slots - (int64_t)nrows * L.n_str) / L.n_ret;  // splits over all rows
   std::vector<std::pair<double, int>> heap;  // (keys per split, row), max-heap
   for (int r = 0; r < nrows; ++r)
     if (cap[r] > 1) heap.emplace_back((double)std::max<int32_t>(1, lens[r]), r);
@@ -514,7 +492,6 @@ void fill_decode_common(const duo_cache *c, int32_t layer, const void *q, void *
   p->scale_log2 = sc * 1.4426950408889634f;
   p->err = duo::device_error_word();
   p->pool = c->reproducible ? 0 : 1;
-  p->str_per_cta = 1;
   p->out_f32 = (d.kv_dtype != DUO_F32 && c->out_dtype == DUO_F32) ? 1 : 0;
   p->shard_lo = c->shard_lo;
   p->shard_hi = c->shard_hi;
@@ -638,9 +615,7 @@ duo_status decode_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &
       p.rows.len[r] = (int32_t)(len_of(c, layer, rows[g0 + r]) + (fused ? 1 : 0));
       rlen[r] = (int32_t)ret_len(c, p.rows.len[r]);
     }
-    p.str_per_cta = str_items_per_cta(c, layer, p.rows.len, nr, cfg);
-    const int64_t str_ctas = ((int64_t)nr * L.n_str + p.str_per_cta - 1) / p.str_per_cta;
-    choose_row_splits(c, layer, rlen, nr, str_ctas, cfg, p.nsplit_r);
+    choose_row_splits(c, layer, rlen, nr, cfg, p.nsplit_r);
     if (part) {
       p.part_o = part->o + (int64_t)g0 * d.n_q_heads * d.head_dim;
       p.part_lse = part->lse + (int64_t)g0 * d.n_q_heads;
@@ -1129,9 +1104,7 @@ duo_status duo_decode_splits(const duo_cache *c, int32_t layer, int32_t *splits)
   int32_t best = 1;
   for (int g0 = 0; g0 < c->desc.batch; g0 += duo::kMaxLaunchRows) {
     const int nr = std::min(duo::kMaxLaunchRows, c->desc.batch - g0);
-    const int spc = str_items_per_cta(c, layer, lens.data() + g0, nr, cfg);
-    const int64_t str_ctas = ((int64_t)nr * c->layers[layer].n_str + spc - 1) / spc;
-    choose_row_splits(c, layer, lens.data() + g0, nr, str_ctas, cfg, sp.data() + g0);
+    choose_row_splits(c, layer, lens.data() + g0, nr, cfg, sp.data() + g0);
     for (int r = 0; r < nr; ++r) best = std::max<int32_t>(best, sp[g0 + r]);
   }
   *splits = best;

@@ -127,7 +127,6 @@ struct DecodeParams {
   const void *knew, *vnew;
   int pdl;             // launched with programmatic dependent launch
   int out_f32;         // bf16 and 4-bit caches: out is float32 instead of bf16
-  int str_per_cta;     // tensor-core decode: (launch row, streaming head) items per streaming CTA
   int pool;            // tensor-core decode: the last eighth of a split head's
                        // tiles is claimed at run time (0: every split gets an
                        // even, fixed share)
