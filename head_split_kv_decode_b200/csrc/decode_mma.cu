@@ -301,10 +301,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // Nothing the previous kernel may have written is read before this.
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // Fused append: the token at position n-1 is not in the cache yet.  The
-  // warp whose tile holds its row writes it there, skips that row, and adds
-  // the key at the end from the inputs (bf16) or from its shared-memory copy
-  // (4-bit).
+  // Fused append: the token at position n-1 is not in the cache yet.  One
+  // warp (see owns_new) writes it there and adds the key at the end from the
+  // inputs (bf16) or from its shared-memory copy (4-bit); the tile walk skips
+  // that row.
   // In partial mode a rank that does not own the streaming heads leaves
   // their rows empty (another shard contributes them).
   if (P.part_o && !retrieval && !P.own_str) {
@@ -315,7 +315,12 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   }
   const bool fused = P.knew != nullptr && new_here_shard;
   const int newk = retrieval ? n - 1 - (int)P.shard_lo : (int)ring_slot(n - 1, P.S, P.R);  // its row
-  const bool owns_new = fused && !split_head && newk >= k0 && newk < k1;
+  // The new token is written and attended by warp 0 of the CTA that walks
+  // its row, or for a split head by warp 0 of split 0, at the start: the tile
+  // that holds the row comes last and is claimed from the pool, so doing the
+  // work (4-bit: quantisation) there would put it on the launch's critical
+  // path.  Whichever warp visits that tile skips the row.
+  const bool owns_new = fused && (split_head ? split == 0 : (newk >= k0 && newk < k1));
   // its K/V in the inputs (bf16); recomputed where used rather than held
   // through the main loop
   auto in_off = [&]() { return ((int64_t)r * P.Hkv + kvh) * (int64_t)(D * 2); };
@@ -443,6 +448,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   float m = -INFINITY, l = 0.f;
   float mq[2] = {-INFINITY, -INFINITY}, lq[2] = {0.f, 0.f}, zq[2] = {0.f, 0.f};
   int f = 20;
+  // 4-bit with at most 4 queries per KV head: the residual of p*sc rides in the
+  // idle query columns 4..7 of the V product (see q4_update)
+  constexpr bool kLoInN = Q4 && G <= 4;
 
   // bf16 cache, one warp: keys [kb0, kb0 + 16) below hi of the buffers Kx/Vx,
   // row index = key, except `skip_key`.  `full` (a compile-time flag)
@@ -605,33 +613,42 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     // The largest V scale of the tile bounds p*sc: with p < 2^(8+f) (the lazy
     // rescale below) and sc < 2^(E-14) for an fp16 exponent field E >= 1,
     // f = 21 - E keeps p*sc < 2^15.  Positive fp16 values order as integers.
+    // The warp-wide maximum is needed only when some lane's own scales ask
+    // for less headroom than f has (rare after the first tiles).
     uint32_t vm = 0;
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) vm = max(vm, max(vsz[kg][0] & 0xffffu, vsz[kg][1] & 0xffffu));
+    ftile = f;
+    if (__any_sync(0xffffffffu, 21 - max((int)(vm >> 10), 1) < f)) {
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, off));
-    ftile = 21 - max((int)(vm >> 10), 1);
+      for (int off = 4; off < 32; off <<= 1) vm = max(vm, __shfl_xor_sync(0xffffffffu, vm, off));
+      ftile = 21 - max((int)(vm >> 10), 1);
+    }
     // ------------------------------------------------------------ S^T = K Q^T
     // A rows g / g+8 are keys kb + g / kb + 8 + g; k-slots follow the channel
     // order of the query fragments (see the set-up)
+    // Per key group two accumulators (channels 32t..32t+15 and +16..+31)
+    // halve the chains of dependent products; each query fragment is loaded
+    // once for both groups.
+    float acc[KG][2][4];
+#pragma unroll
+    for (int kg = 0; kg < KG; ++kg)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[kg][0][i] = acc[kg][1][i] = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
+#pragma unroll
+      for (int kg = 0; kg < KG; ++kg) {
+        const uint32_t x0 = (&kr[kg][0].x)[w], x1 = (&kr[kg][1].x)[w], y0 = x0 >> 8, y1 = x1 >> 8;
+        float(&a)[4] = acc[kg][w >> 1];
+        mma16816_full_f16(a, x0 & kNib0, x1 & kNib0, x0 & kNib1, x1 & kNib1, qf.x, qf.y);
+        mma16816_full_f16(a, y0 & kNib0, y1 & kNib0, y0 & kNib1, y1 & kNib1, qf.z, qf.w);
+      }
+    }
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
       const int kb = kb0 + 16 * kg;
-      // two accumulators (channels 32t..32t+15 and +16..+31) halve the chain
-      // of dependent products
-      float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t w0[4] = {kr[kg][0].x, kr[kg][0].y, kr[kg][0].z, kr[kg][0].w};
-      const uint32_t w1[4] = {kr[kg][1].x, kr[kg][1].y, kr[kg][1].z, kr[kg][1].w};
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
-        const uint32_t x0 = w0[w], x1 = w1[w], y0 = x0 >> 8, y1 = x1 >> 8;
-        float(&acc)[4] = w < 2 ? s : s2;
-        mma16816_full_f16(acc, x0 & kNib0, x1 & kNib0, x0 & kNib1, x1 & kNib1, qf.x, qf.y);
-        mma16816_full_f16(acc, y0 & kNib0, y1 & kNib0, y0 & kNib1, y1 & kNib1, qf.z, qf.w);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) s[i] += s2[i];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float2 kp = half2_bits_to_f2(ksz[kg][h]);  // (scale, zero)
@@ -640,30 +657,35 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         const bool valid = FULL || (key < hi && key != skip_key);
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-          sc[kg][h][e] = valid ? fmaf(s[2 * h + e], a, kp.y * c2q[e]) : -INFINITY;
+          sc[kg][h][e] =
+              valid ? fmaf(acc[kg][0][2 * h + e] + acc[kg][1][2 * h + e], a, kp.y * c2q[e]) : -INFINITY;
       }
     }
   };
   // Online softmax of the scored tile, then O^T += V^T P^T.
   auto q4_update = [&](auto full) {
     constexpr bool FULL = decltype(full)::value;
+    // Rescale when a running max grows by more than 2^8 or the headroom must
+    // shrink (numerator and denominator scale together).  A column's maximum
+    // over its eight key rows is needed only if some lane's own maximum
+    // passes m + 8 (with m = -inf, any finite score does).
     float mx[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       float x = -INFINITY;
 #pragma unroll
       for (int kg = 0; kg < KG; ++kg) x = fmaxf(x, fmaxf(sc[kg][0][e], sc[kg][1][e]));
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
       mx[e] = x;
     }
-    // Rescale when a running max grows by more than 2^8 or the headroom must
-    // shrink (numerator and denominator scale together).
-    bool grow[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) grow[e] = mx[e] > mq[e] + 8.f || (mq[e] == -INFINITY && mx[e] > -INFINITY);
     const bool shrink = ftile < f;  // the same in every lane
-    if (__any_sync(0xffffffffu, grow[0] || grow[1]) || shrink) {
+    if (__any_sync(0xffffffffu, mx[0] > mq[0] + 8.f || mx[1] > mq[1] + 8.f) || shrink) {
+      bool grow[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], off));
+        grow[e] = mx[e] > mq[e] + 8.f;
+      }
       float alpha[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -675,6 +697,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         if (shrink) alpha[e] *= exp2i(ftile - f);
         lq[e] *= alpha[e];
         zq[e] *= alpha[e];
+        // the residual columns (lanes t >= 2) scale with their live columns
+        if (kLoInN) {
+          const float other = __shfl_xor_sync(0xffffffffu, alpha[e], 2);
+          if (t >= 2) alpha[e] = other;
+        }
       }
       if (shrink) f = ftile;
 #pragma unroll
@@ -689,8 +716,12 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
 #pragma unroll
     for (int kg = 0; kg < KG; ++kg) {
       // p*sc per (key, query) as an f16 high part and residual, packed per key
-      // row of P (queries 2t, 2t+1), then transposed to P^T fragments
-      uint32_t ph[2], pl[2];
+      // row of P (queries 2t, 2t+1), then transposed to P^T fragments.  With
+      // G <= 4 the query columns 4..7 are idle, so lanes t = 2, 3 take the
+      // live columns' p*sc from lanes t = 0, 1 and contribute the residuals
+      // there: one product gives the high sums in columns 0..3 and the
+      // residual sums in 4..7, added once at the end.
+      uint32_t ph[2], pl[2] = {0u, 0u};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float2 vp = half2_bits_to_f2(vsz[kg][h]);  // (scale, zero)
@@ -704,13 +735,30 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
           zq[e] = fmaf(p, vp.y, zq[e]);
           pv[e] = p * vp.x;
         }
-        ph[h] = pack_f16(pv[0], pv[1]);
-        const float2 hf = half2_bits_to_f2(ph[h]);
-        pl[h] = pack_f16(pv[0] - hf.x, pv[1] - hf.y);
+        if constexpr (kLoInN) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float other = __shfl_xor_sync(0xffffffffu, pv[e], 2);
+            if (t >= 2) pv[e] = other;
+          }
+          const uint32_t hi = pack_f16(pv[0], pv[1]);
+          const float2 hf = half2_bits_to_f2(hi);
+          const uint32_t lo = pack_f16(pv[0] - hf.x, pv[1] - hf.y);
+          ph[h] = t < 2 ? hi : lo;
+        } else {
+          ph[h] = pack_f16(pv[0], pv[1]);
+          const float2 hf = half2_bits_to_f2(ph[h]);
+          pl[h] = pack_f16(pv[0] - hf.x, pv[1] - hf.y);
+        }
       }
-      // P^T fragment: b0 = keys 2t, 2t+1, b1 = keys 8+2t, 9+2t, of query g
+      // P^T fragment: b0 = keys 2t, 2t+1, b1 = keys 8+2t, 9+2t, of column g
       const uint32_t pb0 = movm_trans(ph[0]), pb1 = movm_trans(ph[1]);
-      const uint32_t pl0 = movm_trans(pl[0]), pl1 = movm_trans(pl[1]);
+      uint32_t pl0 = 0u, pl1 = 0u;
+      (void)pl;
+      if constexpr (!kLoInN) {
+        pl0 = movm_trans(pl[0]);
+        pl1 = movm_trans(pl[1]);
+      }
       // ---------------------------------------------------------- O^T += V^T P^T
       // A rows g / g+8 are channels vchan(mt) / vchan(mt)+1; cols are keys
       // (2t, 2t+1) from ab and (8+2t, 9+2t) from cd, two bytes (4 channels)
@@ -727,10 +775,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
           const int mt = 4 * wi + 2 * hh;
           const uint32_t a0 = ab & kNib0, a1 = ab & kNib1, a2 = cd & kNib0, a3 = cd & kNib1;
           mma16816_full_f16(o[mt], a0, a1, a2, a3, pb0, pb1);
-          mma16816_full_f16(o[mt], a0, a1, a2, a3, pl0, pl1);
+          if (!kLoInN) mma16816_full_f16(o[mt], a0, a1, a2, a3, pl0, pl1);
           const uint32_t b0 = ab8 & kNib0, b1 = ab8 & kNib1, b2 = cd8 & kNib0, b3 = cd8 & kNib1;
           mma16816_full_f16(o[mt + 1], b0, b1, b2, b3, pb0, pb1);
-          mma16816_full_f16(o[mt + 1], b0, b1, b2, b3, pl0, pl1);
+          if (!kLoInN) mma16816_full_f16(o[mt + 1], b0, b1, b2, b3, pl0, pl1);
         }
       }
     }
@@ -786,10 +834,6 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     auto visit = [&](int tt) {
       const int kb0 = tt * T;
       const bool has_new = fused && newk >= kb0 && newk < kb0 + T;
-      if (has_new) {
-        write_new();
-        new_here = true;
-      }
       run_tile(kb0, keys, has_new ? newk : -1);
     };
     unsigned c = 0;
@@ -866,6 +910,13 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   float *red_o = red_l + NWARPS * G;
   // the zero-point sums of this thread's two O^T columns (queries 2t, 2t+1)
   float z0 = 0.f, z1 = 0.f;
+  if constexpr (kLoInN) {
+    // columns 4..7 (lanes t >= 2) hold the residual sums of columns 0..3
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[mt][i] += __shfl_xor_sync(0xffffffffu, o[mt][i], 2);
+  }
   if constexpr (Q4) {
     // sums over the eight key rows g of each query column
 #pragma unroll

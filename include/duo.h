@@ -236,10 +236,11 @@ duo_status duo_decode_attn_rows(duo_cache *cache, int32_t layer, const int32_t *
  * (hotpaper.ai) and of section "Technical principles of DuoAttention" of
  * "What is DuoAttention" (nav.superapi.store), in one pass): append each row's new token (k_new, v_new: [batch, n_kv_heads,
  * head_dim]) at position len and attend with q at that position, exactly as
- * duo_append_kv(.., 1, ..) followed by duo_decode_attn.  The warp whose key
- * tile holds the new token's row takes its K/V from the inputs and writes
- * them to the cache.  Configurations without a fused kernel (fp32 caches,
- * head_dim 64, 4-bit caches) run the two calls.  Advances each row's length
+ * duo_append_kv(.., 1, ..) followed by duo_decode_attn.  One warp of the
+ * launch takes the new token's K/V from the inputs (4-bit caches: quantises
+ * it with duo_append_kv's encoder) and writes it to the cache; the attention
+ * adds that key from the inputs.  Configurations without a fused kernel (fp32
+ * caches, head_dim 64) run the two calls.  Advances each row's length
  * by one.  The launch uses programmatic dependent launch, so its set-up
  * overlaps the previous kernel in the stream.  Errors as for the two calls. */
 duo_status duo_decode_step(duo_cache *cache, int32_t layer, const void *q,
