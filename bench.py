@@ -160,8 +160,12 @@ class ClockSampler:
 DECODE_TRAFFIC_SOURCES = ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "kernels.h",
                           "quant_int4.cuh")
 DECODE_TRAFFIC = {
-    "bf16": {"sha256": None, "dram_bytes": None, "algorithmic_bytes": None},
-    "int4": {"sha256": None, "dram_bytes": None, "algorithmic_bytes": None},
+    # fused step, Llama-3-8B-shaped GQA, 128K, batch 1, one layer
+    "bf16": {"sha256": "4d34133103a7e1ea157446aa22b12fad6d8acdb4ecc73df7b41a784d334f4eba",
+             "dram_bytes": 269800704 + 4463872, "algorithmic_bytes": 269120512},
+    # 4-bit decode, Llama-3-8B-shaped GQA, 1M, batch 1, one layer
+    "int4": {"sha256": "4d34133103a7e1ea157446aa22b12fad6d8acdb4ecc73df7b41a784d334f4eba",
+             "dram_bytes": 285903872 + 5694208, "algorithmic_bytes": 285495496},
 }
 
 
