@@ -103,6 +103,7 @@ SIGNATURES = {
     "duo_set_decode_output": (_I32, [_P, _I32]),
     "duo_test_stall_next_prefill": (_I32, [_P, _I64]),
     "duo_decode_splits": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
+    "duo_decode_streaming_pack": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "duo_poll_device_error": (_I32, [ctypes.POINTER(_I32)]),
     "duo_status_string": (ctypes.c_char_p, [_I32]),
 }
@@ -322,6 +323,12 @@ def duo_set_decode_reproducible(handle, on):
 def duo_decode_splits(handle, layer):
     s = _I32()
     _check(lib().duo_decode_splits(handle, layer, ctypes.byref(s)), "duo_decode_splits")
+    return s.value
+
+
+def duo_decode_streaming_pack(handle, layer):
+    s = _I32()
+    _check(lib().duo_decode_streaming_pack(handle, layer, ctypes.byref(s)), "duo_decode_streaming_pack")
     return s.value
 
 

@@ -261,6 +261,10 @@ class DuoCache:
     def decode_splits(self, layer):
         return B.duo_decode_splits(self.handle, layer)
 
+    def decode_streaming_pack(self, layer):
+        """Streaming heads per streaming CTA of the next decode of `layer`."""
+        return B.duo_decode_streaming_pack(self.handle, layer)
+
     def reset(self):
         B.duo_cache_reset(self.handle)
 

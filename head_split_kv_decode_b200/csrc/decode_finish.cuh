@@ -181,6 +181,53 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   }
 }
 
+// Epilogue of a streaming CTA that holds several streaming heads of launch
+// row r (heads pidx0, pidx0 + 1, ... of the row), each on a group of wph
+// consecutive warps.  The per-warp states are staged as for
+// decode_reduce_store; group h combines warps h*wph .. h*wph + wph - 1 and
+// writes its G query heads directly (or, in partial mode, their normalised
+// rows and log-sum-exps).  Groups past the row's last streaming head write
+// nothing.
+template <typename T, int D, int G, int NWARPS>
+__device__ __forceinline__ void decode_store_groups(const DecodeParams &P, uint8_t *smem, int wph,
+                                                    int r, int pidx0) {
+  constexpr float kLn2 = 0.6931471805599453f;
+  constexpr int NT = NWARPS * 32;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const float *red_m = reinterpret_cast<const float *>(smem);
+  const float *red_l = red_m + NWARPS * G;
+  const float *red_o = red_l + NWARPS * G;
+  const int groups = min(NWARPS / wph, P.n_str - pidx0);
+  // one output element per thread and step; D is a multiple of 32, so the
+  // group and query head are the same across a warp, and lane w < wph holds
+  // the weight of the group's warp w
+  static_assert(D % 32 == 0, "warp-uniform query head");
+  for (int idx = tid; idx < groups * G * D; idx += NT) {
+    const int h = idx / (G * D), g = (idx / D) % G, c = idx % D;
+    const int w0 = h * wph;
+    const float mw = lane < wph ? red_m[(w0 + lane) * G + g] : -INFINITY;
+    float M = mw;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float sw = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+    float L = lane < wph ? red_l[(w0 + lane) * G + g] * sw : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    float O = 0.f;
+    for (int w = 0; w < wph; ++w) O += red_o[((w0 + w) * G + g) * D + c] * __shfl_sync(0xffffffffu, sw, w);
+    const int64_t row = (int64_t)r * P.Hq + (int64_t)P.h.str_heads[pidx0 + h] * G + g;
+    if (P.part_o) {
+      const bool empty = L == 0.f;
+      P.part_o[row * D + c] = empty ? 0.f : O / L;
+      if (c == 0) P.part_lse[row] = empty ? -INFINITY : (M + fast_log2(L)) * kLn2;
+    } else if (P.out_f32) {
+      reinterpret_cast<float *>(P.out)[row * D + c] = O / L;
+    } else {
+      store_out(reinterpret_cast<T *>(P.out) + row * D + c, O / L);
+    }
+  }
+}
+
 // State layout expected: each 8-lane group of a warp holds m[g], l[g] and NP
 // fp32 pairs of the output row of query head g; chan(li, j) gives the channel
 // of pair j's first element for lane li of the group.

@@ -196,10 +196,23 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
   // ---- work item: retrieval CTAs first (launch row r, head, split), then
-  // one CTA per (launch row, streaming head)
+  // per launch row the streaming CTAs, each holding str_pack streaming heads
+  // (heads i*str_pack .. i*str_pack + str_pack - 1 of the row), one per group
+  // of wph = NWARPS/str_pack warps.  A warp's head (pidx, kvh) is the same
+  // across its group; wsub is the warp's rank in the group.
   const int n_ret_ctas = P.cta0[P.rows.n];
+  // (recomputed in the epilogue rather than held through the main loop)
+  auto str_group = [&](int &r_, int &pidx0_, int &wph_) {
+    const int x = (int)blockIdx.x - n_ret_ctas;
+    const int hp = Q4 ? 1 : max(P.str_pack, 1);  // the 4-bit path shares its queries CTA-wide
+    const int per_row = (P.n_str + hp - 1) / hp;
+    r_ = x / per_row;
+    pidx0_ = (x % per_row) * hp;
+    wph_ = NWARPS / hp;
+  };
   int r, kvh, pidx, split, nsplit;
-  bool retrieval;
+  int wph = NWARPS, wsub = warp;
+  bool retrieval, idle = false;
   if ((int)blockIdx.x < n_ret_ctas) {
     int lo = 0, hi = P.rows.n;  // the last r with cta0[r] <= blockIdx.x
     while (hi - lo > 1) {
@@ -214,9 +227,12 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     kvh = P.h.ret_heads[pidx];
     retrieval = true;
   } else {
-    const int x = (int)blockIdx.x - n_ret_ctas;
-    r = x / P.n_str;
-    pidx = x % P.n_str;
+    int pidx0;
+    str_group(r, pidx0, wph);
+    wsub = warp % wph;
+    pidx = pidx0 + warp / wph;
+    idle = pidx >= P.n_str;  // a group past the row's last head: no keys, no output
+    if (idle) pidx = P.n_str - 1;
     kvh = P.h.str_heads[pidx];
     retrieval = false;
     split = 0;
@@ -230,7 +246,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // at page rows from 0; `keys` of them are below n.  Streaming heads hold
   // the whole window.
   const int keys = retrieval ? (int)max((int64_t)0, min((int64_t)n, P.shard_hi) - P.shard_lo)
-                             : min(n, P.W);
+                             : (idle ? 0 : min(n, P.W));
   const bool new_here_shard = !retrieval || (n - 1 >= P.shard_lo && n - 1 < P.shard_hi);
   constexpr int RB = Q4 ? D / 2 : D * 2;  // bytes per key row
   // Streaming heads: one slot buffer, first storage row srow0.  Retrieval
@@ -254,8 +270,9 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
                  : pooled    ? (tiles - tiles / 8) / nsplit
                              : (tiles + nsplit - 1) / nsplit;  // tiles per split share
   const int t1 = min(tiles, (split + 1) * ts);                 // end of this split's share
-  // this warp's first two tiles, [first, first + T) and the one NWARPS tiles on
-  const int first = split_head ? (split * ts + warp) * T : k0 + warp * T;
+  // this warp's first two tiles, [first, first + T) and the one NWARPS (a
+  // streaming group: wph) tiles on
+  const int first = split_head ? (split * ts + warp) * T : k0 + wsub * T;
   const int last = split_head ? min(keys, t1 * T) : k1;
 
   // Bring rows [kb, min(kb + T, last)) of this head (one tile, inside one
@@ -294,7 +311,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   if (lane == 0) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int kb = first + i * NWARPS * T;
+      const int kb = first + i * wph * T;
       if (kb < last) prefetch_tile(kb);
     }
   }
@@ -308,15 +325,20 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // In partial mode a rank that does not own the streaming heads leaves
   // their rows empty (another shard contributes them).
   if (P.part_o && !retrieval && !P.own_str) {
-    const int64_t row0 = (int64_t)r * P.Hq + (int64_t)kvh * G;
-    for (int i = tid; i < G * D; i += NWARPS * 32) P.part_o[row0 * D + i] = 0.f;
-    if (tid < G) P.part_lse[row0 + tid] = -INFINITY;
+    int r_, pidx0, wph_;
+    str_group(r_, pidx0, wph_);
+    for (int hs = 0; hs < NWARPS / wph_ && pidx0 + hs < P.n_str; ++hs) {
+      const int64_t row0 = (int64_t)r * P.Hq + (int64_t)P.h.str_heads[pidx0 + hs] * G;
+      for (int i = tid; i < G * D; i += NWARPS * 32) P.part_o[row0 * D + i] = 0.f;
+      if (tid < G) P.part_lse[row0 + tid] = -INFINITY;
+    }
     return;
   }
   const bool fused = P.knew != nullptr && new_here_shard;
   const int newk = retrieval ? n - 1 - (int)P.shard_lo : (int)ring_slot(n - 1, P.S, P.R);  // its row
-  // The new token is written and attended by warp 0 of the CTA that walks
-  // its row, or for a split head by warp 0 of split 0, at the start: the tile
+  // The new token is written and attended by warp 0 of the CTA (of the
+  // head's group) that walks its row, or for a split head by warp 0 of split
+  // 0, at the start: the tile
   // that holds the row comes last and is claimed from the pool, so doing the
   // work (4-bit: quantisation) there would put it on the launch's critical
   // path.  Whichever warp visits that tile skips the row.
@@ -358,7 +380,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       reinterpret_cast<uint4 *>(dst)[c] = ldg128(src + 16 * c);
     }
   };
-  if (owns_new && warp == 0) write_new();
+  if (owns_new && wsub == 0) write_new();
 
   // ---- query fragments (rows g < G), k-step order matching the K loads
   uint32_t qa[8][2];
@@ -825,7 +847,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       tile(BoolC<false>{}, pk + row * RB, pv + row * RB, lo_k, hi_k, sk);
     }
   };
-  bool new_here = owns_new && warp == 0;  // this warp adds the new token at the end
+  bool new_here = owns_new && wsub == 0;  // this warp adds the new token at the end
   if (split_head) {
     // The first pool claim is issued during the warp's last tile of its
     // share, so that its latency overlaps that tile.
@@ -887,7 +909,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       c = __shfl_sync(0xffffffffu, nx, 0);
     }
   } else {
-    for (int kb0 = k0 + warp * T; kb0 < k1; kb0 += Keys<Q4>::STEP)
+    for (int kb0 = k0 + wsub * T; kb0 < k1; kb0 += wph * T)
       run_tile(kb0, k1, owns_new ? newk : -1);
   }
   if (new_here) {
@@ -961,6 +983,14 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     }
   }
   __syncthreads();
+  if constexpr (!Q4) {
+    if ((int)blockIdx.x >= n_ret_ctas && P.str_pack > 1) {  // several streaming heads, one per warp group
+      int r_, pidx0, wph_;
+      str_group(r_, pidx0, wph_);
+      decode_store_groups<__nv_bfloat16, D, G, NWARPS>(P, smem, wph_, r_, pidx0);
+      return;
+    }
+  }
   decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(
       P, smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
       (int64_t)r * P.n_ret + pidx, (int64_t)(retrieval ? P.cta0[r] : 0) + (int64_t)pidx * nsplit,
@@ -989,7 +1019,8 @@ cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
     cfg->num_sms = sms;
     return cudaSuccess;
   }
-  const int grid = d.cta0[d.rows.n] + d.rows.n * d.n_str;
+  const int hp = Q4 ? 1 : (d.str_pack > 1 ? d.str_pack : 1);
+  const int grid = d.cta0[d.rows.n] + d.rows.n * ((d.n_str + hp - 1) / hp);
   if (grid == 0) return cudaSuccess;
   if (!d.pdl) {
     kern<<<grid, NWARPS * 32, smem, s>>>(d);

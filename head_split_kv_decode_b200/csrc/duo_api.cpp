@@ -200,13 +200,13 @@ int choose_splits(const duo_cache *c, int layer, int64_t n, const duo::DecodeCon
 }
 
 // Tensor-core decode: splits per retrieval head of each launch row.  The
-// SMs' CTA slots left after the streaming heads are handed out one split at
-// a time to the row whose splits currently hold the most keys (every row
-// starts with one), which minimises the longest split; a row gets at most one
-// split per two CTA iterations of keys and at most DUO_MAX_SPLITS.  A forced
-// count applies to every row, capped by its length.
+// SMs' CTA slots left after the str_ctas streaming CTAs are handed out one
+// split at a time to the row whose splits currently hold the most keys (every
+// row starts with one), which minimises the longest split; a row gets at most
+// one split per two CTA iterations of keys and at most DUO_MAX_SPLITS.  A
+// forced count applies to every row, capped by its length.
 void choose_row_splits(const duo_cache *c, int layer, const int32_t *lens, int nrows,
-                       const duo::DecodeConfig &cfg, int16_t *out) {
+                       const duo::DecodeConfig &cfg, int64_t str_ctas, int16_t *out) {
   const auto &L = c->layers[layer];
   std::vector<int64_t> cap(nrows);
   for (int r = 0; r < nrows; ++r) {
@@ -219,7 +219,7 @@ void choose_row_splits(const duo_cache *c, int layer, const int32_t *lens, int n
   }
   if (L.n_ret == 0 || c->forced_splits > 0) return;
   const int64_t slots = (int64_t)cfg.num_sms * (cfg.ctas_per_sm > 0 ? cfg.ctas_per_sm : 1);
-  const int64_t budget = (slots - (int64_t)nrows * L.n_str) / L.n_ret;  // splits over all rows
+  const int64_t budget = (slots - str_ctas) / L.n_ret;  // splits over all rows
   std::vector<std::pair<double, int>> heap;  // (keys per split, row), max-heap
   for (int r = 0; r < nrows; ++r)
     if (cap[r] > 1) heap.emplace_back((double)std::max<int32_t>(1, lens[r]), r);
@@ -234,6 +234,54 @@ void choose_row_splits(const duo_cache *c, int layer, const int32_t *lens, int n
       std::push_heap(heap.begin(), heap.end());
     }
   }
+}
+
+// Tensor-core decode on a bf16 cache: streaming heads per streaming CTA.
+// A streaming head is a window of at most S + R keys, so its CTA is short
+// next to a retrieval split of a long row; packing hp heads into one CTA (one
+// group of 16/hp warps each) frees SM slots for retrieval splits.  Taken:
+// the hp in {1, 2, 4, 8}, at most the row's streaming heads, that gives the
+// most retrieval CTAs while a streaming warp's keys (its head's window over
+// its group) stay within 3/4 of a retrieval warp's in the longest split; the
+// smallest such hp on a tie.  Lengths are the rows' retrieval keys (lens)
+// and the longest streaming window (win).
+int choose_str_pack(const duo_cache *c, int layer, const int32_t *lens, int nrows, int64_t win,
+                    const duo::DecodeConfig &cfg) {
+  const auto &L = c->layers[layer];
+  if (L.n_ret == 0 || L.n_str <= 1 || c->forced_splits > 0) return 1;
+  const int64_t win_t = (win + 15) / 16 * 16;  // rows of the window's tiles of 16 keys
+  int best = 1;
+  int64_t best_ctas = -1;
+  int16_t ns[duo::kMaxLaunchRows];
+  for (int hp = 1; hp <= 8 && hp <= 2 * L.n_str - 1; hp *= 2) {
+    const int64_t str_ctas = (int64_t)nrows * ((L.n_str + hp - 1) / hp);
+    choose_row_splits(c, layer, lens, nrows, cfg, str_ctas, ns);
+    int64_t ret_ctas = 0;
+    double longest = 0.0;  // keys of the longest split
+    for (int r = 0; r < nrows; ++r) {
+      ret_ctas += (int64_t)L.n_ret * ns[r];
+      longest = std::max(longest, (double)std::max<int32_t>(1, lens[r]) / ns[r]);
+    }
+    if (hp > 1 && (double)(hp * win_t) > 0.75 * longest) break;
+    if (ret_ctas > best_ctas) {
+      best = hp;
+      best_ctas = ret_ctas;
+    }
+  }
+  return best;
+}
+
+// One tensor-core decode launch of nr rows, with retrieval keys rlen and
+// lengths len (the query included): split counts into ns; returns the
+// streaming heads per streaming CTA.
+int plan_launch(const duo_cache *c, int layer, const int32_t *rlen, const int32_t *len, int nr,
+                const duo::DecodeConfig &cfg, int16_t *ns) {
+  const auto &L = c->layers[layer];
+  int64_t win = 0;  // the longest streaming window of the launch
+  for (int r = 0; r < nr; ++r) win = std::max<int64_t>(win, std::min<int64_t>(len[r], c->W));
+  const int hp = c->desc.kv_dtype == DUO_BF16 ? choose_str_pack(c, layer, rlen, nr, win, cfg) : 1;
+  choose_row_splits(c, layer, rlen, nr, cfg, (int64_t)nr * ((L.n_str + hp - 1) / hp), ns);
+  return hp;
 }
 
 // Rows of one call: every batch row in order (rows == NULL), or a list of
@@ -492,6 +540,7 @@ void fill_decode_common(const duo_cache *c, int32_t layer, const void *q, void *
   p->scale_log2 = sc * 1.4426950408889634f;
   p->err = duo::device_error_word();
   p->pool = c->reproducible ? 0 : 1;
+  p->str_pack = 1;
   p->out_f32 = (d.kv_dtype != DUO_F32 && c->out_dtype == DUO_F32) ? 1 : 0;
   p->shard_lo = c->shard_lo;
   p->shard_hi = c->shard_hi;
@@ -615,7 +664,7 @@ duo_status decode_rows(duo_cache *c, int32_t layer, const std::vector<int32_t> &
       p.rows.len[r] = (int32_t)(len_of(c, layer, rows[g0 + r]) + (fused ? 1 : 0));
       rlen[r] = (int32_t)ret_len(c, p.rows.len[r]);
     }
-    choose_row_splits(c, layer, rlen, nr, cfg, p.nsplit_r);
+    p.str_pack = plan_launch(c, layer, rlen, p.rows.len, nr, cfg, p.nsplit_r);
     if (part) {
       p.part_o = part->o + (int64_t)g0 * d.n_q_heads * d.head_dim;
       p.part_lse = part->lse + (int64_t)g0 * d.n_q_heads;
@@ -1083,6 +1132,26 @@ duo_status duo_set_decode_reproducible(duo_cache *c, int32_t on) {
   return DUO_OK;
 }
 
+// The plan of a tensor-core decode of every row at the current lengths: the
+// largest split count a row gets and the largest streaming pack of a launch.
+void decode_plan_all_rows(const duo_cache *c, int32_t layer, const duo::DecodeConfig &cfg,
+                          int32_t *splits, int32_t *pack) {
+  std::vector<int32_t> lens(c->desc.batch), rlen(c->desc.batch);
+  std::vector<int16_t> sp(c->desc.batch);
+  for (int b = 0; b < c->desc.batch; ++b) {
+    lens[b] = (int32_t)std::max<int64_t>(1, len_of(c, layer, b));
+    rlen[b] = (int32_t)ret_len(c, lens[b]);
+  }
+  *splits = 1;
+  *pack = 1;
+  for (int g0 = 0; g0 < c->desc.batch; g0 += duo::kMaxLaunchRows) {
+    const int nr = std::min(duo::kMaxLaunchRows, c->desc.batch - g0);
+    *pack = std::max<int32_t>(*pack, plan_launch(c, layer, rlen.data() + g0, lens.data() + g0, nr,
+                                                 cfg, sp.data() + g0));
+    for (int r = 0; r < nr; ++r) *splits = std::max<int32_t>(*splits, sp[g0 + r]);
+  }
+}
+
 duo_status duo_decode_splits(const duo_cache *c, int32_t layer, int32_t *splits) {
   if (!c || !splits || layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
   duo::DecodeConfig cfg{};
@@ -1097,17 +1166,24 @@ duo_status duo_decode_splits(const duo_cache *c, int32_t layer, int32_t *splits)
     return DUO_OK;
   }
   // the largest count an all-rows decode of the current lengths gives a row
-  std::vector<int32_t> lens(c->desc.batch);
-  std::vector<int16_t> sp(c->desc.batch);
-  for (int b = 0; b < c->desc.batch; ++b)
-    lens[b] = (int32_t)std::max<int64_t>(1, len_of(c, layer, b));
-  int32_t best = 1;
-  for (int g0 = 0; g0 < c->desc.batch; g0 += duo::kMaxLaunchRows) {
-    const int nr = std::min(duo::kMaxLaunchRows, c->desc.batch - g0);
-    choose_row_splits(c, layer, lens.data() + g0, nr, cfg, sp.data() + g0);
-    for (int r = 0; r < nr; ++r) best = std::max<int32_t>(best, sp[g0 + r]);
-  }
+  int32_t best = 1, pack = 1;
+  decode_plan_all_rows(c, layer, cfg, &best, &pack);
   *splits = best;
+  return DUO_OK;
+}
+
+duo_status duo_decode_streaming_pack(const duo_cache *c, int32_t layer, int32_t *heads_per_cta) {
+  if (!c || !heads_per_cta || layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
+  if (!mma_path(c)) {
+    *heads_per_cta = 1;
+    return DUO_OK;
+  }
+  duo::DecodeConfig cfg{};
+  cudaError_t e = cached_decode_config(const_cast<duo_cache *>(c), &cfg);
+  if (e != cudaSuccess) return launch_status(e);
+  int32_t best = 1, pack = 1;
+  decode_plan_all_rows(c, layer, cfg, &best, &pack);
+  *heads_per_cta = pack;
   return DUO_OK;
 }
 

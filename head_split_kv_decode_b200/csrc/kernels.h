@@ -130,6 +130,10 @@ struct DecodeParams {
   int pool;            // tensor-core decode: the last eighth of a split head's
                        // tiles is claimed at run time (0: every split gets an
                        // even, fixed share)
+  int str_pack;        // tensor-core decode, bf16 cache: streaming heads per
+                       // streaming CTA (1, 2, 4 or 8), each on NWARPS/str_pack
+                       // warps; the CTAs of launch row r are
+                       // cta0[rows.n] + r*ceil(n_str/str_pack) + i
 };
 
 struct PrefillParams {

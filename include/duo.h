@@ -421,6 +421,16 @@ duo_status duo_set_decode_output(duo_cache *cache, int32_t dtype);
 duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
                              int32_t *splits);
 
+/* Streaming heads per streaming CTA that the next decode of this layer will
+ * use (a scheduling choice; the pages have no counterpart).  The tensor-core
+ * decode on a bf16 cache may run 2, 4 or 8 of a row's streaming heads in one
+ * CTA, one group of warps each, when their windows are short next to the
+ * retrieval splits: the SMs this frees take more retrieval splits.  1 for
+ * every other configuration.  Outputs do not depend on it beyond rounding.
+ * Errors: DUO_ERR_ARG (null cache or pointer, layer out of range). */
+duo_status duo_decode_streaming_pack(const duo_cache *cache, int32_t layer,
+                                     int32_t *heads_per_cta);
+
 /* Testing hook for the failure path of the bounded in-kernel waits (the
  * pages have no counterpart).  The next duo_prefill_attn or
  * duo_prefill_attn_rows on this cache issues none of its tile loads, and its
