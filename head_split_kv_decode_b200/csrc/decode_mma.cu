@@ -899,6 +899,12 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     }
     for (; tt < t1; tt += NWARPS) {
       if (pooled && tt + NWARPS >= t1 && lane == 0) c = atomicAdd(next, 1u);
+      // bf16, packed layout: the warp's next tile goes to L2 while this one
+      // is loaded and multiplied (one bulk prefetch; no registers held), so
+      // each warp keeps two tiles in flight.  With a block table the
+      // prefetch would wait on a table load, and the 4-bit path keeps its
+      // next tile in registers instead.
+      if (!Q4 && !P.ret.table && lane == 0 && tt + NWARPS < t1) prefetch_tile((tt + NWARPS) * T);
       visit(tt);
     }
     c = __shfl_sync(0xffffffffu, c, 0);
