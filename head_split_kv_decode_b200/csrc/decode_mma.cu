@@ -929,6 +929,19 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
            reinterpret_cast<const uint8_t *>(P.vnew) + in_off(), 0, 1, -1);
   }
 
+  // The epilogue's parameter fields (output and workspace pointers), read
+  // once after a loop of tens of microseconds and by then out of the uniform
+  // cache, are fetched back into it by one thread while the warps stage their
+  // states; reading them cold delayed the partial store by up to 3 us.
+  if (tid == 0) {
+    const char *pp = reinterpret_cast<const char *>(&P);
+    asm volatile("prefetchu.L1 [%0];" ::"l"(pp + offsetof(DecodeParams, out)));
+    asm volatile("prefetchu.L1 [%0];" ::"l"(pp + offsetof(DecodeParams, Hq)));
+    asm volatile("prefetchu.L1 [%0];" ::"l"(pp + offsetof(DecodeParams, part_o)));
+    asm volatile("prefetchu.L1 [%0];" ::"l"(pp + offsetof(DecodeParams, ws_o)));
+    asm volatile("prefetchu.L1 [%0];" ::"l"(pp + offsetof(DecodeParams, ws_next)));
+    asm volatile("prefetchu.L1 [%0];" ::"l"(pp + offsetof(DecodeParams, out_f32)));
+  }
   // the next kernel in the stream may start its set-up now
   asm volatile("griddepcontrol.launch_dependents;");
 
