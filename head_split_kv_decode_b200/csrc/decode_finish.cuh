@@ -81,98 +81,56 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   }
   __syncthreads();
   if (!s_last) return;
-  // weights w_s = 2^(lse_s - max) per (split, query head), then the weighted
-  // sum of the partials.  Warp w sums splits w, w+NWARPS, ... (U at a time,
-  // their loads in flight together); lane l owns channels [4l, 4l+4) of every
-  // query head (D/4 float4 per head row; for D = 64 the upper lanes idle).
-  // The first batch of partials is loaded before the weights are reduced, so
-  // that its latency overlaps that reduction.
-  float *s_w = reinterpret_cast<float *>(smem);          // [nsplit][G]
-  float *s_den = s_w + nsplit * G;                       // [G]
-  float *s_mx = s_den + G;                               // [G]
-  float *s_acc = s_w + ((nsplit * G + 2 * G + 3) & ~3);  // [NWARPS][G][D], 16-byte aligned
-  constexpr int L4 = D / 4;
-  constexpr int U = G >= 8 ? 2 : 4;
-  const bool owns = lane < L4;
-  const float4 *src = reinterpret_cast<const float4 *>(P.ws_o + part0 * G * D) + (owns ? lane : 0);
-  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 v[U][G];
+  // Each warp produces 32 output channels of one query head (one per lane)
+  // from all splits: the lanes load every split's partial at their channel
+  // and the splits' log-sum-exps in one burst, so the merge costs one round
+  // trip to L2, with the weights 2^(lse_s - max) formed by shuffles (no
+  // shared memory, no barrier).  Splits are taken kHeld at a time, the
+  // running sum rescaled to each chunk's maximum (one chunk up to kHeld).
+  constexpr int SL = D / 32;     // 32-channel slices of a query head
+  constexpr int kHeld = 64;      // partials a lane holds at once
+  for (int sl = warp; sl < G * SL; sl += NWARPS) {
+    const int g = sl / SL, c = (sl % SL) * 32 + lane;
+    const float *po = P.ws_o + (part0 * G + g) * D + c;  // split s at po[s * G * D]
+    const float *pl = P.ws_lse + part0 * G + g;          // split s at pl[s * G]
+    float M = -INFINITY, den = 0.f, acc = 0.f;
+    for (int s0 = 0; s0 < nsplit; s0 += kHeld) {
+      const int ns = min(nsplit - s0, kHeld);
+      float x[kHeld / 32], v[kHeld];
 #pragma unroll
-  for (int u = 0; u < U; ++u)
+      for (int i = 0; i < kHeld / 32; ++i)
+        x[i] = 32 * i + lane < ns ? __ldcg(pl + (int64_t)(s0 + 32 * i + lane) * G) : -INFINITY;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int sp = warp + u * NWARPS;
-      v[u][g] = (owns && sp < nsplit) ? __ldcg(src + (sp * G + g) * L4) : zero4;
-    }
-  // warp g (and g + NWARPS, ...) reduces query head g over the splits, one
-  // split per lane at a time
-  for (int g = warp; g < G; g += NWARPS) {
-    float M = -INFINITY;
-    for (int sp = lane; sp < nsplit; sp += 32) {
-      const float x = __ldcg(P.ws_lse + (part0 + sp) * G + g);
-      s_w[sp * G + g] = x;
-      M = fmaxf(M, x);
-    }
+      for (int i = 0; i < kHeld; ++i) v[i] = i < ns ? __ldcg(po + (int64_t)(s0 + i) * G * D) : 0.f;
+      float m = x[0];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float den = 0.f;
-    for (int sp = lane; sp < nsplit; sp += 32) {
-      const float x = s_w[sp * G + g];
-      const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);  // a split that claimed no keys
-      s_w[sp * G + g] = w;
-      den += w;
-    }
+      for (int i = 1; i < kHeld / 32; ++i) m = fmaxf(m, x[i]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-    if (lane == 0) {
-      s_den[g] = den;
-      s_mx[g] = M;
-    }
-  }
-  __syncthreads();
-  float4 acc[G];
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float Mn = fmaxf(M, m);
+      if (Mn == -INFINITY) continue;  // no split of this chunk (or before) saw a key
+      const float a = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+      acc *= a;
+      den *= a;
+      M = Mn;
+      float w[kHeld / 32], d = 0.f;
 #pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = zero4;
-  auto fma4 = [&](float4 &a, float w, const float4 &x) {
-    a.x += w * x.x;
-    a.y += w * x.y;
-    a.z += w * x.z;
-    a.w += w * x.w;
-  };
-  int sp = warp;
-  while (true) {
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const int su = sp + u * NWARPS;
-        if (su < nsplit) fma4(acc[g], s_w[su * G + g], v[u][g]);
+      for (int i = 0; i < kHeld / 32; ++i) {
+        w[i] = x[i] == -INFINITY ? 0.f : fast_exp2(x[i] - M);  // a split that claimed no keys: 0
+        d += w[i];
       }
-    sp += U * NWARPS;
-    if (sp >= nsplit) break;
 #pragma unroll
-    for (int u = 0; u < U; ++u)
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      den += d;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const int su = sp + u * NWARPS;
-        v[u][g] = (owns && su < nsplit) ? __ldcg(src + (su * G + g) * L4) : zero4;
-      }
-  }
-  if (owns) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) reinterpret_cast<float4 *>(s_acc + (warp * G + g) * D)[lane] = acc[g];
-  }
-  __syncthreads();
-  for (int idx = tid; idx < G * D; idx += NT) {
-    const int g = idx / D, c = idx % D;
-    float num = 0.f;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) num += s_acc[(w * G + g) * D + c];
+      for (int i = 0; i < kHeld; ++i) acc += __shfl_sync(0xffffffffu, w[i / 32], i % 32) * v[i];
+    }
+    const bool empty = den == 0.f;
     if (P.part_o) {
-      P.part_o[(out_row + g) * D + c] = num / s_den[g];
-      if (c == 0) P.part_lse[out_row + g] = (s_mx[g] + fast_log2(s_den[g])) * kLn2;
+      P.part_o[(out_row + g) * D + c] = empty ? 0.f : acc / den;
+      if (c == 0) P.part_lse[out_row + g] = empty ? -INFINITY : (M + fast_log2(den)) * kLn2;
     } else {
-      put(g * D + c, num / s_den[g]);
+      put(g * D + c, acc / den);
     }
   }
   if (tid == 0) {  // leave the ticket (and chunk counter) ready for the next call
