@@ -68,16 +68,19 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
   if (direct) return;
 
   // ---- the last split of this head to finish merges all splits.  The
-  // barrier orders the CTA's partial stores before thread 0's fence, which
-  // (being cumulative) publishes them before the ticket; the CTA that draws
-  // the last ticket fences again before the barrier that lets its threads
-  // read the other splits' partials.
+  // barrier orders the CTA's partial stores before thread 0's ticket, an
+  // atomic with release and acquire semantics at GPU scope: the release
+  // (cumulative over what the barrier ordered before it) publishes the
+  // partials with the ticket, and the acquire by the CTA that draws the last
+  // ticket, followed by the barrier below, orders its threads' reads of the
+  // other splits' partials after their release.  (One atomic in place of a
+  // fence, the atomic and a second fence.)
   __syncthreads();
   unsigned *cnt = P.ws_cnt + unit;
   if (tid == 0) {
-    __threadfence();
-    s_last = (atomicAdd(cnt, 1u) == (unsigned)(nsplit - 1));
-    if (s_last) __threadfence();
+    unsigned prev;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(cnt) : "memory");
+    s_last = (prev == (unsigned)(nsplit - 1));
   }
   __syncthreads();
   if (!s_last) return;

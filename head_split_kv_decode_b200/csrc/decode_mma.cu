@@ -258,16 +258,18 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   constexpr int T = 16 * KG;  // keys per warp tile
   constexpr int kBlockMask = ~(kPageTokens - 1);
   // A retrieval head with several splits is cut into tiles of T keys.  Each
-  // split walks a fixed share of them; with P.pool the shares cover 7/8 of
-  // the tiles and the rest is claimed one tile at a time by warps that have
-  // finished (see below), so a CTA that gets less memory bandwidth takes
-  // fewer tiles and the splits finish together.  Each CTA leaves one
-  // partial.  Streaming heads and single-split heads walk [k0, k1).
+  // split walks a fixed share of them; with P.pool the shares cover 13/16 of
+  // the tiles (4-bit: 7/8) and the rest is claimed one tile at a time by
+  // warps that have finished (see below), so a CTA that gets less memory
+  // bandwidth takes fewer tiles and the splits finish together.  (The 4-bit
+  // path keeps the smaller pool: its pool tiles miss the register-pipelined
+  // walk of the fixed share.)  Each CTA leaves one partial.  Streaming heads
+  // and single-split heads walk [k0, k1).
   const bool split_head = retrieval && nsplit > 1;
   const bool pooled = split_head && P.pool;
   const int tiles = (keys + T - 1) / T;
   const int ts = !split_head ? 0
-                 : pooled    ? (tiles - tiles / 8) / nsplit
+                 : pooled    ? (tiles - (Q4 ? tiles / 8 : 3 * tiles / 16)) / nsplit
                              : (tiles + nsplit - 1) / nsplit;  // tiles per split share
   const int t1 = min(tiles, (split + 1) * ts);                 // end of this split's share
   // this warp's first two tiles, [first, first + T) and the one NWARPS (a

@@ -127,9 +127,9 @@ struct DecodeParams {
   const void *knew, *vnew;
   int pdl;             // launched with programmatic dependent launch
   int out_f32;         // bf16 and 4-bit caches: out is float32 instead of bf16
-  int pool;            // tensor-core decode: the last eighth of a split head's
-                       // tiles is claimed at run time (0: every split gets an
-                       // even, fixed share)
+  int pool;            // tensor-core decode: the last 3/16 (4-bit: 1/8) of a
+                       // split head's tiles is claimed at run time (0: every
+                       // split gets an even, fixed share)
   int str_pack;        // tensor-core decode, bf16 cache: streaming heads per
                        // streaming CTA (1, 2, 4 or 8), each on NWARPS/str_pack
                        // warps; the CTAs of launch row r are

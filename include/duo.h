@@ -395,8 +395,9 @@ duo_status duo_set_decode_splits(duo_cache *cache, int32_t splits);
 
 /* How the tensor-core decode (bf16 and 4-bit caches, head_dim 128) shares a
  * split retrieval head's keys among its splits.  By default (on = 0) each
- * split takes a fixed share of 7/8 of the key tiles and the last eighth goes,
- * one tile at a time, to whichever warps finish first, so that splits running
+ * split takes a fixed share of 13/16 of the key tiles (7/8 on a 4-bit cache)
+ * and the rest goes, one tile at a time, to whichever warps finish first, so
+ * that splits running
  * on SMs that get less memory bandwidth do less work and all finish together.
  * Which keys each split sums then varies between calls, and outputs can differ
  * in the last bits.  on = 1 gives every split an even fixed share instead:
