@@ -187,11 +187,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // 4-bit fused step: the new token of the head as quantised by its owning
   // warp: K codes [0, 64), V codes [64, 128), K (scale, zero) at 128 and V's
   // at 136, each padded to 8 bytes
-  __shared__ __align__(16) uint8_t s_new[Q4 ? 144 : 16];
-  // 4-bit: the query fragments, the same in every warp (they depend on the
-  // lane only), as [4][32 lanes][4 words]; the tile reloads them instead of
-  // holding 16 registers through it
-  __shared__ __align__(16) uint32_t s_q[Q4 ? 4 * 32 * 4 : 4];
+  __shared__ __align__(16) uint8_t s_new[Q4 ? kMaxStrPack * 144 : 16];  // one slot per warp group
+  // 4-bit: the query fragments of each group's head, the same in every warp
+  // of the group (they depend on the lane only), as [group][4][32 lanes][4
+  // words]; the tile reloads them instead of holding 16 registers through it
+  __shared__ __align__(16) uint32_t s_q[Q4 ? kMaxStrPack * 4 * 32 * 4 : 4];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // (recomputed in the epilogue rather than held through the main loop)
   auto str_group = [&](int &r_, int &pidx0_, int &wph_) {
     const int x = (int)blockIdx.x - n_ret_ctas;
-    const int hp = Q4 ? 1 : max(P.str_pack, 1);  // the 4-bit path shares its queries CTA-wide
+    const int hp = max(P.str_pack, 1);
     const int per_row = (P.n_str + hp - 1) / hp;
     r_ = x / per_row;
     pidx0_ = (x % per_row) * hp;
@@ -249,6 +249,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
                              : (idle ? 0 : min(n, P.W));
   const bool new_here_shard = !retrieval || (n - 1 >= P.shard_lo && n - 1 < P.shard_hi);
   constexpr int RB = Q4 ? D / 2 : D * 2;  // bytes per key row
+  // this lane's query fragments in s_q, and the offset of the new-token slot
+  // in s_new, of its group's head (4-bit)
+  const uint32_t sq = smem_u32(s_q) + (uint32_t)(((warp / wph) * 128 + lane) * 16);
+  const int snew = Q4 ? (warp / wph) * 144 : 0;
   // Streaming heads: one slot buffer, first storage row srow0.  Retrieval
   // heads: key tiles are addressed block by block (a tile never crosses a
   // block of the paged layout), with key indices local to the block.
@@ -363,13 +367,13 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         uint8_t *sz = which ? (retrieval ? P.p.ret_v_sz : P.p.str_v_sz)
                             : (retrieval ? P.p.ret_k_sz : P.p.str_k_sz);
         *reinterpret_cast<uint16_t *>(codes + row * RB + 2 * lane) = (uint16_t)packed;
-        *reinterpret_cast<uint16_t *>(s_new + 64 * which + 2 * lane) = (uint16_t)packed;
+        *reinterpret_cast<uint16_t *>(s_new + snew + 64 * which + 2 * lane) = (uint16_t)packed;
         if (lane == 0) {
           __half2 pair;
           pair.x = sch;
           pair.y = zph;
           reinterpret_cast<__half2 *>(sz)[row] = pair;
-          *reinterpret_cast<uint2 *>(s_new + 128 + 8 * which) =
+          *reinterpret_cast<uint2 *>(s_new + snew + 128 + 8 * which) =
               make_uint2(*reinterpret_cast<const uint32_t *>(&pair), 0u);
         }
       }
@@ -430,10 +434,10 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       // S^T: this thread scores queries 2t and 2t+1
       c2q[0] = __shfl_sync(0xffffffffu, c2, (2 * t) << 2);
       c2q[1] = __shfl_sync(0xffffffffu, c2, (2 * t + 1) << 2);
-      if (warp == 0) {
+      if (wsub == 0) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4 *>(&s_q[(j * 32 + lane) * 4]) =
+          *reinterpret_cast<uint4 *>(&s_q[((warp / wph) * 128 + j * 32 + lane) * 4]) =
               make_uint4(qa[2 * j][0], qa[2 * j][1], qa[2 * j + 1][0], qa[2 * j + 1][1]);
       }
       __syncthreads();
@@ -661,7 +665,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
       for (int i = 0; i < 4; ++i) acc[kg][0][i] = acc[kg][1][i] = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      const uint4 qf = lds128(smem_u32(&s_q[(w * 32 + lane) * 4]));  // k-steps 2w, 2w+1
+      const uint4 qf = lds128(sq + 512u * w);  // k-steps 2w, 2w+1
 #pragma unroll
       for (int kg = 0; kg < KG; ++kg) {
         const uint32_t x0 = (&kr[kg][0].x)[w], x1 = (&kr[kg][1].x)[w], y0 = x0 >> 8, y1 = x1 >> 8;
@@ -924,8 +928,8 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     // the new token: key 0 of a one-row buffer, the inputs (bf16) or the
     // warp's quantised copy in shared memory (4-bit)
     if constexpr (Q4)
-      tile_q4(BoolC<false>{}, IntC<1>{}, s_new + k_off, s_new + 64 + v_off, s_new + 128 + s_off,
-              s_new + 136 + s_off, 0, 1, -1);
+      tile_q4(BoolC<false>{}, IntC<1>{}, s_new + snew + k_off, s_new + snew + 64 + v_off,
+              s_new + snew + 128 + s_off, s_new + snew + 136 + s_off, 0, 1, -1);
     else
       tile(BoolC<false>{}, reinterpret_cast<const uint8_t *>(P.knew) + in_off(),
            reinterpret_cast<const uint8_t *>(P.vnew) + in_off(), 0, 1, -1);
@@ -1004,13 +1008,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
     }
   }
   __syncthreads();
-  if constexpr (!Q4) {
-    if ((int)blockIdx.x >= n_ret_ctas && P.str_pack > 1) {  // several streaming heads, one per warp group
-      int r_, pidx0, wph_;
-      str_group(r_, pidx0, wph_);
-      decode_store_groups<__nv_bfloat16, D, G, NWARPS>(P, smem, wph_, r_, pidx0);
-      return;
-    }
+  if ((int)blockIdx.x >= n_ret_ctas && P.str_pack > 1) {  // several streaming heads, one per warp group
+    int r_, pidx0, wph_;
+    str_group(r_, pidx0, wph_);
+    decode_store_groups<__nv_bfloat16, D, G, NWARPS>(P, smem, wph_, r_, pidx0);
+    return;
   }
   decode_reduce_store<__nv_bfloat16, D, G, NWARPS>(
       P, smem, &s_last, nsplit == 1, (int64_t)r * P.Hq + (int64_t)kvh * G,
@@ -1040,7 +1042,7 @@ cudaError_t run(const DecodeParams &d, cudaStream_t s, DecodeConfig *cfg) {
     cfg->num_sms = sms;
     return cudaSuccess;
   }
-  const int hp = Q4 ? 1 : (d.str_pack > 1 ? d.str_pack : 1);
+  const int hp = d.str_pack > 1 ? d.str_pack : 1;
   const int grid = d.cta0[d.rows.n] + d.rows.n * ((d.n_str + hp - 1) / hp);
   if (grid == 0) return cudaSuccess;
   if (!d.pdl) {

@@ -236,7 +236,7 @@ void choose_row_splits(const duo_cache *c, int layer, const int32_t *lens, int n
   }
 }
 
-// Tensor-core decode on a bf16 cache: streaming heads per streaming CTA.
+// Tensor-core decode: streaming heads per streaming CTA.
 // A streaming head is a window of at most S + R keys, so its CTA is short
 // next to a retrieval split of a long row; packing hp heads into one CTA (one
 // group of 16/hp warps each) frees SM slots for retrieval splits.  Taken:
@@ -253,7 +253,7 @@ int choose_str_pack(const duo_cache *c, int layer, const int32_t *lens, int nrow
   int best = 1;
   int64_t best_ctas = -1;
   int16_t ns[duo::kMaxLaunchRows];
-  for (int hp = 1; hp <= 8 && hp <= 2 * L.n_str - 1; hp *= 2) {
+  for (int hp = 1; hp <= duo::kMaxStrPack && hp <= 2 * L.n_str - 1; hp *= 2) {
     const int64_t str_ctas = (int64_t)nrows * ((L.n_str + hp - 1) / hp);
     choose_row_splits(c, layer, lens, nrows, cfg, str_ctas, ns);
     int64_t ret_ctas = 0;
@@ -279,7 +279,7 @@ int plan_launch(const duo_cache *c, int layer, const int32_t *rlen, const int32_
   const auto &L = c->layers[layer];
   int64_t win = 0;  // the longest streaming window of the launch
   for (int r = 0; r < nr; ++r) win = std::max<int64_t>(win, std::min<int64_t>(len[r], c->W));
-  const int hp = c->desc.kv_dtype == DUO_BF16 ? choose_str_pack(c, layer, rlen, nr, win, cfg) : 1;
+  const int hp = choose_str_pack(c, layer, rlen, nr, win, cfg);
   choose_row_splits(c, layer, rlen, nr, cfg, (int64_t)nr * ((L.n_str + hp - 1) / hp), ns);
   return hp;
 }

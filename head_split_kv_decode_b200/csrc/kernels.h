@@ -83,6 +83,9 @@ struct AppendParams {
   int64_t n_tok;
 };
 
+// Most streaming heads one tensor-core decode CTA takes (DecodeParams::str_pack).
+constexpr int kMaxStrPack = 8;
+
 struct DecodeParams {
   const void *q;   // [B][Hq][D] (tensor-core decode: [rows.n][Hq][D])
   void *out;       // same shape as q
@@ -130,8 +133,8 @@ struct DecodeParams {
   int pool;            // tensor-core decode: the last 3/16 (4-bit: 1/8) of a
                        // split head's tiles is claimed at run time (0: every
                        // split gets an even, fixed share)
-  int str_pack;        // tensor-core decode, bf16 cache: streaming heads per
-                       // streaming CTA (1, 2, 4 or 8), each on NWARPS/str_pack
+  int str_pack;        // tensor-core decode: streaming heads per streaming CTA
+                       // (1, 2, 4 or 8 = kMaxStrPack), each on NWARPS/str_pack
                        // warps; the CTAs of launch row r are
                        // cta0[rows.n] + r*ceil(n_str/str_pack) + i
 };

@@ -424,8 +424,8 @@ duo_status duo_decode_splits(const duo_cache *cache, int32_t layer,
 
 /* Streaming heads per streaming CTA that the next decode of this layer will
  * use (a scheduling choice; the pages have no counterpart).  The tensor-core
- * decode on a bf16 cache may run 2, 4 or 8 of a row's streaming heads in one
- * CTA, one group of warps each, when their windows are short next to the
+ * decode (bf16 and 4-bit caches) may run 2, 4 or 8 of a row's streaming heads
+ * in one CTA, one group of warps each, when their windows are short next to the
  * retrieval splits: the SMs this frees take more retrieval splits.  1 for
  * every other configuration.  Outputs do not depend on it beyond rounding.
  * Errors: DUO_ERR_ARG (null cache or pointer, layer out of range). */

@@ -135,3 +135,39 @@ def test_packed_sequence_shards():
     ref = OA.decode_reference(f64(q), f64(K), f64(V), mask.numpy(), S, R)
     assert_parity(out, ref, "bf16", "merged shards")
     assert duo_poll_device_error() == 0
+
+
+def test_packed_int4_decode_and_step():
+    """4-bit cache: three streaming heads packed into one CTA of four warp
+    groups (one group idle), each group with its own query fragments in
+    shared memory.  A decode and two fused steps against the oracle fed the
+    identically dequantised K/V (float32 outputs), then every code and
+    (scale, zero) pair in the cache, the new tokens' ring slots included."""
+    from test_int4_gpu import _check_cache_bytes as check_int4_bytes
+    from test_int4_gpu import _dequant_history, _inputs
+    B_, Hq, Hkv, S, R, n0, steps = 1, 24, 6, 4, 60, 52000, 2
+    n = n0 + steps
+    mask = _mask(Hkv, (0, 2, 4))
+    K, V, _ = _inputs(91, B_, n, Hq, Hkv, D)
+    Q = synth.kv_field(915, range(B_), range(n0 - 1, n), Hq, D, device="cuda").to(BF)
+    cache = DuoCache(1, B_, Hq, Hkv, D, "int4", n, mask[None], S, R)
+    cache.set_decode_output(torch.float32)
+    for p0 in range(0, n0, 8192):
+        p1 = min(n0, p0 + 8192)
+        cache.append(0, K[:, p0:p1].contiguous(), V[:, p0:p1].contiguous())
+    assert cache.decode_streaming_pack(0) > 1
+    Kh, Kc, Ks, Kz = _dequant_history(K)
+    Vh, Vc, Vs, Vz = _dequant_history(V)
+    out = cache.decode(0, Q[:, 0].contiguous())
+    torch.cuda.synchronize()
+    ref = OA.decode_reference(f64(Q[:, 0]), Kh[:, :n0], Vh[:, :n0], mask.numpy(), S, R)
+    assert_parity(out, ref, "int4", "packed 4-bit decode")
+    for i in range(steps):
+        t = n0 + i
+        q = Q[:, i + 1].contiguous()
+        out = cache.step(0, q, K[:, t].contiguous(), V[:, t].contiguous())
+        torch.cuda.synchronize()
+        ref = OA.decode_reference(f64(q), Kh[:, :t + 1], Vh[:, :t + 1], mask.numpy(), S, R)
+        assert_parity(out, ref, "int4", "packed 4-bit step at %d" % t)
+    check_int4_bytes(cache, Kc, Ks, Kz, Vc, Vs, Vz, mask, B_, n, Hkv, S, R)
+    assert duo_poll_device_error() == 0
