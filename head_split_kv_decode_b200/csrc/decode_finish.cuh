@@ -125,8 +125,16 @@ __device__ __forceinline__ void decode_reduce_store(const DecodeParams &P, uint8
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
       den += d;
+      // four independent chains, and nothing past the chunk's splits
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 0; i < kHeld; ++i) acc += __shfl_sync(0xffffffffu, w[i / 32], i % 32) * v[i];
+      for (int i = 0; i < kHeld; i += 4) {
+        if (i < ns) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) a4[k] += __shfl_sync(0xffffffffu, w[(i + k) / 32], (i + k) % 32) * v[i + k];
+        }
+      }
+      acc += (a4[0] + a4[1]) + (a4[2] + a4[3]);
     }
     const bool empty = den == 0.f;
     if (P.part_o) {
