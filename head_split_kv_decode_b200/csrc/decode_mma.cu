@@ -188,10 +188,11 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
   // warp: K codes [0, 64), V codes [64, 128), K (scale, zero) at 128 and V's
   // at 136, each padded to 8 bytes
   __shared__ __align__(16) uint8_t s_new[Q4 ? kMaxStrPack * 144 : 16];  // one slot per warp group
-  // 4-bit: the query fragments of each group's head, the same in every warp
-  // of the group (they depend on the lane only), as [group][4][32 lanes][4
-  // words]; the tile reloads them instead of holding 16 registers through it
-  __shared__ __align__(16) uint32_t s_q[Q4 ? kMaxStrPack * 4 * 32 * 4 : 4];
+  // The query fragments of each warp group's head, the same in every warp of
+  // the group (they depend on the lane only), as [group][4][32 lanes][4
+  // words]: the tile reloads them instead of holding 16 registers through it
+  // (on the bf16 path that removed every register spill of the kernel)
+  __shared__ __align__(16) uint32_t s_q[kMaxStrPack * 4 * 32 * 4];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;  // mma fragment coordinates
 
@@ -249,8 +250,8 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
                              : (idle ? 0 : min(n, P.W));
   const bool new_here_shard = !retrieval || (n - 1 >= P.shard_lo && n - 1 < P.shard_hi);
   constexpr int RB = Q4 ? D / 2 : D * 2;  // bytes per key row
-  // this lane's query fragments in s_q, and the offset of the new-token slot
-  // in s_new, of its group's head (4-bit)
+  // this lane's query fragments in s_q, and (4-bit) the offset of the
+  // new-token slot in s_new, of its group's head
   const uint32_t sq = smem_u32(s_q) + (uint32_t)(((warp / wph) * 128 + lane) * 16);
   const int snew = Q4 ? (warp / wph) * 144 : 0;
   // Streaming heads: one slot buffer, first storage row srow0.  Retrieval
@@ -454,6 +455,13 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         qa[k][0] = pack_bf16(q0, q1);  // exact: the inputs are bf16
         qa[k][1] = pack_bf16(q2, q3);
       }
+      if (wsub == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4 *>(&s_q[((warp / wph) * 128 + j * 32 + lane) * 4]) =
+              make_uint4(qa[2 * j][0], qa[2 * j][1], qa[2 * j + 1][0], qa[2 * j + 1][1]);
+      }
+      __syncthreads();
     }
   }
 
@@ -509,15 +517,22 @@ __global__ void __launch_bounds__(NWARPS * 32, 1) decode_mma_kernel(const __grid
         vr[i][h] = ok ? ldg128(Vx + key * RB + 16 * (8 * h + g)) : make_uint4(0, 0, 0, 0);
     }
     // ------------------------------------------------------------ S = Q K^T
+    // (query fragments from s_q, one 16-byte load per two k-steps for both
+    // halves of the tile)
     float sc[2][2];
+    float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int sp = 0; sp < 4; ++sp) {
+      const uint4 qf = lds128(sq + 512u * sp);  // k-steps 2sp, 2sp+1
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        mma16816(s2[nt], qf.x, qf.y, kr[nt][sp].x, kr[nt][sp].y);
+        mma16816(s2[nt], qf.z, qf.w, kr[nt][sp].z, kr[nt][sp].w);
+      }
+    }
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int sp = 0; sp < 4; ++sp) {
-        mma16816(s, qa[2 * sp][0], qa[2 * sp][1], kr[nt][sp].x, kr[nt][sp].y);
-        mma16816(s, qa[2 * sp + 1][0], qa[2 * sp + 1][1], kr[nt][sp].z, kr[nt][sp].w);
-      }
+      float(&s)[4] = s2[nt];
       // scores of query g at keys kb0 + 8*nt + 2t + e
       const int key = kb0 + 8 * nt + 2 * t;
 #pragma unroll
