@@ -161,11 +161,11 @@ DECODE_TRAFFIC_SOURCES = ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "k
                           "quant_int4.cuh")
 DECODE_TRAFFIC = {
     # fused step, Llama-3-8B-shaped GQA, 128K, batch 1, one layer
-    "bf16": {"sha256": "0a1b4808e9c1312f53606de14750731bb68785b58e957c2c86b12466640895a8",
-             "dram_bytes": 269502720 + 5117952, "algorithmic_bytes": 269120512},
+    "bf16": {"sha256": "7fada1562d235c33557bf34c111051c91582cf759e9f68473d1c05dac7ae3281",
+             "dram_bytes": 269190144 + 3686656, "algorithmic_bytes": 269120512},
     # 4-bit fused step, Llama-3-8B-shaped GQA, 1M, batch 1, one layer
-    "int4": {"sha256": "0a1b4808e9c1312f53606de14750731bb68785b58e957c2c86b12466640895a8",
-             "dram_bytes": 285977856 + 4743680, "algorithmic_bytes": 285495496},
+    "int4": {"sha256": "7fada1562d235c33557bf34c111051c91582cf759e9f68473d1c05dac7ae3281",
+             "dram_bytes": 285927680 + 3641088, "algorithmic_bytes": 285495496},
 }
 
 
