@@ -102,6 +102,8 @@ SIGNATURES = {
     "duo_set_decode_reproducible": (_I32, [_P, _I32]),
     "duo_set_decode_output": (_I32, [_P, _I32]),
     "duo_test_stall_next_prefill": (_I32, [_P, _I64]),
+    "duo_test_plan_decode": (_I32, [_P, _I32, ctypes.POINTER(_I32), _I32, _I32, _I32,
+                                    ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
     "duo_decode_splits": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "duo_decode_streaming_pack": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "duo_poll_device_error": (_I32, [ctypes.POINTER(_I32)]),
@@ -309,6 +311,19 @@ def duo_test_stall_next_prefill(handle, wait_ns):
     """Testing hook: the next pre-fill loads nothing and its waits give up
     after wait_ns (the timeout path, without any fault)."""
     _check(lib().duo_test_stall_next_prefill(handle, int(wait_ns)), "duo_test_stall_next_prefill")
+
+
+def duo_test_plan_decode(handle, layer, lens, num_sms, ctas_per_sm=1):
+    """Testing hook: the tensor-core decode's plan for one launch of rows with
+    these lengths (query included) on num_sms SMs, computed on the host.
+    Returns (splits per row, streaming heads per streaming CTA)."""
+    n = len(lens)
+    arr = (_I32 * max(n, 1))(*[int(x) for x in lens])
+    out = (_I32 * max(n, 1))()
+    pack = _I32()
+    _check(lib().duo_test_plan_decode(handle, layer, arr, n, num_sms, ctas_per_sm, out,
+                                      ctypes.byref(pack)), "duo_test_plan_decode")
+    return list(out)[:n], pack.value
 
 
 def duo_set_decode_output(handle, dtype):

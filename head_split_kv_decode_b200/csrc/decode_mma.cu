@@ -1098,6 +1098,10 @@ bool decode_mma_supported(int kv_type, int D, int G) {
 // Both the bf16 and the 4-bit tensor-core decode take the new token themselves.
 bool decode_can_fuse_append(int kv_type, int D, int G) { return decode_mma_supported(kv_type, D, G); }
 
+int decode_mma_tile_rows(int kv_type) {
+  return kv_type == kINT4 ? dm::Keys<true>::STEP : dm::Keys<false>::STEP;
+}
+
 cudaError_t decode_mma_config(int kv_type, int G, DecodeConfig *cfg) {
   DecodeParams dummy{};
   return kv_type == kINT4 ? dm::dispatch<true>(dummy, G, nullptr, cfg)

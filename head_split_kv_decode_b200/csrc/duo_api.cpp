@@ -1172,6 +1172,29 @@ duo_status duo_decode_splits(const duo_cache *c, int32_t layer, int32_t *splits)
   return DUO_OK;
 }
 
+duo_status duo_test_plan_decode(const duo_cache *c, int32_t layer, const int32_t *lens,
+                                int32_t n_rows, int32_t num_sms, int32_t ctas_per_sm, int32_t *splits,
+                                int32_t *pack) {
+  if (!c || !lens || !splits || !pack || layer < 0 || layer >= c->desc.layers || n_rows <= 0 ||
+      n_rows > duo::kMaxLaunchRows || num_sms <= 0 || ctas_per_sm <= 0)
+    return DUO_ERR_ARG;
+  if (!mma_path(c)) return DUO_ERR_UNSUPPORTED;
+  duo::DecodeConfig cfg{};
+  cfg.num_sms = num_sms;
+  cfg.ctas_per_sm = ctas_per_sm;
+  cfg.tile_rows = duo::decode_mma_tile_rows(c->desc.kv_dtype == DUO_INT4 ? duo::kINT4 : duo::kBF16);
+  int32_t len[duo::kMaxLaunchRows], rlen[duo::kMaxLaunchRows];
+  int16_t ns[duo::kMaxLaunchRows];
+  for (int r = 0; r < n_rows; ++r) {
+    if (lens[r] < 1) return DUO_ERR_ARG;
+    len[r] = lens[r];
+    rlen[r] = (int32_t)ret_len(c, lens[r]);
+  }
+  *pack = plan_launch(c, layer, rlen, len, n_rows, cfg, ns);
+  for (int r = 0; r < n_rows; ++r) splits[r] = ns[r];
+  return DUO_OK;
+}
+
 duo_status duo_decode_streaming_pack(const duo_cache *c, int32_t layer, int32_t *heads_per_cta) {
   if (!c || !heads_per_cta || layer < 0 || layer >= c->desc.layers) return DUO_ERR_ARG;
   if (!mma_path(c)) {

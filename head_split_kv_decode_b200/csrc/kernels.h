@@ -189,6 +189,9 @@ bool decode_can_fuse_append(int kv_type, int D, int G);
 // DecodeParams.rows (any launch rows, each at its own length) and the paged
 // layout; the CUDA-core decode takes every batch row at one length, packed.
 bool decode_mma_supported(int kv_type, int D, int G);
+// Keys a CTA of the tensor-core decode walks per iteration (16 warps x one
+// tile each); host-only, no device needed.
+int decode_mma_tile_rows(int kv_type);
 cudaError_t launch_prefill(const PrefillParams &p, cudaStream_t s);
 cudaError_t launch_table_writes(int32_t *table, const TableWrites &w, cudaStream_t s);
 cudaError_t launch_dequant_history(const DequantParams &d, cudaStream_t s);

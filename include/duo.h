@@ -442,6 +442,21 @@ duo_status duo_decode_streaming_pack(const duo_cache *cache, int32_t layer,
  * runs normally.  Errors: DUO_ERR_ARG. */
 duo_status duo_test_stall_next_prefill(duo_cache *cache, int64_t wait_ns);
 
+/* Testing hook for the tensor-core decode's launch planner (a scheduling
+ * choice; the pages have no counterpart), host only: no device is touched.
+ * For one launch of n_rows rows (1 .. DUO_MAX_LAUNCH_ROWS) of this layer
+ * whose lengths, the query included, are lens[r] >= 1, on a device of
+ * num_sms SMs taking ctas_per_sm decode CTAs each, writes each row's split
+ * count per retrieval head to splits[r] and the streaming heads per
+ * streaming CTA to *pack: the plan duo_decode_attn_rows would launch with
+ * those lengths (duo_set_decode_splits applies).  Errors: DUO_ERR_ARG;
+ * DUO_ERR_UNSUPPORTED for a configuration without the tensor-core decode
+ * (fp32 caches, head_dim 64). */
+duo_status duo_test_plan_decode(const duo_cache *cache, int32_t layer,
+                                const int32_t *lens, int32_t n_rows,
+                                int32_t num_sms, int32_t ctas_per_sm,
+                                int32_t *splits, int32_t *pack);
+
 /* Read and clear the device-side error word that bounded in-kernel waits set
  * when they give up.  Synchronises the device.  Returns DUO_ERR_TIMEOUT if it
  * was set, DUO_OK otherwise; *code (may be NULL) receives the raw word.
