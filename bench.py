@@ -161,10 +161,10 @@ DECODE_TRAFFIC_SOURCES = ("decode_mma.cu", "decode_finish.cuh", "common.cuh", "k
                           "quant_int4.cuh")
 DECODE_TRAFFIC = {
     # fused step, Llama-3-8B-shaped GQA, 128K, batch 1, one layer
-    "bf16": {"sha256": "009c3eca859ffb4f7d0e37a551ccf9b18e05bc32ba34435c04ffe4ac2c7f0ab2",
+    "bf16": {"sha256": "72fc0ba15249c58de89e634ce90f414aba1fb1a82678080280855fd71d386b41",
              "dram_bytes": 269190144 + 3686656, "algorithmic_bytes": 269120512},
     # 4-bit fused step, Llama-3-8B-shaped GQA, 1M, batch 1, one layer
-    "int4": {"sha256": "009c3eca859ffb4f7d0e37a551ccf9b18e05bc32ba34435c04ffe4ac2c7f0ab2",
+    "int4": {"sha256": "72fc0ba15249c58de89e634ce90f414aba1fb1a82678080280855fd71d386b41",
              "dram_bytes": 285927680 + 3641088, "algorithmic_bytes": 285495496},
 }
 

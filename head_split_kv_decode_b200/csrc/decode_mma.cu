@@ -2,9 +2,10 @@
 // (mma.sync m16n8k16, fp32 accumulate), for head_dim 128 and a bf16 or 4-bit
 // KV cache.
 //
-// Same work split as the CUDA-core decode (split-K over retrieval pages, one
-// CTA per streaming slot buffer, last split merges); what changes is the inner
-// product.  Per warp and per 16 keys:
+// Work split: split-K over retrieval pages (the last split of a head merges
+// the partials), streaming slot buffers one per CTA or several per CTA on
+// groups of warps (DecodeParams::str_pack); what changes against the
+// CUDA-core decode is the inner product.  Per warp and per 16 keys:
 //   S[16 x 8]  = Q[16 x 128] . K^T      two key tiles of 8, 8 k-steps each
 //   O[16 x 8] += P[16 x 16] . V         one per 8-channel output tile (16)
 // Rows 0..G-1 of the 16-row operands are the G query heads sharing the KV head
@@ -15,8 +16,10 @@
 // B fragment of K is one contiguous 16-byte load of its key row (the query
 // fragment follows the same order), and output channels are assigned so that
 // a thread's V operand comes from 32 contiguous bytes per key.  K and V are
-// loaded straight from global memory into registers; nothing is staged in
-// shared memory except the final cross-warp combine.
+// loaded straight from global memory into registers (each warp's next tile
+// is prefetched into L2 meanwhile); shared memory holds only the query
+// fragments (reloaded per tile rather than held in registers) and the final
+// cross-warp combine.
 //
 // 4-bit cache (f16 operands): a nibble masked into the low bits of a 16-bit
 // half, all other bits zero, is the f16 subnormal u * 2^-24 exactly, and one
