@@ -6,8 +6,9 @@ warps each, and gives the SMs this frees to retrieval splits.  Each case
 checks that packing was chosen and compares the CUDA path with the fp64
 oracle: MHA (one query per KV head), a pack whose last CTA has fewer heads
 than groups, the fused step (new token written and attended by the head's
-group) with float32 output, rows of different lengths, and sequence shards
-(partial outputs, the streaming heads on one shard only).
+group) with float32 output, rows of different lengths (packed and paged
+layouts), sequence shards (partial outputs, the streaming heads on one shard
+only), and the 4-bit cache.
 """
 
 import pytest
@@ -170,4 +171,47 @@ def test_packed_int4_decode_and_step():
         ref = OA.decode_reference(f64(q), Kh[:, :t + 1], Vh[:, :t + 1], mask.numpy(), S, R)
         assert_parity(out, ref, "int4", "packed 4-bit step at %d" % t)
     check_int4_bytes(cache, Kc, Ks, Kz, Vc, Vs, Vz, mask, B_, n, Hkv, S, R)
+    assert duo_poll_device_error() == 0
+
+
+def test_packed_paged_rows_and_steps():
+    """Paged layout: four rows of 40000, 25000, 9000 and 500 tokens in one
+    launch with the streaming heads packed; decode_rows, then two fused steps
+    on every row (each at its own position), against the oracle per row."""
+    Hq, Hkv, S, R = 32, 8, 4, 60
+    mask = _mask(Hkv, (1, 6))
+    lens = [40000, 25000, 9000, 500]
+    steps = 2
+    blocks = sum((n + steps + 255) // 256 for n in lens) + 8
+    cache = DuoCache(1, 4, Hq, Hkv, D, "bf16", max(lens) + steps, mask[None], S, R, pool_blocks=blocks)
+    top = max(lens) + steps
+    K, V = _seq(81, 4, top, Hkv), _seq(82, 4, top, Hkv)
+    Q = _seq(83, 4, top, Hq)
+    for r, n in enumerate(lens):
+        for p0 in range(0, n, 8192):
+            p1 = min(n, p0 + 8192)
+            cache.append_rows(0, [r], K[r:r + 1, p0:p1].contiguous(), V[r:r + 1, p0:p1].contiguous())
+    assert cache.decode_streaming_pack(0) > 1
+    rows = [2, 0, 3, 1]  # listed out of order
+    q = torch.cat([Q[r:r + 1, lens[r] - 1] for r in rows]).contiguous()
+    out = cache.decode_rows(0, rows, q)
+    torch.cuda.synchronize()
+    for i, r in enumerate(rows):
+        n = lens[r]
+        ref = OA.decode_reference(f64(q[i:i + 1]), f64(K[r:r + 1, :n]), f64(V[r:r + 1, :n]),
+                                  mask.numpy(), S, R)
+        assert_parity(out[i:i + 1], ref, "bf16", "paged row %d (%d tokens)" % (r, n))
+    rows = [0, 1, 2, 3]
+    for s_ in range(steps):
+        pos = [lens[r] + s_ for r in rows]
+        q = torch.cat([Q[r:r + 1, pos[r]] for r in rows]).contiguous()
+        kn = torch.cat([K[r:r + 1, pos[r]] for r in rows]).contiguous()
+        vn = torch.cat([V[r:r + 1, pos[r]] for r in rows]).contiguous()
+        out = cache.step_rows(0, rows, q, kn, vn)
+        torch.cuda.synchronize()
+        for r in rows:
+            t = pos[r] + 1
+            ref = OA.decode_reference(f64(q[r:r + 1]), f64(K[r:r + 1, :t]), f64(V[r:r + 1, :t]),
+                                      mask.numpy(), S, R)
+            assert_parity(out[r:r + 1], ref, "bf16", "paged step %d row %d" % (s_, r))
     assert duo_poll_device_error() == 0
